@@ -1,0 +1,219 @@
+// append.cuh -- k_quant_pack: key transform, INT2 quantization and packing of
+// new K/V rows into the paged cache (the cache-write side of Dual-QK: "Paired
+// transforms instead of shared rotation" -- partial key whitening, channel-0
+// protection; "Throughput on SGLang" -- 2 bits per stored value).
+#pragma once
+
+#include "common.cuh"
+
+namespace dqk {
+
+template <int D>
+struct AppendSmem {
+    static constexpr int NG = D / kGroup;
+    static constexpr int kMaxBlockBytes = 8 * D + 128 * NG + 64;
+    float tk[D * (D + 1)];           // T_K[j], rows padded by one float (bank-conflict free)
+    float x[kPage][D];               // one input row per warp
+    uint8_t kcode[kPage][D];         // plain codes of the page being rewritten
+    uint8_t vcode[kPage][D];
+    uint16_t kscale[kPage][NG], kmin[kPage][NG], kch0[kPage];
+    uint16_t vscale[kPage][NG], vmin[kPage][NG], vch0[kPage];
+    uint4 blk[kMaxBlockBytes / 16];  // the packed block
+};
+
+// Quantize the D values a warp holds (lane owns channels lane + 32*m, i.e.
+// channel `lane` of group m) into codes / fp16 scale / fp16 min / BF16 ch0.
+// protect: channel 0 goes to BF16, is excluded from group 0's range and its
+// code is 0.  Group min/max of the fp32 values by warp shuffles (with -0
+// read as +0), then fp64 arithmetic with single RNE roundings.
+template <int NG>
+__device__ __forceinline__ void quantize_warp(const float (&vals)[NG], bool protect, int lane,
+                                              uint8_t *codes, uint16_t *scale, uint16_t *minv,
+                                              uint16_t *ch0) {
+#pragma unroll
+    for (int m = 0; m < NG; ++m) {
+        const float x = vals[m] + 0.0f;
+        const bool excluded = protect && m == 0 && lane == 0;
+        float lo = excluded ? __int_as_float(0x7f800000) : x;
+        float hi = excluded ? __int_as_float(0xff800000) : x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        const uint16_t sh = f64_to_f16_rne(((double)hi - (double)lo) / 3.0);
+        const uint16_t mh = f64_to_f16_rne((double)lo);
+        const double s = f16_to_f64(sh), mn = f16_to_f64(mh);
+        int code = 0;
+        if (!excluded && s != 0.0) {
+            const double r = rint(((double)x - mn) / s);
+            code = r < 0.0 ? 0 : (r > 3.0 ? 3 : (int)r);
+        }
+        codes[m * kGroup + lane] = (uint8_t)code;
+        if (lane == 0) {
+            scale[m] = sh;
+            minv[m] = mh;
+        }
+    }
+    if (lane == 0) *ch0 = protect ? f32_to_bf16_rne(vals[0]) : (uint16_t)0;
+}
+
+__device__ __forceinline__ float load_elem(const void *p, int dtype, size_t idx) {
+    if (dtype == DQK_BF16) return bf16_to_f32(reinterpret_cast<const uint16_t *>(p)[idx]);
+    return reinterpret_cast<const float *>(p)[idx];
+}
+
+// Block <-> plain arrays.  One thread per 32-bit code word.
+template <int D>
+__device__ void unpack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
+    constexpr int NG = D / kGroup;
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(S.blk);
+    for (int idx = threadIdx.x; idx < 2 * 32 * NG; idx += blockDim.x) {
+        const bool is_v = idx >= 32 * NG;
+        const int widx = is_v ? idx - 32 * NG : idx;
+        const int lane = widx / NG, W = widx % NG, gid = lane >> 2, tig = lane & 3;
+        const uint32_t word = w[((is_v ? L.vc : L.kc) >> 2) + widx];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int q = W * 8 + i;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const uint8_t code = (uint8_t)((word >> (16 * e + 2 * i)) & 3u);
+                if (!is_v) {
+                    const int tr = q & 1, cb = (q >> 1) & 1, s = (q >> 2) & 1, g = q >> 3;
+                    S.kcode[gid + 8 * tr][32 * g + 16 * s + 8 * cb + 2 * tig + e] = code;
+                } else {
+                    const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
+                    S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid] = code;
+                }
+            }
+        }
+    }
+    const uint16_t *h = reinterpret_cast<const uint16_t *>(S.blk);
+    for (int idx = threadIdx.x; idx < kPage * NG; idx += blockDim.x) {
+        const int t = idx / NG, g = idx % NG;
+        S.kscale[t][g] = h[(L.ks >> 1) + kscale_idx(NG, t, g)];
+        S.kmin[t][g] = h[(L.km >> 1) + kscale_idx(NG, t, g)];
+        S.vscale[t][g] = h[(L.vs >> 1) + vscale_idx(NG, t, g)];
+        S.vmin[t][g] = h[(L.vm >> 1) + vscale_idx(NG, t, g)];
+    }
+    for (int t = threadIdx.x; t < kPage; t += blockDim.x) {
+        S.kch0[t] = h[(L.k0 >> 1) + k0_idx(t)];
+        S.vch0[t] = v_ch0 ? h[(L.v0 >> 1) + t] : (uint16_t)0;
+    }
+}
+
+template <int D>
+__device__ void pack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
+    constexpr int NG = D / kGroup;
+    uint32_t *w = reinterpret_cast<uint32_t *>(S.blk);
+    for (int idx = threadIdx.x; idx < 2 * 32 * NG; idx += blockDim.x) {
+        const bool is_v = idx >= 32 * NG;
+        const int widx = is_v ? idx - 32 * NG : idx;
+        const int lane = widx / NG, W = widx % NG, gid = lane >> 2, tig = lane & 3;
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int q = W * 8 + i;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                uint32_t code;
+                if (!is_v) {
+                    const int tr = q & 1, cb = (q >> 1) & 1, s = (q >> 2) & 1, g = q >> 3;
+                    code = S.kcode[gid + 8 * tr][32 * g + 16 * s + 8 * cb + 2 * tig + e];
+                } else {
+                    const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
+                    code = S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid];
+                }
+                word |= (code & 3u) << (16 * e + 2 * i);
+            }
+        }
+        w[((is_v ? L.vc : L.kc) >> 2) + widx] = word;
+    }
+    uint16_t *h = reinterpret_cast<uint16_t *>(S.blk);
+    for (int idx = threadIdx.x; idx < kPage * NG; idx += blockDim.x) {
+        const int t = idx / NG, g = idx % NG;
+        h[(L.ks >> 1) + kscale_idx(NG, t, g)] = S.kscale[t][g];
+        h[(L.km >> 1) + kscale_idx(NG, t, g)] = S.kmin[t][g];
+        h[(L.vs >> 1) + vscale_idx(NG, t, g)] = S.vscale[t][g];
+        h[(L.vm >> 1) + vscale_idx(NG, t, g)] = S.vmin[t][g];
+    }
+    for (int t = threadIdx.x; t < kPage; t += blockDim.x) {
+        h[(L.k0 >> 1) + k0_idx(t)] = S.kch0[t];
+        if (v_ch0) h[(L.v0 >> 1) + t] = S.vch0[t];
+    }
+}
+
+// Grid: x = work items (sequence, touched page) strided, y = kv head.
+// Block: 16 warps, warp w owns token slot w of the page being rewritten.
+// Each item: read the old block, overwrite the appended slots, write back
+// with 128-bit stores.  T_K[j] is staged once per CTA.
+template <int D>
+__global__ void __launch_bounds__(512) k_quant_pack(
+    const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin,
+    int dtype, int batch, const int *__restrict__ new_lens, const int *__restrict__ seq_before,
+    const int *__restrict__ page_table, int max_pages, int slots_per_seq, uint8_t *__restrict__ pool,
+    long long num_pages, int hkv, int v_ch0) {
+    constexpr int NG = D / kGroup;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    AppendSmem<D> &S = *reinterpret_cast<AppendSmem<D> *>(smem_raw);
+    const int j = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Layout L = make_layout(D, v_ch0);
+
+    const float *T = t_k + (size_t)j * D * D;
+    for (int idx = threadIdx.x; idx < D * D; idx += blockDim.x)
+        S.tk[(idx / D) * (D + 1) + (idx % D)] = T[idx];
+    __syncthreads();
+
+    const int items = batch * slots_per_seq;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const int b = item / slots_per_seq, slot = item % slots_per_seq;
+        const int n = new_lens[b], L0 = seq_before[b];
+        if (n <= 0) continue;
+        const int page = L0 / kPage + slot;
+        if (page > (L0 + n - 1) / kPage) continue;
+        const int phys = (L0 >= 0 && page < max_pages) ? page_table[(size_t)b * max_pages + page] : -1;
+        if (phys < 0 || phys >= num_pages) {
+            if (threadIdx.x == 0) dqk_flag_error(kErrBounds);
+            continue;
+        }
+        long long row0 = 0;
+        for (int bb = 0; bb < b; ++bb) row0 += new_lens[bb];
+        uint4 *blk_g = reinterpret_cast<uint4 *>(pool + ((size_t)phys * hkv + j) * L.bytes);
+
+        for (int o = threadIdx.x; o < L.bytes / 16; o += blockDim.x) S.blk[o] = blk_g[o];
+        __syncthreads();
+        unpack_block<D>(S, L, v_ch0);
+        __syncthreads();
+
+        const int pos = page * kPage + warp;
+        if (pos >= L0 && pos < L0 + n) {
+            const size_t base = ((size_t)(row0 + (pos - L0)) * hkv + j) * D;
+#pragma unroll
+            for (int m = 0; m < NG; ++m) S.x[warp][lane + 32 * m] = load_elem(kin, dtype, base + lane + 32 * m);
+            __syncwarp();
+            float kp[NG];
+#pragma unroll
+            for (int m = 0; m < NG; ++m) {
+                const float *row = &S.tk[(lane + 32 * m) * (D + 1)];
+                double s = 0.0;
+#pragma unroll 8
+                for (int i = 0; i < D; ++i) s = fma((double)row[i], (double)S.x[warp][i], s);
+                kp[m] = __double2float_rn(s);
+            }
+            quantize_warp<NG>(kp, true, lane, S.kcode[warp], S.kscale[warp], S.kmin[warp], &S.kch0[warp]);
+            float vv[NG];
+#pragma unroll
+            for (int m = 0; m < NG; ++m) vv[m] = load_elem(vin, dtype, base + lane + 32 * m);
+            quantize_warp<NG>(vv, v_ch0 != 0, lane, S.vcode[warp], S.vscale[warp], S.vmin[warp], &S.vch0[warp]);
+        }
+        __syncthreads();
+        pack_block<D>(S, L, v_ch0);
+        __syncthreads();
+        for (int o = threadIdx.x; o < L.bytes / 16; o += blockDim.x) blk_g[o] = S.blk[o];
+        __syncthreads();
+    }
+}
+
+}  // namespace dqk

@@ -1,0 +1,248 @@
+// dualqk.cu -- libdualqk: host side of the C ABI declared in include/dualqk.h
+// (argument checks, launch planning) and the single translation unit that
+// holds every kernel of the decode hot path.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "append.cuh"
+#include "attend_simple.cuh"
+#include "qprep.cuh"
+
+namespace {
+
+using namespace dqk;
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+dqk_status check_layer(const dqk_layer_desc *L) {
+    if (!L) return DQK_ERR_INVALID_ARG;
+    if (L->head_dim != 64 && L->head_dim != 128) return DQK_ERR_UNSUPPORTED;
+    if (L->num_kv_heads <= 0 || L->num_q_heads <= 0 || L->num_q_heads % L->num_kv_heads)
+        return DQK_ERR_INVALID_ARG;
+    const int G = L->num_q_heads / L->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return DQK_ERR_UNSUPPORTED;
+    if (L->page_size != kPage || L->group_size != kGroup) return DQK_ERR_UNSUPPORTED;
+    if (L->v_ch0_protect != 0 && L->v_ch0_protect != 1) return DQK_ERR_INVALID_ARG;
+    if (!L->pool || !aligned(L->pool, 16) || L->num_pages <= 0) return DQK_ERR_INVALID_ARG;
+    return DQK_OK;
+}
+
+// Workspace layout of the decode: [qsel | part_o | part_ml], 256-B aligned.
+struct DecodePlan {
+    int d, G, ns, tokens_per_split;
+    size_t off_qsel, off_o, off_ml, bytes;
+};
+
+DecodePlan plan_decode(const dqk_layer_desc *L, int batch, int max_pages) {
+    DecodePlan P;
+    P.d = L->head_dim;
+    P.G = L->num_q_heads / L->num_kv_heads;
+    P.ns = (max_pages + kSimplePagesPerSplit - 1) / kSimplePagesPerSplit;
+    P.tokens_per_split = kSimplePagesPerSplit * kPage;
+    const size_t rows = (size_t)batch * L->num_q_heads;
+    P.off_qsel = 256;
+    P.off_o = round_up(P.off_qsel + rows * P.d * sizeof(float), 256);
+    P.off_ml = round_up(P.off_o + rows * P.ns * P.d * sizeof(float), 256);
+    P.bytes = round_up(P.off_ml + rows * P.ns * 2 * sizeof(float), 256);
+    return P;
+}
+
+dqk_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? DQK_OK : DQK_ERR_CUDA;
+}
+
+struct DecodeArgs {
+    const dqk_layer_desc *L;
+    const void *q;
+    dqk_dtype q_dtype;
+    int batch;
+    const int *seq_lens, *page_table;
+    int max_pages, pct;
+    float *out;
+    int16_t *sel_out;
+    void *ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+dqk_status check_decode(const DecodeArgs &a, DecodePlan &P) {
+    dqk_status st = check_layer(a.L);
+    if (st != DQK_OK) return st;
+    if (!a.L->t_q || !a.q || !a.seq_lens || !a.page_table || !a.out || !a.ws) return DQK_ERR_INVALID_ARG;
+    if (a.q_dtype != DQK_F32 && a.q_dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
+    if (a.batch <= 0 || a.max_pages <= 0 || a.pct < 0 || a.pct > 99) return DQK_ERR_INVALID_ARG;
+    if (!aligned(a.ws, 256) || !aligned(a.out, 16)) return DQK_ERR_INVALID_ARG;
+    P = plan_decode(a.L, a.batch, a.max_pages);
+    if (a.ws_bytes < P.bytes) return DQK_ERR_WORKSPACE_TOO_SMALL;
+    return DQK_OK;
+}
+
+template <int D>
+dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
+    const int G = P.G;
+    const size_t smem = (size_t)D * (D + 1) * 4 + (size_t)G * D * 4 + (size_t)G * D;
+    if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return DQK_ERR_CUDA;
+    float *qsel = reinterpret_cast<float *>(static_cast<char *>(a.ws) + P.off_qsel);
+    const int threads = (G < 4 ? 4 : G) * 32;
+    k_qprep<D><<<dim3(a.L->num_kv_heads, a.batch), threads, smem, a.stream>>>(
+        a.L->t_q, a.q, a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qsel, a.sel_out);
+    return launch_status();
+}
+
+template <int D, int G>
+dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
+    char *ws = static_cast<char *>(a.ws);
+    k_attend_simple<D, G><<<dim3(P.ns, a.L->num_kv_heads, a.batch), kSimpleThreads, 0, a.stream>>>(
+        static_cast<const uint8_t *>(a.L->pool), a.L->num_kv_heads, a.L->v_ch0_protect, a.L->num_pages,
+        a.seq_lens, a.page_table, a.max_pages, reinterpret_cast<const float *>(ws + P.off_qsel), P.ns,
+        reinterpret_cast<float *>(ws + P.off_o), reinterpret_cast<float *>(ws + P.off_ml));
+    return launch_status();
+}
+
+template <int D>
+dqk_status run_attend(const DecodeArgs &a, const DecodePlan &P) {
+    switch (P.G) {
+        case 1: return run_attend_g<D, 1>(a, P);
+        case 2: return run_attend_g<D, 2>(a, P);
+        case 4: return run_attend_g<D, 4>(a, P);
+        default: return run_attend_g<D, 8>(a, P);
+    }
+}
+
+template <int D>
+dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
+    char *ws = static_cast<char *>(a.ws);
+    k_combine_simple<D><<<dim3(a.L->num_q_heads, a.batch), D, 0, a.stream>>>(
+        a.seq_lens, a.L->num_q_heads, P.ns, P.tokens_per_split, reinterpret_cast<const float *>(ws + P.off_o),
+        reinterpret_cast<const float *>(ws + P.off_ml), a.out);
+    return launch_status();
+}
+
+enum Stage { kPrepare = 1, kAttend = 2, kCombine = 4 };
+
+dqk_status decode_stages(const DecodeArgs &a, int stages) {
+    DecodePlan P;
+    dqk_status st = check_decode(a, P);
+    if (st != DQK_OK) return st;
+    const bool d128 = a.L->head_dim == 128;
+    if (stages & kPrepare) {
+        st = d128 ? run_prepare<128>(a, P) : run_prepare<64>(a, P);
+        if (st != DQK_OK) return st;
+    }
+    if (stages & kAttend) {
+        st = d128 ? run_attend<128>(a, P) : run_attend<64>(a, P);
+        if (st != DQK_OK) return st;
+    }
+    if (stages & kCombine) {
+        st = d128 ? run_combine<128>(a, P) : run_combine<64>(a, P);
+        if (st != DQK_OK) return st;
+    }
+    return DQK_OK;
+}
+
+template <int D>
+dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk_dtype dtype, int batch,
+                      const int *new_lens, const int *seq_before, int max_new, const int *page_table,
+                      int max_pages, cudaStream_t stream) {
+    const size_t smem = sizeof(AppendSmem<D>);
+    if (cudaFuncSetAttribute(k_quant_pack<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return DQK_ERR_CUDA;
+    const int slots = (max_new + kPage - 1) / kPage + 1;
+    const long long items = (long long)batch * slots;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long long gx = (2LL * sms + L->num_kv_heads - 1) / L->num_kv_heads;
+    if (gx > items) gx = items;
+    if (gx < 1) gx = 1;
+    k_quant_pack<D><<<dim3((unsigned)gx, L->num_kv_heads), 512, smem, stream>>>(
+        L->t_k, k, v, dtype, batch, new_lens, seq_before, page_table, max_pages, slots,
+        static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dqk_block_bytes(const dqk_layer_desc *layer) {
+    if (!layer || (layer->head_dim != 64 && layer->head_dim != 128)) return 0;
+    if (layer->v_ch0_protect != 0 && layer->v_ch0_protect != 1) return 0;
+    return (size_t)make_layout(layer->head_dim, layer->v_ch0_protect).bytes;
+}
+
+dqk_status dqk_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
+                      const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
+                      int max_pages, dqk_stream_t stream) {
+    dqk_status st = check_layer(layer);
+    if (st != DQK_OK) return st;
+    if (!layer->t_k || !k || !v || !new_lens || !seq_lens_before || !page_table) return DQK_ERR_INVALID_ARG;
+    if (dtype != DQK_F32 && dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
+    if (batch <= 0 || max_pages <= 0 || max_new < 0) return DQK_ERR_INVALID_ARG;
+    if (!aligned(k, 4) || !aligned(v, 4)) return DQK_ERR_INVALID_ARG;
+    if (max_new == 0) return DQK_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return layer->head_dim == 128
+               ? run_append<128>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages, s)
+               : run_append<64>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages, s);
+}
+
+size_t dqk_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max_pages) {
+    if (check_layer(layer) != DQK_OK || batch <= 0 || max_pages <= 0) return 0;
+    return plan_decode(layer, batch, max_pages).bytes;
+}
+
+#define DQK_DECODE_ARGS                                                                                   \
+    const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype, int batch, const int *seq_lens,        \
+        const int *page_table, int max_pages, int sparsity_pct, float *out, int16_t *sel_out, void *workspace, \
+        size_t workspace_bytes, dqk_stream_t stream
+#define DQK_DECODE_PACK                                                                                   \
+    DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out, sel_out,   \
+                 workspace, workspace_bytes, static_cast<cudaStream_t>(stream)}
+
+dqk_status dqk_decode(DQK_DECODE_ARGS) {
+    DQK_DECODE_PACK;
+    return decode_stages(a, kPrepare | kAttend | kCombine);
+}
+dqk_status dqk_decode_prepare(DQK_DECODE_ARGS) {
+    DQK_DECODE_PACK;
+    return decode_stages(a, kPrepare);
+}
+dqk_status dqk_decode_attend(DQK_DECODE_ARGS) {
+    DQK_DECODE_PACK;
+    return decode_stages(a, kAttend);
+}
+dqk_status dqk_decode_combine(DQK_DECODE_ARGS) {
+    DQK_DECODE_PACK;
+    return decode_stages(a, kCombine);
+}
+
+dqk_status dqk_last_device_error(dqk_stream_t stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DQK_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_dqk_device_error, sizeof(word)) != cudaSuccess) return DQK_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(g_dqk_device_error, &zero, sizeof(zero)) != cudaSuccess) return DQK_ERR_CUDA;
+    if (word & kErrBounds) return DQK_ERR_DEVICE_BOUNDS;
+    if (word & kErrTimeout) return DQK_ERR_TIMEOUT;
+    return DQK_OK;
+}
+
+const char *dqk_status_string(dqk_status s) {
+    switch (s) {
+        case DQK_OK: return "DQK_OK";
+        case DQK_ERR_INVALID_ARG: return "DQK_ERR_INVALID_ARG";
+        case DQK_ERR_UNSUPPORTED: return "DQK_ERR_UNSUPPORTED";
+        case DQK_ERR_WORKSPACE_TOO_SMALL: return "DQK_ERR_WORKSPACE_TOO_SMALL";
+        case DQK_ERR_CUDA: return "DQK_ERR_CUDA";
+        case DQK_ERR_DEVICE_BOUNDS: return "DQK_ERR_DEVICE_BOUNDS";
+        case DQK_ERR_TIMEOUT: return "DQK_ERR_TIMEOUT";
+    }
+    return "DQK_UNKNOWN_STATUS";
+}
+
+}  // extern "C"

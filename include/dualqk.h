@@ -1,0 +1,197 @@
+/*
+ * dualqk.h -- C ABI of libdualqk, the B200 (sm_100a) decode hot path of
+ * Dual-QK: paired key/query transforms, INT2 KV cache with BF16 key channel 0,
+ * and query-channel-pruned attention over a paged cache.
+ *
+ * What the method is (page titles and sections):
+ *  - "How does Dual-QK compress KV caches to 2-bit while keeping accuracy at
+ *    128K context?", section "Paired transforms instead of shared rotation":
+ *    a non-orthogonal key transform T_K (partial key whitening) flattens keys
+ *    for INT2 storage, a paired query transform T_Q (query-aligned basis)
+ *    sharpens queries for channel pruning, channel 0 is protected.
+ *  - same page, section "Why the cache becomes a bottleneck": the pair must
+ *    preserve query-key dot products, so T_Q = T_K^{-T} and (T_Q q).(T_K k)
+ *    = q.k; query-channel pruning reduces key-cache reads.
+ *  - same page, section "Throughput on SGLang": 2 bits per stored value and
+ *    40 % of key channels removed from reads.
+ *  - "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches",
+ *    abstract: INT2 K/V, channel-0 protection, 40 % query-channel sparsity.
+ * Details the pages leave open are fixed as follows: asymmetric INT2 per token
+ * in groups of 32 channels with fp16 scale and min, codes rounded half to even,
+ * top-k ties broken toward the lower channel index, RoPE applied by the caller
+ * before T_K, key channel 0 in BF16 (value channel 0 optionally).
+ *
+ * Conventions for every call:
+ *  - Ownership: the caller allocates and owns every buffer (pool, page tables,
+ *    q/k/v, out, workspace).  The library allocates nothing and keeps no state
+ *    besides one device error word per device (see dqk_last_device_error).
+ *  - Pointers marked (device) must be device memory of the current device;
+ *    (host) means host memory.  All work is enqueued on `stream` (a
+ *    cudaStream_t value, NULL for the legacy default stream); no call
+ *    synchronizes except dqk_last_device_error.
+ *  - Errors: every call returns a dqk_status.  Invalid arguments are rejected
+ *    before anything is launched.  A failed launch returns DQK_ERR_CUDA.
+ *    Out-of-range page ids or lengths found on the device do not fault: the
+ *    kernel skips the access and sets the device error word.
+ */
+#ifndef DUALQK_H
+#define DUALQK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *dqk_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    DQK_OK = 0,
+    DQK_ERR_INVALID_ARG = 1,         /* null pointer, bad size, bad layer descriptor */
+    DQK_ERR_UNSUPPORTED = 2,         /* head_dim, group ratio or page size not built */
+    DQK_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < dqk_decode_workspace_size */
+    DQK_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+    DQK_ERR_DEVICE_BOUNDS = 5,       /* device saw a page id / length out of range */
+    DQK_ERR_TIMEOUT = 6              /* a bounded device wait gave up */
+} dqk_status;
+
+typedef enum { DQK_F32 = 0, DQK_BF16 = 1 } dqk_dtype;
+
+/* One attention layer's cache description.
+ *  head_dim       64 or 128 (d).
+ *  num_q_heads    Hq; num_kv_heads Hkv; Hq % Hkv == 0 and G = Hq/Hkv in
+ *                 {1, 2, 4, 8}.  Query head h reads kv head h / G.
+ *  page_size      must be 16 tokens.
+ *  group_size     must be 32 channels.
+ *  v_ch0_protect  0: value channel 0 quantized like the others (default);
+ *                 1: value channel 0 kept in BF16 as well.
+ *  t_k, t_q       (device) fp32 [Hkv][d][d] row-major: k' = T_K k,
+ *                 q' = T_Q q.  The caller supplies T_Q = T_K^{-T}.
+ *  pool           (device) the paged cache: num_pages * Hkv blocks of
+ *                 dqk_block_bytes() bytes, block (page p, kv head j) at byte
+ *                 offset (p * Hkv + j) * dqk_block_bytes().  16-byte aligned.
+ */
+typedef struct {
+    int head_dim;
+    int num_q_heads;
+    int num_kv_heads;
+    int page_size;
+    int group_size;
+    int v_ch0_protect;
+    const float *t_k;
+    const float *t_q;
+    void *pool;
+    long long num_pages;
+} dqk_layer_desc;
+
+/* Bytes of one (page, kv head) block: 16 tokens of INT2 codes, fp16
+ * scale/min per 32-channel group for K and V, and the BF16 channel 0.
+ * d = 128: 1568 (98 B per token and kv head), d = 64: 800 (50 B); +32 with
+ * v_ch0_protect.  Returns 0 for an unsupported descriptor.
+ *
+ * Block layout (byte offsets, NG = d/32 groups, P = 16 tokens; the code
+ * sections are in the operand order of the decode kernel's tensor-core
+ * tiles, each lane of a warp reading 4*NG contiguous bytes):
+ *   KC = 0            K codes, 4*d bytes: code of (token t, channel c) is in the
+ *                     32-bit word at KC + 4*(lane*NG + W), bit 16*e + 2*i, with
+ *                     g=c/32, s=(c%32)/16, cb=(c%16)/8, tig=(c%8)/2, e=c%2,
+ *                     lane=4*(t%8)+tig, q=((2g+s)*2+cb)*2+t/8, W=q/8, i=q%8.
+ *   KS = 4d           K scale fp16 [t][g]
+ *   KM = KS + 32*NG   K min   fp16 [t][g]
+ *   K0 = KM + 32*NG   K channel 0 BF16, token t at index 2*(t%8) + t/8
+ *   VC = K0 + 32      V codes, 4*d bytes: (t, c) is in the word at
+ *                     VC + 4*(lane*NG + W), bit 16*e + 2*i, with m=c/16,
+ *                     cr=(c%16)/8, tb=t/8, tig=(t%8)/2, e=t%2,
+ *                     lane=4*(c%8)+tig, q=(2m+cr)*2+tb, W=q/8, i=q%8.
+ *   VS = VC + 4d      V scale fp16, (t, g) at index 2*(NG*(t/2) + g) + t%2
+ *   VM = VS + 32*NG   V min fp16, same indexing
+ *   V0 = VM + 32*NG   V channel 0 BF16 [t] (only with v_ch0_protect)
+ * The code slot of a protected channel 0 holds 0.
+ */
+size_t dqk_block_bytes(const dqk_layer_desc *layer);
+
+/* dqk_append -- transform, quantize and pack new K/V rows into the cache.
+ * Passages: key transform and INT2 storage with channel-0 protection ("Paired
+ * transforms instead of shared rotation"; "Throughput on SGLang").
+ *  k, v             (device) [sum(new_lens)][Hkv][d] rows, dtype DQK_F32 or
+ *                   DQK_BF16, sequence b's rows after those of b-1; RoPE
+ *                   already applied to k.
+ *  new_lens         (device) int [batch]: rows appended to sequence b.
+ *  seq_lens_before  (device) int [batch]: tokens already cached; the rows go
+ *                   to positions seq_lens_before[b] .. +new_lens[b]-1.
+ *  max_new          (host) upper bound of new_lens[] (sizes the launch).
+ *  page_table       (device) int [batch][max_pages]: logical page -> physical
+ *                   page in the pool; entries covering the new positions must
+ *                   be valid and not shared with another sequence being
+ *                   appended in the same call.
+ * Per token and kv head: k' = fp32(fp64 sum over i ascending of
+ * T_K[c][i]*k[i]); per group g: scale = fp16((max-min)/3), min = fp16(min)
+ * (fp64 arithmetic, RNE, saturating), code = clamp(rne((x-min)/scale), 0, 3)
+ * or 0 when scale == 0; key channel 0 -> BF16, left out of group 0's range.
+ * Values: same quantizer, no transform.  Positions of the touched pages that
+ * are not appended keep their bytes.  The caller advances its lengths.
+ */
+dqk_status dqk_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype,
+                      int batch, const int *new_lens, const int *seq_lens_before, int max_new,
+                      const int *page_table, int max_pages, dqk_stream_t stream);
+
+/* Device workspace needed by dqk_decode for `batch` sequences of at most
+ * max_pages pages (query prep, split partials, counters).  0 = unsupported. */
+size_t dqk_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max_pages);
+
+/* dqk_decode -- pruned-channel attention of one decode query per head.
+ * Passages: channel pruning of the query ("Why the cache becomes a
+ * bottleneck"; "Throughput on SGLang": 40 % of key channels removed from
+ * reads), attention over the INT2 cache.
+ *  q            (device) [batch][Hq][d], DQK_F32 or DQK_BF16, RoPE applied.
+ *  seq_lens     (device) int [batch]: tokens to attend (appended ones
+ *               included); 0 gives a zero output row.
+ *  page_table   (device) int [batch][max_pages].
+ *  sparsity_pct 0..99: n_keep = d - floor(pct*d/100) channels are kept per
+ *               query head, channel 0 always, then the largest |q'_c| of
+ *               channels 1..d-1, ties to the lower index.
+ *  out          (device) fp32 [batch][Hq][d].
+ *  sel_out      (device, nullable) int16 [batch][Hq][n_keep]: the kept
+ *               channels in ascending order.
+ *  workspace    (device) >= dqk_decode_workspace_size(layer, batch,
+ *               max_pages) bytes, 256-byte aligned; contents need no
+ *               initialisation and are scratch after the call.
+ * q' = fp32(fp64 sequential T_Q q); s_t = q'_S . k^'_t / sqrt(d) over the
+ * kept channels with k^' = min + code*scale (BF16 value for channel 0);
+ * out = softmax(s) . v^.  Computed as split-K flash decoding: per split an
+ * online softmax with fp32 partials (m, l, o), then a log-sum-exp combine.
+ * Equal to dqk_decode_prepare + dqk_decode_attend + dqk_decode_combine.
+ */
+dqk_status dqk_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype, int batch,
+                      const int *seq_lens, const int *page_table, int max_pages,
+                      int sparsity_pct, float *out, int16_t *sel_out, void *workspace,
+                      size_t workspace_bytes, dqk_stream_t stream);
+
+/* The three stages of dqk_decode, exported so callers can place or time them
+ * separately.  Same arguments; each uses the ones its stage needs. */
+dqk_status dqk_decode_prepare(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
+                              int batch, const int *seq_lens, const int *page_table,
+                              int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
+                              void *workspace, size_t workspace_bytes, dqk_stream_t stream);
+dqk_status dqk_decode_attend(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
+                             int batch, const int *seq_lens, const int *page_table,
+                             int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
+                             void *workspace, size_t workspace_bytes, dqk_stream_t stream);
+dqk_status dqk_decode_combine(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
+                              int batch, const int *seq_lens, const int *page_table,
+                              int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
+                              void *workspace, size_t workspace_bytes, dqk_stream_t stream);
+
+/* Synchronizes `stream`, then reads and clears the current device's error
+ * word: DQK_OK, DQK_ERR_DEVICE_BOUNDS or DQK_ERR_TIMEOUT (DQK_ERR_CUDA if the
+ * stream itself reports an error).  All calls on a device share the word. */
+dqk_status dqk_last_device_error(dqk_stream_t stream);
+
+/* Static, human-readable name of a status. */
+const char *dqk_status_string(dqk_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DUALQK_H */

@@ -149,7 +149,7 @@ void oracle_transform_f64(int d, const double *T, const double *x, double *y)
 /* x: d fp32 values (already transformed for keys).  protect_ch0: channel 0
  * is stored in BF16, left out of group 0's min/max, and its code slot is 0.
  * Per group g (channels 32g..32g+31):
- *   mn, mx      = min / max over the group (fp32 values)
+ *   mn, mx      = min / max over the group (fp32 values; a zero is +0)
  *   scale_h     = fp16( (mx - mn) / 3 )          (fp64 arithmetic)
  *   min_h       = fp16( mn )
  *   code_c      = 0 if scale_h == 0, else clamp(rne((x_c - min_h)/scale_h), 0, 3)
@@ -164,7 +164,7 @@ void oracle_quantize_vec(int d, const float *x, int protect_ch0,
         int first = (g == 0 && protect_ch0) ? 1 : 0;
         double mn = INFINITY, mx = -INFINITY;
         for (int c = lo + first; c < hi; ++c) {
-            double v = (double)x[c];
+            double v = (double)x[c] + 0.0;      /* READING: -0 and +0 are the value 0 */
             if (v < mn) mn = v;
             if (v > mx) mx = v;
         }
