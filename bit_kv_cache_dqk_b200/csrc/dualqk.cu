@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "append.cuh"
@@ -220,6 +221,56 @@ dqk_status dqk_decode_attend(DQK_DECODE_ARGS) {
 dqk_status dqk_decode_combine(DQK_DECODE_ARGS) {
     DQK_DECODE_PACK;
     return decode_stages(a, kCombine);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// dqk_decode_noalloc: the decode for callers that cannot hand over a device
+// workspace.  Its scratch is this file-scope array in the module's static
+// device memory (one per device that loads the library).  Host code must not
+// pass the symbol itself to a kernel -- on the host it is only a stand-in --
+// so its device address is looked up with cudaGetSymbolAddress, once per
+// device, on that device's first call.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_dqk_noalloc_ws[DQK_NOALLOC_WORKSPACE_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+dqk_status noalloc_workspace(void **ws) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DQK_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return DQK_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dqk_noalloc_ws) != cudaSuccess || !p) return DQK_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ws = g_noalloc_ptr[dev];
+    return DQK_OK;
+}
+}  // namespace
+
+extern "C" {
+
+dqk_status dqk_decode_noalloc(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype, int batch,
+                              const int *seq_lens, const int *page_table, int max_pages, int sparsity_pct,
+                              float *out, int16_t *sel_out, dqk_stream_t stream) {
+    dqk_status st = check_layer(layer);
+    if (st != DQK_OK) return st;
+    if (batch <= 0 || max_pages <= 0) return DQK_ERR_INVALID_ARG;
+    if (plan_decode(layer, batch, max_pages).bytes > (size_t)DQK_NOALLOC_WORKSPACE_BYTES)
+        return DQK_ERR_WORKSPACE_TOO_SMALL;
+    void *ws = nullptr;
+    st = noalloc_workspace(&ws);
+    if (st != DQK_OK) return st;
+    DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out, sel_out,
+                 ws, (size_t)DQK_NOALLOC_WORKSPACE_BYTES, static_cast<cudaStream_t>(stream)};
+    return decode_stages(a, kPrepare | kAttend | kCombine);
 }
 
 dqk_status dqk_last_device_error(dqk_stream_t stream) {

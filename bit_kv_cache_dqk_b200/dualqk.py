@@ -25,7 +25,9 @@ DQK_F32, DQK_BF16 = 0, 1
 
 EXPORTED = ["dqk_block_bytes", "dqk_append", "dqk_decode_workspace_size", "dqk_decode",
             "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine",
-            "dqk_last_device_error", "dqk_status_string"]
+            "dqk_decode_noalloc", "dqk_last_device_error", "dqk_status_string"]
+
+DQK_NOALLOC_WORKSPACE_BYTES = 8 << 20
 
 
 class dqk_layer_desc(C.Structure):
@@ -47,6 +49,8 @@ for _n in ("dqk_decode", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_
     getattr(_lib, _n).restype = C.c_int
     getattr(_lib, _n).argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P,
                                   C.c_size_t, _P]
+_lib.dqk_decode_noalloc.restype = C.c_int
+_lib.dqk_decode_noalloc.argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P]
 _lib.dqk_last_device_error.restype = C.c_int
 _lib.dqk_last_device_error.argtypes = [_P]
 _lib.dqk_status_string.restype = C.c_char_p
@@ -135,6 +139,15 @@ def dqk_decode_combine(layer, q, q_dtype, batch, seq_lens, page_table, max_pages
     return _decode(_lib.dqk_decode_combine, "dqk_decode_combine", layer, q, q_dtype, batch, seq_lens,
                    page_table, max_pages, sparsity_pct, out, sel_out, workspace, workspace_bytes, stream,
                    raise_on_error)
+
+
+def dqk_decode_noalloc(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out,
+                       sel_out, stream=None, raise_on_error=True) -> int:
+    """dqk_decode for callers that cannot provide a workspace (the library's
+    static scratch is used; see include/dualqk.h)."""
+    st = _lib.dqk_decode_noalloc(C.byref(layer), _addr(q), q_dtype, batch, _addr(seq_lens), _addr(page_table),
+                                 max_pages, sparsity_pct, _addr(out), _addr(sel_out), _stream(stream))
+    return _check(st, "dqk_decode_noalloc", raise_on_error)
 
 
 def dqk_last_device_error(stream=None) -> int:

@@ -24,7 +24,8 @@
  * Conventions for every call:
  *  - Ownership: the caller allocates and owns every buffer (pool, page tables,
  *    q/k/v, out, workspace).  The library allocates nothing and keeps no state
- *    besides one device error word per device (see dqk_last_device_error).
+ *    besides one device error word per device (see dqk_last_device_error) and
+ *    the static scratch of dqk_decode_noalloc.
  *  - Pointers marked (device) must be device memory of the current device;
  *    (host) means host memory.  All work is enqueued on `stream` (a
  *    cudaStream_t value, NULL for the legacy default stream); no call
@@ -182,6 +183,34 @@ dqk_status dqk_decode_combine(const dqk_layer_desc *layer, const void *q, dqk_dt
                               int batch, const int *seq_lens, const int *page_table,
                               int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
                               void *workspace, size_t workspace_bytes, dqk_stream_t stream);
+
+/* Largest workspace dqk_decode_noalloc can serve: 8 MiB of static device
+ * memory per device that loads the library. */
+#define DQK_NOALLOC_WORKSPACE_BYTES (8u << 20)
+
+/* dqk_decode_noalloc -- dqk_decode without a caller-provided workspace.
+ * The paper has no counterpart: this exists for callers that cannot allocate
+ * device memory at decode time -- for example a plugin inside a host engine
+ * whose op interface offers no scratch buffer, or a serving loop that forbids
+ * allocation once it is warmed up (a cudaMalloc there can stall on the driver
+ * or fail when the memory pool is full).
+ *  Arguments and results: as dqk_decode, minus workspace/workspace_bytes.
+ *  Scratch: a fixed DQK_NOALLOC_WORKSPACE_BYTES array in the library's static
+ *  device memory, held by every device that loads the library until the
+ *  process exits.  A request needing more than that (see
+ *  dqk_decode_workspace_size) returns DQK_ERR_WORKSPACE_TOO_SMALL with nothing
+ *  launched.  The call allocates nothing.
+ *  Set-up: the first call on a device (with that device current) looks up the
+ *  array's device address once; make that first call before any stream
+ *  capture.
+ *  Sharing: every call on a device uses the same array.  Calls whose work
+ *  overlaps on the GPU (different streams, no ordering between them) race on
+ *  it; order them on one stream or with events.  The decode needs no zeroed
+ *  scratch: each call writes what it reads. */
+dqk_status dqk_decode_noalloc(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
+                              int batch, const int *seq_lens, const int *page_table,
+                              int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
+                              dqk_stream_t stream);
 
 /* Synchronizes `stream`, then reads and clears the current device's error
  * word: DQK_OK, DQK_ERR_DEVICE_BOUNDS or DQK_ERR_TIMEOUT (DQK_ERR_CUDA if the
