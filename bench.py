@@ -301,7 +301,7 @@ def run_dqk(args):
         line = {
             "metric": METRIC, "value": agg["value"], "unit": "KV-tokens/s", "n_gpus": nranks,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": agg["ms_per_step"],
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int2-kv/f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int2-kv/f16-mma/f32-acc",
             "data": "synthetic",
             "config": {"workload": f"{w.name}: batch {w.batch}, {w.hq}/{w.hkv} heads, head_dim {w.d}, "
                                    f"context {int(layer.lens.max())}, 16-token pages ({w.page_order} order), "

@@ -3,13 +3,15 @@
 // holds every kernel of the decode hot path.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "common.cuh"
 #include "append.cuh"
-#include "attend_simple.cuh"
+#include "attend.cuh"
 #include "qprep.cuh"
 
 namespace {
@@ -32,24 +34,55 @@ dqk_status check_layer(const dqk_layer_desc *L) {
     return DQK_OK;
 }
 
-// Workspace layout of the decode: [qsel | part_o | part_ml], 256-B aligned.
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+}
+
+// Decode plan and workspace layout: [header | qf | qm | q0 | partial records],
+// every section 256-byte aligned.
 struct DecodePlan {
-    int d, G, ns, tokens_per_split;
-    size_t off_qsel, off_o, off_ml, bytes;
+    int d, G, NT, NG, hc, pps, nchunks, num_ctas, stages, bb;
+    size_t off_qf, off_qm, off_q0, off_part, bytes, smem;
 };
 
-DecodePlan plan_decode(const dqk_layer_desc *L, int batch, int max_pages) {
-    DecodePlan P;
+constexpr int kMaxAttendCtas = 320;
+
+bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.d = L->head_dim;
     P.G = L->num_q_heads / L->num_kv_heads;
-    P.ns = (max_pages + kSimplePagesPerSplit - 1) / kSimplePagesPerSplit;
-    P.tokens_per_split = kSimplePagesPerSplit * kPage;
-    const size_t rows = (size_t)batch * L->num_q_heads;
-    P.off_qsel = 256;
-    P.off_o = round_up(P.off_qsel + rows * P.d * sizeof(float), 256);
-    P.off_ml = round_up(P.off_o + rows * P.ns * P.d * sizeof(float), 256);
-    P.bytes = round_up(P.off_ml + rows * P.ns * 2 * sizeof(float), 256);
-    return P;
+    P.NT = P.G > 4 ? 2 : 1;
+    P.NG = P.d / kGroup;
+    const int hkv = L->num_kv_heads;
+    if (hkv <= kConsumerWarps) {
+        if (kConsumerWarps % hkv) return false;
+        P.hc = hkv;
+    } else {
+        if (hkv % kConsumerWarps) return false;
+        P.hc = kConsumerWarps;
+    }
+    P.pps = kConsumerWarps / P.hc;
+    P.nchunks = hkv / P.hc;
+    // Records are sized for kMaxAttendCtas so the workspace size does not depend
+    // on the device; the launch (check_decode) uses one CTA per SM up to that bound.
+    P.num_ctas = kMaxAttendCtas;
+    P.bb = make_layout(P.d, L->v_ch0_protect).bytes;
+    const size_t stage_bytes = (size_t)kConsumerWarps * P.bb;
+    const size_t per_stage = stage_bytes + 2 * sizeof(uint64_t) + 8;
+    const size_t budget = 227 * 1024 - 64;
+    P.stages = (int)std::min<size_t>(kMaxStages, budget / per_stage);
+    P.smem = P.stages * per_stage + 16;
+    const size_t R = (size_t)batch * P.nchunks;
+    const size_t bj = (size_t)batch * hkv;
+    P.off_qf = 256;
+    P.off_qm = round_up(P.off_qf + bj * P.NT * P.NG * 2 * 32 * sizeof(uint2), 256);
+    P.off_q0 = round_up(P.off_qm + bj * P.NT * 32 * sizeof(uint32_t), 256);
+    P.off_part = round_up(P.off_q0 + (size_t)batch * L->num_q_heads * sizeof(float), 256);
+    const size_t records = ((size_t)kMaxAttendCtas + R - 1) * P.pps * P.hc * P.G;
+    P.bytes = round_up(P.off_part + records * (2 + P.d) * sizeof(float), 256);
+    return true;
 }
 
 dqk_status launch_status() {
@@ -77,32 +110,74 @@ dqk_status check_decode(const DecodeArgs &a, DecodePlan &P) {
     if (a.q_dtype != DQK_F32 && a.q_dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
     if (a.batch <= 0 || a.max_pages <= 0 || a.pct < 0 || a.pct > 99) return DQK_ERR_INVALID_ARG;
     if (!aligned(a.ws, 256) || !aligned(a.out, 16)) return DQK_ERR_INVALID_ARG;
-    P = plan_decode(a.L, a.batch, a.max_pages);
+    if (!plan_decode(a.L, a.batch, P)) return DQK_ERR_UNSUPPORTED;
     if (a.ws_bytes < P.bytes) return DQK_ERR_WORKSPACE_TOO_SMALL;
+    P.num_ctas = std::min(device_sms(), kMaxAttendCtas);
+    if (P.num_ctas <= 0) return DQK_ERR_CUDA;
     return DQK_OK;
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream finishes; it orders itself with
+// griddepcontrol.wait before touching that kernel's outputs.
+template <typename... KArgs, typename... Args>
+dqk_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? DQK_OK : DQK_ERR_CUDA;
 }
 
 template <int D>
 dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
     const int G = P.G;
-    const size_t smem = (size_t)D * (D + 1) * 4 + (size_t)G * D * 4 + (size_t)G * D;
+    const size_t smem = (size_t)D * (D + 1) * 4 + (size_t)G * D * 4 + (size_t)G * P.NG * 4 + (size_t)G * D;
     if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DQK_ERR_CUDA;
-    float *qsel = reinterpret_cast<float *>(static_cast<char *>(a.ws) + P.off_qsel);
+    char *ws = static_cast<char *>(a.ws);
+    const float qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
     const int threads = (G < 4 ? 4 : G) * 32;
     k_qprep<D><<<dim3(a.L->num_kv_heads, a.batch), threads, smem, a.stream>>>(
-        a.L->t_q, a.q, a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qsel, a.sel_out);
+        a.L->t_q, a.q, a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qscale,
+        reinterpret_cast<uint2 *>(ws + P.off_qf), reinterpret_cast<uint32_t *>(ws + P.off_qm),
+        reinterpret_cast<float *>(ws + P.off_q0), a.sel_out);
     return launch_status();
 }
 
 template <int D, int G>
 dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
+    if (cudaFuncSetAttribute(k_attend<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
+        return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
-    k_attend_simple<D, G><<<dim3(P.ns, a.L->num_kv_heads, a.batch), kSimpleThreads, 0, a.stream>>>(
-        static_cast<const uint8_t *>(a.L->pool), a.L->num_kv_heads, a.L->v_ch0_protect, a.L->num_pages,
-        a.seq_lens, a.page_table, a.max_pages, reinterpret_cast<const float *>(ws + P.off_qsel), P.ns,
-        reinterpret_cast<float *>(ws + P.off_o), reinterpret_cast<float *>(ws + P.off_ml));
-    return launch_status();
+    AttendParams prm;
+    prm.pool = static_cast<const uint8_t *>(a.L->pool);
+    prm.num_pages = a.L->num_pages;
+    prm.seq_lens = a.seq_lens;
+    prm.page_table = a.page_table;
+    prm.qf = reinterpret_cast<const uint2 *>(ws + P.off_qf);
+    prm.qm = reinterpret_cast<const uint32_t *>(ws + P.off_qm);
+    prm.q0 = reinterpret_cast<const float *>(ws + P.off_q0);
+    prm.part = reinterpret_cast<float *>(ws + P.off_part);
+    prm.batch = a.batch;
+    prm.hq = a.L->num_q_heads;
+    prm.hkv = a.L->num_kv_heads;
+    prm.hc = P.hc;
+    prm.pps = P.pps;
+    prm.nchunks = P.nchunks;
+    prm.max_pages = a.max_pages;
+    prm.bb = P.bb;
+    prm.v_ch0 = a.L->v_ch0_protect;
+    prm.stages = P.stages;
+    prm.num_ctas = P.num_ctas;
+    return launch_pdl(k_attend<D, G>, dim3(P.num_ctas), dim3(kAttendThreads), P.smem, a.stream, prm);
 }
 
 template <int D>
@@ -118,10 +193,9 @@ dqk_status run_attend(const DecodeArgs &a, const DecodePlan &P) {
 template <int D>
 dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
     char *ws = static_cast<char *>(a.ws);
-    k_combine_simple<D><<<dim3(a.L->num_q_heads, a.batch), D, 0, a.stream>>>(
-        a.seq_lens, a.L->num_q_heads, P.ns, P.tokens_per_split, reinterpret_cast<const float *>(ws + P.off_o),
-        reinterpret_cast<const float *>(ws + P.off_ml), a.out);
-    return launch_status();
+    return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(D), 0, a.stream, a.seq_lens, a.batch,
+                      a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pps, P.nchunks, P.num_ctas,
+                      reinterpret_cast<const float *>(ws + P.off_part), a.out);
 }
 
 enum Stage { kPrepare = 1, kAttend = 2, kCombine = 4 };
@@ -195,7 +269,9 @@ dqk_status dqk_append(const dqk_layer_desc *layer, const void *k, const void *v,
 
 size_t dqk_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max_pages) {
     if (check_layer(layer) != DQK_OK || batch <= 0 || max_pages <= 0) return 0;
-    return plan_decode(layer, batch, max_pages).bytes;
+    DecodePlan P;
+    if (!plan_decode(layer, batch, P)) return 0;
+    return P.bytes;
 }
 
 #define DQK_DECODE_ARGS                                                                                   \
@@ -263,8 +339,9 @@ dqk_status dqk_decode_noalloc(const dqk_layer_desc *layer, const void *q, dqk_dt
     dqk_status st = check_layer(layer);
     if (st != DQK_OK) return st;
     if (batch <= 0 || max_pages <= 0) return DQK_ERR_INVALID_ARG;
-    if (plan_decode(layer, batch, max_pages).bytes > (size_t)DQK_NOALLOC_WORKSPACE_BYTES)
-        return DQK_ERR_WORKSPACE_TOO_SMALL;
+    DecodePlan P;
+    if (!plan_decode(layer, batch, P)) return DQK_ERR_UNSUPPORTED;
+    if (P.bytes > (size_t)DQK_NOALLOC_WORKSPACE_BYTES) return DQK_ERR_WORKSPACE_TOO_SMALL;
     void *ws = nullptr;
     st = noalloc_workspace(&ws);
     if (st != DQK_OK) return st;
