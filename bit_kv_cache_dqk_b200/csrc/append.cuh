@@ -73,19 +73,26 @@ __device__ void unpack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
         const int widx = is_v ? idx - 32 * NG : idx;
         const int lane = widx / NG, W = widx % NG, gid = lane >> 2, tig = lane & 3;
         const uint32_t word = w[((is_v ? L.vc : L.kc) >> 2) + widx];
+        if (!is_v) {
+            // byte j, field f: group g = f % NG, register r = W + NG * (f / NG)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int f = 0; f < 4; ++f) {
+                    const int g = f % NG, r = W + NG * (f / NG);
+                    S.kcode[gid + 8 * (r & 1)][32 * g + 16 * (r >> 1) + 4 * tig + j] =
+                        (uint8_t)((word >> (8 * j + 2 * f)) & 3u);
+                }
+            continue;
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int q = W * 8 + i;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const uint8_t code = (uint8_t)((word >> (16 * e + 2 * i)) & 3u);
-                if (!is_v) {
-                    const int tr = q & 1, cb = (q >> 1) & 1, s = (q >> 2) & 1, g = q >> 3;
-                    S.kcode[gid + 8 * tr][32 * g + 16 * s + 8 * cb + 2 * tig + e] = code;
-                } else {
-                    const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
-                    S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid] = code;
-                }
+                const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
+                S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid] = code;
             }
         }
     }
@@ -112,20 +119,25 @@ __device__ void pack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
         const int widx = is_v ? idx - 32 * NG : idx;
         const int lane = widx / NG, W = widx % NG, gid = lane >> 2, tig = lane & 3;
         uint32_t word = 0;
+        if (!is_v) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int q = W * 8 + i;
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                uint32_t code;
-                if (!is_v) {
-                    const int tr = q & 1, cb = (q >> 1) & 1, s = (q >> 2) & 1, g = q >> 3;
-                    code = S.kcode[gid + 8 * tr][32 * g + 16 * s + 8 * cb + 2 * tig + e];
-                } else {
-                    const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
-                    code = S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid];
+                for (int f = 0; f < 4; ++f) {
+                    const int g = f % NG, r = W + NG * (f / NG);
+                    word |= ((uint32_t)S.kcode[gid + 8 * (r & 1)][32 * g + 16 * (r >> 1) + 4 * tig + j] & 3u)
+                            << (8 * j + 2 * f);
                 }
-                word |= (code & 3u) << (16 * e + 2 * i);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = W * 8 + i;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
+                    word |= ((uint32_t)S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid] & 3u)
+                            << (16 * e + 2 * i);
+                }
             }
         }
         w[((is_v ? L.vc : L.kc) >> 2) + widx] = word;

@@ -8,15 +8,17 @@
 // [floor(c*U/C), floor((c+1)*U/C)): every CTA streams the same number of pages
 // whatever the length mix.  A producer warp brings whole units in with 1-D bulk
 // async copies (one copy = 16 tokens x up to 8 kv heads, contiguous) into a
-// ring of `stages` shared-memory buffers guarded by mbarriers; 8 consumer
-// warps, one per (kv head, page slot), run the tensor-core math.
+// ring of shared-memory stages of 16 (page, kv head) blocks guarded by
+// mbarriers.  8 consumer warps each own one kv head and take two pages of it
+// per stage, processed together (two independent instruction streams).
 //
 // Per consumer warp and page (16 tokens x G query heads), with
 // qs = q' * log2(e)/sqrt(d) on the kept channels:
-//   QK   D_g[t, n] = sum_{c in g} code[t, c] * qs_hilo[c, n]     (m16n8k16, per group)
-//        n = (head, fp16 high/low part of qs): the hi/lo split uses the columns
-//        a GQA group of 4 leaves free, so q is carried at ~22 bits;
-//        s[t, h] = sum_g scale[t, g] * (D_g[t,(h,hi)] + D_g[t,(h,lo)])
+//   QK   D_g[t, n] = sum_{c in g} code[t, c] * Q[c, n]    (m16n8k32 u8 x s8, per group)
+//        n = (head, piece): qs ~= sigma_g (Q1 + Q2/256) in two int8 pieces placed
+//        in the columns a GQA group of 4 leaves free (16 bits relative to the
+//        group's largest |qs|); one AND per 4 codes forms the u8 operand;
+//        s[t, h] = sum_g scale[t, g] * kappa_g * (D_g[t,(h,1)] + D_g[t,(h,2)]/256)
 //                + sum_g min[t, g] * Qsum[g, h]   (one extra m16n8k16)
 //                + qs_0[h] * k0[t]                (BF16 channel 0, fp32)
 //   online softmax in base 2 (running max per head, exact rescale on growth)
@@ -24,7 +26,7 @@
 //        with p~ = fp16(p); one extra m16n8k16 gives sum_t p~ * vmin[t, g] and
 //        l = sum_t p~ (a row of ones), so numerator and denominator see the
 //        same rounded weights.
-// Codes become exact fp16 operands with one LOP3 and one HSUB2 per pair.
+// Value codes become exact fp16 operands with one LOP3 and one HSUB2 per pair.
 #pragma once
 
 #include "common.cuh"
@@ -32,10 +34,11 @@
 
 namespace dqk {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kAttendThreads = (kConsumerWarps + 1) * 32;
-constexpr int kMaxStages = 16;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: a stuck pipeline reports DQK_ERR_TIMEOUT
+constexpr int kConsumerWarps = 8;                           // one kv head each (chunks of <= 8 heads)
+constexpr int kStageBlocks = 2 * kConsumerWarps;            // (page, kv head) blocks per stage
+constexpr int kAttendThreads = (kConsumerWarps + 1) * 32;   // + 1 producer warp
+constexpr int kMaxStages = 8;                               // ring depth cap
+constexpr uint64_t kWaitLimitNs = 1000000000ull;            // 1 s: a stuck pipeline reports DQK_ERR_TIMEOUT
 
 struct AttendParams {
     const uint8_t *pool;
@@ -43,10 +46,11 @@ struct AttendParams {
     const int *seq_lens;
     const int *page_table;
     const uint2 *qf;
+    const float *qk;
     const uint32_t *qm;
     const float *q0;
     float *part;
-    int batch, hq, hkv, hc, pps, nchunks, max_pages, bb, v_ch0, stages, num_ctas;
+    int batch, hq, hkv, hc, pps, pw, nchunks, max_pages, bb, v_ch0, stages, num_ctas;
 };
 
 // ---------------------------------------------------------------------------
@@ -99,8 +103,9 @@ __host__ __device__ __forceinline__ long long cta_of_unit(long long u, long long
     return ((u + 1) * C - 1) / U;
 }
 
-__device__ __forceinline__ size_t record_index(int slot, int ps, int jl, int hh, int pps, int hc, int G) {
-    return (((size_t)slot * pps + ps) * hc + jl) * G + hh;
+// Partial record of (slot = CTA + run, warp pair index pi, kv head jl, query head hh).
+__host__ __device__ __forceinline__ size_t record_index(int slot, int pi, int jl, int hh, int pw, int hc, int G) {
+    return (((size_t)slot * pw + pi) * hc + jl) * G + hh;
 }
 
 // ---------------------------------------------------------------------------
@@ -113,23 +118,233 @@ struct AttendTile {
     static constexpr int NM = D / 16;          // m-tiles of the PV product
 };
 
+// Online-softmax state of one consumer warp for one (run, kv head).
+template <int D, int G>
+struct WarpState {
+    using T = AttendTile<D, G>;
+    uint2 qbi[T::NT][T::NG];       // QK B fragments (s8 pieces Q1/Q2 of the kept, scaled q')
+    float4 kap[T::NT][T::NG];      // kappa, kappa/256, -M*kappa, -M*kappa/256 of this thread's head
+    uint32_t qmin[T::NT];          // min-term B fragment
+    float q0v[T::NT];              // scaled q'_0 of this thread's head
+    float m_run[T::NT];            // running max (log2 units) of this thread's head
+    float oacc[T::NT][T::NM][4];   // PV accumulators (columns 2*tig hold head tig)
+    float macc[T::NT][4];          // rows: group min terms, softmax denominator, channel 0
+};
+
+// Per-lane byte offsets into a block, fixed for the kernel.
+struct LaneOffsets {
+    uint32_t lane16;   // lane * 16: K/V code words
+    uint32_t gid8;     // (lane/4) * 8: K scales of token gid (token gid+8 at +64)
+    uint32_t kmin;     // K min pair of token gid for this lane's column pair
+    uint32_t gid4;     // (lane/4) * 4: K channel 0 of tokens gid, gid+8
+    uint32_t tig16;    // (lane%4) * 16: V scale pairs of tokens 2tig.. (+64: 2tig+8..)
+    uint32_t vmin;     // V min pair of row min(gid, NG-1), tokens 2tig, 2tig+1
+    int srcA;          // lane holding p of (token 2tig, head gid/2); +4: token 2tig+1
+    uint32_t ones_lane, vmin_mask, kmin_mask;
+};
+
+// NB (page, kv head) blocks at shared addresses sb[]: 16 tokens x G query heads
+// each, same run.  MASKED (NB == 1 only): only the first nv tokens are valid.
+template <int D, int G, int NB, bool MASKED>
+__device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpState<D, G> &st, int lane,
+                                        const LaneOffsets &o, int v_ch0) {
+    using T = AttendTile<D, G>;
+    constexpr int NG = T::NG, NT = T::NT;
+    constexpr Layout Ly = make_layout(D, 0);   // section offsets do not depend on v_ch0 (V0 is last)
+    static_assert(NB == 1 || !MASKED, "masked blocks are processed alone");
+    const int gid = lane >> 2, tig = lane & 3;
+
+    // ---------------------------------------------------------------- keys
+    uint32_t kw[NB][NG], ks0[NB][NG / 2], ks1[NB][NG / 2], km0[NB], km1[NB];
+    float k0a[NB], k0b[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        if constexpr (NG == 4) {
+            const uint4 v = ld_s128(sb[b] + o.lane16 + Ly.kc);
+            kw[b][0] = v.x; kw[b][1] = v.y; kw[b][2] = v.z; kw[b][3] = v.w;
+            const uint32_t a = sb[b] + o.gid8;
+            const uint2 x = ld_s64(a + Ly.ks), y = ld_s64(a + Ly.ks + 64);
+            ks0[b][0] = x.x; ks0[b][1] = x.y; ks1[b][0] = y.x; ks1[b][1] = y.y;
+        } else {
+            const uint2 v = ld_s64(sb[b] + (o.lane16 >> 1) + Ly.kc);
+            kw[b][0] = v.x; kw[b][1] = v.y;
+            const uint32_t a = sb[b] + (o.gid8 >> 1);
+            ks0[b][0] = ld_s32(a + Ly.ks);
+            ks1[b][0] = ld_s32(a + Ly.ks + 32);
+        }
+        const uint32_t akm = sb[b] + o.kmin;
+        km0[b] = ld_s32(akm + Ly.km) & o.kmin_mask;
+        km1[b] = ld_s32(akm + Ly.km + 16 * NG) & o.kmin_mask;
+        const uint32_t k0w = ld_s32(sb[b] + o.gid4 + Ly.k0);
+        k0a[b] = __uint_as_float(k0w << 16);
+        k0b[b] = __uint_as_float(k0w & 0xffff0000u);
+    }
+    float a0[NB][NT], a1[NB][NT], cmin[NB][NT][4];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            a0[b][nt] = 0.0f;
+            a1[b][nt] = 0.0f;
+            cmin[b][nt][0] = cmin[b][nt][1] = cmin[b][nt][2] = cmin[b][nt][3] = 0.0f;
+            mma_f16(cmin[b][nt], km0[b], km1[b], 0u, 0u, st.qmin[nt], 0u);
+        }
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const uint32_t msk = 0x03030303u << (2 * g);   // group g's field in every byte: code * 4^g
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            uint32_t A0, A1, A2, A3;
+            if constexpr (NG == 4) {
+                A0 = kw[b][0] & msk; A1 = kw[b][1] & msk; A2 = kw[b][2] & msk; A3 = kw[b][3] & msk;
+            } else {
+                A0 = kw[b][0] & msk; A1 = kw[b][1] & msk;
+                A2 = (kw[b][0] >> 4) & msk; A3 = (kw[b][1] >> 4) & msk;
+            }
+            // key scales * 2^-112 (integer ops only)
+            const float sa = (g & 1) ? f16hi_scaled(ks0[b][g >> 1]) : f16lo_scaled(ks0[b][g >> 1]);
+            const float sbv = (g & 1) ? f16hi_scaled(ks1[b][g >> 1]) : f16lo_scaled(ks1[b][g >> 1]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                int dg[4] = {kMagicI, kMagicI, kMagicI, kMagicI};
+                mma_u8s8(dg, A0, A1, A2, A3, st.qbi[nt][g].x, st.qbi[nt][g].y);
+                // (M + I) * kappa - M * kappa = I * kappa, one rounding
+                const float4 kp = st.kap[nt][g];
+                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[0]), kp.x, kp.z), a0[b][nt]);
+                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[1]), kp.y, kp.w), a0[b][nt]);
+                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[2]), kp.x, kp.z), a1[b][nt]);
+                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[3]), kp.y, kp.w), a1[b][nt]);
+            }
+        }
+    }
+    float s0[NB][NT], s1[NB][NT];
+    bool grow = false;
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            s0[b][nt] = fmaf(a0[b][nt], kTwoPow112, fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0] + cmin[b][nt][1]));
+            s1[b][nt] = fmaf(a1[b][nt], kTwoPow112, fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2] + cmin[b][nt][3]));
+            if constexpr (MASKED) {
+                if (gid >= nv) s0[b][nt] = -INFINITY;
+                if (gid + 8 >= nv) s1[b][nt] = -INFINITY;
+            }
+            grow |= (s0[b][nt] > st.m_run[nt]) | (s1[b][nt] > st.m_run[nt]);
+        }
+    // The running max only moves when a score exceeds it (rare after the first
+    // pages): then take the exact max over these pages and rescale.
+    if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float mx = fmaxf(s0[0][nt], s1[0][nt]);
+#pragma unroll
+            for (int b = 1; b < NB; ++b) mx = fmaxf(mx, fmaxf(s0[b][nt], s1[b][nt]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mnew = fmaxf(st.m_run[nt], mx);
+            const float alpha = fast_exp2(st.m_run[nt] - mnew);   // 0 when the old max is -inf
+#pragma unroll
+            for (int m = 0; m < T::NM; ++m) {
+                st.oacc[nt][m][0] *= alpha;
+                st.oacc[nt][m][2] *= alpha;
+            }
+            st.macc[nt][0] *= alpha;
+            st.macc[nt][2] *= alpha;
+            st.m_run[nt] = mnew;
+        }
+    }
+
+    // ---------------------------------------------------------------- values
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        uint32_t vw[NG], vsa[NG], vsb[NG];   // vsa/vsb: scale pairs of tokens (2tig, 2tig+1) and (+8, +9)
+        if constexpr (NG == 4) {
+            const uint4 v = ld_s128(sb[b] + o.lane16 + Ly.vc);
+            vw[0] = v.x; vw[1] = v.y; vw[2] = v.z; vw[3] = v.w;
+            const uint32_t a = sb[b] + o.tig16;
+            const uint4 x = ld_s128(a + Ly.vs), y = ld_s128(a + Ly.vs + 64);
+            vsa[0] = x.x; vsa[1] = x.y; vsa[2] = x.z; vsa[3] = x.w;
+            vsb[0] = y.x; vsb[1] = y.y; vsb[2] = y.z; vsb[3] = y.w;
+        } else {
+            const uint2 v = ld_s64(sb[b] + (o.lane16 >> 1) + Ly.vc);
+            vw[0] = v.x; vw[1] = v.y;
+            const uint32_t a = sb[b] + (o.tig16 >> 1);
+            const uint2 x = ld_s64(a + Ly.vs), y = ld_s64(a + Ly.vs + 32);
+            vsa[0] = x.x; vsa[1] = x.y;
+            vsb[0] = y.x; vsb[1] = y.y;
+        }
+        // A rows of the min / denominator / channel-0 product: row g < NG = v-min
+        // of group g, row NG = ones, row NG+1 = value channel 0 (when protected).
+        const uint32_t avm = sb[b] + o.vmin;
+        uint32_t vma = (ld_s32(avm + Ly.vm) & o.vmin_mask) | o.ones_lane;
+        uint32_t vmb = (ld_s32(avm + Ly.vm + 16 * NG) & o.vmin_mask) | o.ones_lane;
+        if (v_ch0) {
+            const Layout L1 = make_layout(D, 1);
+            const uint32_t a = ld_s32(sb[b] + L1.v0 + tig * 4), c = ld_s32(sb[b] + L1.v0 + 16 + tig * 4);
+            if (gid == NG + 1) {
+                vma = pack_f16x2(__uint_as_float(a << 16), __uint_as_float(a & 0xffff0000u));
+                vmb = pack_f16x2(__uint_as_float(c << 16), __uint_as_float(c & 0xffff0000u));
+            }
+        }
+        if constexpr (MASKED) {
+            // rows past the end of the sequence hold stale bytes: zero their factors
+            const uint32_t ma = (2 * tig < nv ? 0x0000ffffu : 0u) | (2 * tig + 1 < nv ? 0xffff0000u : 0u);
+            const uint32_t mb = (2 * tig + 8 < nv ? 0x0000ffffu : 0u) | (2 * tig + 9 < nv ? 0xffff0000u : 0u);
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                vsa[g] &= ma;
+                vsb[g] &= mb;
+            }
+            vma &= ma;
+            vmb &= mb;
+        }
+        // P~ in the PV B-operand layout (column gid = head gid/2 of the n-tile; odd
+        // columns duplicate even ones and are never read back).
+        uint32_t pb0[NT], pb1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float p0 = fast_exp2(s0[b][nt] - st.m_run[nt]), p1 = fast_exp2(s1[b][nt] - st.m_run[nt]);
+            const uint32_t pp = pack_f16x2(p0, p1);   // lo: token gid, hi: token gid+8
+            const uint32_t w0 = __shfl_sync(0xffffffffu, pp, o.srcA);
+            const uint32_t w1 = __shfl_sync(0xffffffffu, pp, o.srcA + 4);
+            pb0[nt] = prmt(w0, w1, 0x5410u);   // tokens 2tig, 2tig+1
+            pb1[nt] = prmt(w0, w1, 0x7632u);   // tokens 2tig+8, 2tig+9
+            mma_f16(st.macc[nt], vma, 0u, vmb, 0u, pb0[nt], pb1[nt]);
+        }
+#pragma unroll
+        for (int w2 = 0; w2 < NG; ++w2) {       // word w2 holds m-tiles 2*w2, 2*w2+1 (= group w2)
+            const uint32_t x = vw[w2], xh = x >> 10;
+            const uint32_t e0 = code_field<0>(x, xh), e2 = code_field<2>(x, xh);
+            const uint32_t e1 = code_field<1>(x, xh), e3 = code_field<3>(x, xh);
+            const uint32_t f0 = code_field<4>(x, xh), f2 = code_field<6>(x, xh);
+            const uint32_t f1 = code_field<5>(x, xh), f3 = code_field<7>(x, xh);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t b0 = hmul2(pb0[nt], vsa[w2]), b1 = hmul2(pb1[nt], vsb[w2]);
+                mma_f16(st.oacc[nt][2 * w2], e0, e2, e1, e3, b0, b1);
+                mma_f16(st.oacc[nt][2 * w2 + 1], f0, f2, f1, f3, b0, b1);
+            }
+        }
+    }
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams p) {
     using T = AttendTile<D, G>;
     constexpr int NG = T::NG, NT = T::NT, NM = T::NM;
     extern __shared__ __align__(128) unsigned char attend_smem[];
-    unsigned char *smem_raw = attend_smem;
     const int S = p.stages;
-    const uint32_t stage_bytes = (uint32_t)(kConsumerWarps * p.bb);
-    unsigned char *stage_mem = smem_raw;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw + (size_t)S * stage_bytes);
-    uint64_t *empty = full + S;
-    unsigned char *valid = reinterpret_cast<unsigned char *>(empty + S);   // [S][8]
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(valid + S * 8);
+    const uint32_t stage_bytes = (uint32_t)(kStageBlocks * p.bb);
+    unsigned char *stage_mem = attend_smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(attend_smem + (size_t)S * stage_bytes);
+    uint64_t *empty = full + kMaxStages;
+    unsigned char *valid = reinterpret_cast<unsigned char *>(empty + kMaxStages);   // [kMaxStages][kStageBlocks]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(valid + kMaxStages * kStageBlocks);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = p.batch * p.nchunks;
-    const long long C = p.num_ctas;
+    const int pps = p.pps;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -141,27 +356,26 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     }
     __syncthreads();
 
-    const long long U = warp_total_units(p.seq_lens, p.nchunks, R, lane);
-    const long long u0 = (long long)blockIdx.x * U / C, u1 = ((long long)blockIdx.x + 1) * U / C;
-    const long long nunits = u1 - u0;
-    const int iters = (int)((nunits + p.pps - 1) / p.pps);
+    const int U = (int)warp_total_units(p.seq_lens, p.nchunks, R, lane);
+    const int u0 = (int)((long long)blockIdx.x * U / p.num_ctas);
+    const int u1 = (int)(((long long)blockIdx.x + 1) * U / p.num_ctas);
+    const int nunits = u1 - u0;
+    const int iters = (nunits + pps - 1) / pps;
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
-        // Let the next kernel in the stream start its prologue early.
-        grid_dependents_launch();
+        grid_dependents_launch();   // the combine kernel may start its prologue
         if (iters == 0) return;
         int r;
-        long long ur;
-        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, ur);
+        long long urll;
+        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
+        int ur = (int)urll;
         int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
         const uint32_t copy_bytes = (uint32_t)(p.hc * p.bb);
-        // byte offset in the pool of unit ubase + lane, or -1
-        auto fetch = [&](long long ubase, int &r_c, long long &ur_c, int &np_c) -> long long {
-            const long long u = ubase + lane;
-            int rr = r_c;
-            long long st = ur_c;
-            int np = np_c;
+        // pool byte offset of unit ubase + lane (or -1); moves the cursor to unit ubase + 32
+        auto fetch = [&](int ubase) -> long long {
+            const int u = ubase + lane;
+            int rr = r, st = ur, np = npr;
             while (rr < R && u >= st + np) {
                 st += np;
                 ++rr;
@@ -169,8 +383,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
             }
             long long off = -1;
             if (u < u1 && rr < R) {
-                const int b = rr / p.nchunks, chunk = rr % p.nchunks;
-                const long long page = u - st;
+                const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
+                const int page = u - st;
                 if (page < p.max_pages) {
                     const int phys = p.page_table[(size_t)b * p.max_pages + page];
                     if (phys >= 0 && phys < p.num_pages)
@@ -178,29 +392,22 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
                 }
                 if (off < 0) dqk_flag_error(kErrBounds);
             }
-            // advance the warp cursor to the run of unit ubase + 32
-            rr = __shfl_sync(0xffffffffu, rr, 31);
-            st = __shfl_sync(0xffffffffu, st, 31);
-            np = __shfl_sync(0xffffffffu, np, 31);
-            r_c = rr;
-            ur_c = st;
-            np_c = np;
+            r = __shfl_sync(0xffffffffu, rr, 31);
+            ur = __shfl_sync(0xffffffffu, st, 31);
+            npr = __shfl_sync(0xffffffffu, np, 31);
             return off;
         };
-        long long off_next = fetch(u0, r, ur, npr);
+        long long off_next = fetch(u0);
+        int it = 0, stage = 0;
+        uint32_t phase = 0;
         bool ok = true;
-        int it = 0;
-        for (long long ubase = u0; ubase < u1 && ok; ubase += 32) {
+        for (int ubase = u0; ubase < u1 && ok; ubase += 32) {
             const long long off_cur = off_next;
-            if (ubase + 32 < u1) off_next = fetch(ubase + 32, r, ur, npr);
-            // stage iterations whose units lie in this batch of 32
-            for (; ok && (long long)it * p.pps < nunits && u0 + (long long)it * p.pps < ubase + 32; ++it) {
-                const int s = it % S;
-                const uint32_t round = (uint32_t)(it / S);
+            if (ubase + 32 < u1) off_next = fetch(ubase + 32);
+            for (; it < iters && u0 + it * pps < ubase + 32; ++it) {
                 int good = 1;
-                if (lane == 0) good = mbar_wait_bounded(&empty[s], (round & 1u) ^ 1u, kWaitLimitNs) && !*abort_flag;
-                good = __shfl_sync(0xffffffffu, good, 0);
-                if (!good) {
+                if (lane == 0) good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs) && !*abort_flag;
+                if (!__shfl_sync(0xffffffffu, good, 0)) {
                     if (lane == 0) {
                         *abort_flag = 1;
                         dqk_flag_error(kErrTimeout);
@@ -208,54 +415,48 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
                     ok = false;
                     break;
                 }
-                uint32_t bytes = 0;
-                long long offs[8];
-#pragma unroll
-                for (int ps = 0; ps < 8; ++ps) {
-                    const long long u = u0 + (long long)it * p.pps + ps;
-                    const int src = (int)(u - ubase);
-                    long long o = __shfl_sync(0xffffffffu, off_cur, src & 31);
-                    if (ps >= p.pps || u >= u1) o = -1;
-                    offs[ps] = o;
-                    if (o >= 0) bytes += copy_bytes;
-                }
-                if (lane == 0) {
-#pragma unroll
-                    for (int ps = 0; ps < 8; ++ps)
-                        if (ps < p.pps) valid[s * 8 + ps] = offs[ps] >= 0 ? 1 : 0;
-                    mbar_arrive_expect_tx(&full[s], bytes);
-#pragma unroll
-                    for (int ps = 0; ps < 8; ++ps)
-                        if (ps < p.pps && offs[ps] >= 0)
-                            bulk_copy_g2s(stage_mem + (size_t)s * stage_bytes + (size_t)ps * copy_bytes,
-                                          p.pool + offs[ps], copy_bytes, &full[s]);
+                // lane k < pps fills page slot k of this stage
+                const int uk = u0 + it * pps + lane;
+                const long long off = __shfl_sync(0xffffffffu, off_cur, (uk - ubase) & 31);
+                const bool have = lane < pps && uk < u1 && off >= 0;
+                const unsigned ballot = __ballot_sync(0xffffffffu, have);
+                if (lane < pps) valid[stage * kStageBlocks + lane] = have ? 1 : 0;
+                __syncwarp();
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(ballot) * copy_bytes);
+                __syncwarp();
+                if (have)
+                    bulk_copy_g2s(stage_mem + (size_t)stage * stage_bytes + (size_t)lane * copy_bytes, p.pool + off,
+                                  copy_bytes, &full[stage]);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
         }
-        // never leave with copies in flight: wait (bounded) for the last round of each stage
-        if (lane == 0) {
-            const int issued = it;
-            for (int k = issued - 1; k >= 0 && k >= issued - S; --k)
+        // never leave with copies in flight (exit path: wait, bounded, for the last round of each stage)
+        if (lane == 0)
+            for (int k = it - 1; k >= 0 && k >= it - S; --k)
                 (void)mbar_wait_bounded(&full[k % S], (uint32_t)(k / S) & 1u, kWaitLimitNs);
-        }
         return;
     }
 
     // ---------------------------------------------------------------- consumers
-    const int jl = warp % p.hc, ps = warp / p.hc;
+    // warp: kv head jl of the chunk, page pair pi of each stage (pages 2pi, 2pi+1)
+    const int jl = warp % p.hc, pi = warp / p.hc;
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
 
-    // Every (run, page slot, kv head) record this warp could own starts empty:
-    // a run shorter than the page slots leaves some warps without a page.
-    if (nunits > 0 && ps < p.pps) {
+    // Every (run, pair, kv head) record this warp could own starts empty: a run
+    // shorter than the page slots leaves some warps without a page.
+    if (nunits > 0) {
         int r;
-        long long ur;
-        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, ur);
+        long long urll;
+        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
+        int ur = (int)urll;
         int np = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
         while (r < R && ur < u1) {
             if (np > 0 && lane < G) {
-                float *rec = p.part + record_index(slot_base + r, ps, jl, lane, p.pps, p.hc, G) * (2 + D);
+                float *rec = p.part + record_index(slot_base + r, pi, jl, lane, p.pw, p.hc, G) * (2 + D);
                 rec[0] = -INFINITY;
                 rec[1] = 0.0f;
             }
@@ -267,40 +468,52 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     if (iters == 0) return;
     grid_dependency_wait();     // query fragments come from k_qprep
 
-    int r;
-    long long ur;
-    warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, ur);
-    int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-    int cur_run = -1, Lb = 0;
+    int r, ur, npr;
+    {
+        long long urll;
+        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
+        ur = (int)urll;
+        npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
+    }
+    int cur_run = -1, run_end = -1, partial_u = -1, nv_last = kPage;
 
-    uint2 qb[NT][NG][2];
-    uint32_t qmin[NT];
-    float q0v[NT], m_run[NT];
-    float oacc[NT][NM][4];
-    float macc[NT][4];
+    WarpState<D, G> st;
+    LaneOffsets lo;
+    lo.lane16 = lane * 16;
+    lo.gid8 = gid * 8;
+    lo.kmin = gid * 2 * NG + (tig & (NG / 2 - 1)) * 4;   // in range for every lane; kmin_mask zeroes the rest
+    lo.gid4 = gid * 4;
+    lo.tig16 = tig * 16;
+    lo.vmin = (tig * NG + (gid < NG ? gid : 0)) * 4;
+    lo.srcA = (2 * tig) * 4 + (gid >> 1);
+    lo.ones_lane = gid == NG ? 0x3C003C00u : 0u;
+    lo.vmin_mask = gid < NG ? 0xffffffffu : 0u;
+    lo.kmin_mask = tig < NG / 2 ? 0xffffffffu : 0u;
 
     auto start_run = [&](int rr) {
-        const int b = rr / p.nchunks, chunk = rr % p.nchunks;
+        const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
         const int j = chunk * p.hc + jl;
         const size_t bj = (size_t)b * p.hkv + j;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
-#pragma unroll
-                for (int s = 0; s < 2; ++s) qb[nt][g][s] = p.qf[(((bj * NT + nt) * NG + g) * 2 + s) * 32 + lane];
-            qmin[nt] = p.qm[(bj * NT + nt) * 32 + lane];
+            for (int g = 0; g < NG; ++g) {
+                st.qbi[nt][g] = p.qf[((bj * NT + nt) * NG + g) * 32 + lane];
+                const float kappa = p.qk[((bj * NT + nt) * NG + g) * 4 + tig];
+                st.kap[nt][g] = make_float4(kappa, kappa * (1.0f / 256.0f), -kMagicF * kappa,
+                                            -kMagicF * kappa * (1.0f / 256.0f));
+            }
+            st.qmin[nt] = p.qm[(bj * NT + nt) * 32 + lane];
             const int hh = 4 * nt + tig;
-            q0v[nt] = hh < G ? p.q0[(size_t)b * p.hq + j * G + hh] : 0.0f;
-            m_run[nt] = -INFINITY;
+            st.q0v[nt] = hh < G ? p.q0[(size_t)b * p.hq + j * G + hh] : 0.0f;
+            st.m_run[nt] = -INFINITY;
 #pragma unroll
             for (int m = 0; m < NM; ++m)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) oacc[nt][m][e] = 0.0f;
+                for (int e = 0; e < 4; ++e) st.oacc[nt][m][e] = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) macc[nt][e] = 0.0f;
+            for (int e = 0; e < 4; ++e) st.macc[nt][e] = 0.0f;
         }
-        Lb = p.seq_lens[b];
         cur_run = rr;
     };
 
@@ -309,33 +522,50 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
         for (int nt = 0; nt < NT; ++nt) {
             float minterm[NG];
 #pragma unroll
-            for (int g = 0; g < NG; ++g) minterm[g] = __shfl_sync(0xffffffffu, macc[nt][0], g * 4 + tig);
-            const float l = __shfl_sync(0xffffffffu, macc[nt][0], NG * 4 + tig);
-            const float v0t = __shfl_sync(0xffffffffu, macc[nt][0], (NG + 1) * 4 + tig);
+            for (int g = 0; g < NG; ++g) minterm[g] = __shfl_sync(0xffffffffu, st.macc[nt][0], g * 4 + tig);
+            const float l = __shfl_sync(0xffffffffu, st.macc[nt][0], NG * 4 + tig);
+            const float v0t = __shfl_sync(0xffffffffu, st.macc[nt][0], (NG + 1) * 4 + tig);
             const int hh = 4 * nt + tig;
             if (hh < G) {
-                float *rec = p.part + record_index(slot_base + rr, ps, jl, hh, p.pps, p.hc, G) * (2 + D);
+                float *rec = p.part + record_index(slot_base + rr, pi, jl, hh, p.pw, p.hc, G) * (2 + D);
                 if (gid == 0) {
-                    rec[0] = m_run[nt];
+                    rec[0] = st.m_run[nt];
                     rec[1] = l;
                 }
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
                     const int c0 = 16 * m + gid, c1 = c0 + 8;
                     const float mt = minterm[m >> 1];
-                    rec[2 + c0] = (p.v_ch0 && c0 == 0) ? v0t : oacc[nt][m][0] + mt;
-                    rec[2 + c1] = oacc[nt][m][2] + mt;
+                    rec[2 + c0] = (p.v_ch0 && c0 == 0) ? v0t : st.oacc[nt][m][0] + mt;
+                    rec[2 + c1] = st.oacc[nt][m][2] + mt;
                 }
             }
         }
     };
 
-    const uint32_t kOnes = 0x3C003C00u;
+    // move to the run holding unit u (u >= run_end)
+    auto switch_run = [&](int u) {
+        if (cur_run >= 0) finish_run(cur_run);
+        while (r < R && u >= ur + npr) {
+            ur += npr;
+            ++r;
+            npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
+        }
+        start_run(r);
+        run_end = ur + npr;
+        const int Lb = p.seq_lens[r / p.nchunks];
+        partial_u = (Lb & (kPage - 1)) ? run_end - 1 : -1;
+        nv_last = Lb - (npr - 1) * kPage;
+    };
+
     bool ok = true;
+    int stage = 0;
+    uint32_t phase = 0;
+    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((2 * pi * p.hc + jl) * p.bb);
+    const uint32_t pair_gap = (uint32_t)(p.hc * p.bb);
+    const uint32_t valid_addr = smem_addr(valid) + 2 * pi;
     for (int it = 0; it < iters; ++it) {
-        const int s = it % S;
-        const uint32_t round = (uint32_t)(it / S);
-        if (!mbar_wait_bounded(&full[s], round & 1u, kWaitLimitNs) || *abort_flag) {
+        if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
             if (lane == 0) {
                 *abort_flag = 1;
                 dqk_flag_error(kErrTimeout);
@@ -343,181 +573,36 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
             ok = false;
             break;
         }
-        const long long u = u0 + (long long)it * p.pps + ps;
-        if (ps < p.pps && u < u1) {
-            while (r < R && u >= ur + npr) {
-                ur += npr;
-                ++r;
-                npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-            }
-            if (r != cur_run) {
-                if (cur_run >= 0) finish_run(cur_run);
-                start_run(r);
-            }
-            if (valid[s * 8 + ps]) {
-                const long long page = u - ur;
-                const int nv = (int)min((long long)kPage, (long long)Lb - page * kPage);
-                const unsigned char *blk = stage_mem + (size_t)s * stage_bytes + (size_t)(ps * p.hc + jl) * p.bb;
-                const Layout Ly = make_layout(D, p.v_ch0);
-
-                // ------------------------------------------------ key side
-                uint32_t kw[NG];
-                if constexpr (NG == 4) {
-                    const uint4 v = lds128(blk + Ly.kc + lane * 16);
-                    kw[0] = v.x; kw[1] = v.y; kw[2] = v.z; kw[3] = v.w;
-                } else {
-                    const uint2 v = lds64(blk + Ly.kc + lane * 8);
-                    kw[0] = v.x; kw[1] = v.y;
+        const int ua = u0 + it * pps + 2 * pi, ub = ua + 1;
+        if (ua < u1) {
+            const uint32_t vv = ld_s16(valid_addr + stage * kStageBlocks);   // flags of slots 2pi, 2pi+1 (even address)
+            if (ua >= run_end) switch_run(ua);
+            const uint32_t sa = blk_a + (uint32_t)stage * stage_bytes;
+            if (ub < run_end && ub < u1 && ub != partial_u && vv == 0x0101u) {
+                const uint32_t sbb[2] = {sa, sa + pair_gap};
+                consume<D, G, 2, false>(sbb, kPage, st, lane, lo, p.v_ch0);
+            } else {
+                const uint32_t s1[1] = {sa};
+                if (vv & 0xffu) {
+                    if (ua == partial_u) consume<D, G, 1, true>(s1, nv_last, st, lane, lo, p.v_ch0);
+                    else consume<D, G, 1, false>(s1, kPage, st, lane, lo, p.v_ch0);
                 }
-                uint32_t ks0[(NG + 1) / 2], ks1[(NG + 1) / 2];   // fp16 scale pairs of tokens gid, gid+8
-                if constexpr (NG == 4) {
-                    const uint2 a = lds64(blk + Ly.ks + gid * 8), c = lds64(blk + Ly.ks + (gid + 8) * 8);
-                    ks0[0] = a.x; ks0[1] = a.y; ks1[0] = c.x; ks1[1] = c.y;
-                } else {
-                    ks0[0] = lds32(blk + Ly.ks + gid * 4);
-                    ks1[0] = lds32(blk + Ly.ks + (gid + 8) * 4);
-                }
-                const bool has_min = tig < NG / 2;
-                const uint32_t km0 = has_min ? lds32(blk + Ly.km + gid * 2 * NG + tig * 4) : 0u;
-                const uint32_t km1 = has_min ? lds32(blk + Ly.km + (gid + 8) * 2 * NG + tig * 4) : 0u;
-                const uint32_t k0w = lds32(blk + Ly.k0 + gid * 4);
-                const float k0a = __uint_as_float(k0w << 16), k0b = __uint_as_float(k0w & 0xffff0000u);
-
-                uint32_t ka[NG][2][4];
-#pragma unroll
-                for (int g = 0; g < NG; ++g) {
-                    const uint32_t x = kw[g], xh = x >> 10;
-                    ka[g][0][0] = code_field<0>(x, xh);
-                    ka[g][0][1] = code_field<1>(x, xh);
-                    ka[g][0][2] = code_field<2>(x, xh);
-                    ka[g][0][3] = code_field<3>(x, xh);
-                    ka[g][1][0] = code_field<4>(x, xh);
-                    ka[g][1][1] = code_field<5>(x, xh);
-                    ka[g][1][2] = code_field<6>(x, xh);
-                    ka[g][1][3] = code_field<7>(x, xh);
-                }
-
-                float p0[NT], p1[NT], alpha[NT];
-                bool grow = false;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float cm[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_f16(cm, km0, km1, 0u, 0u, qmin[nt], 0u);
-                    float s0 = cm[0] + cm[1], s1 = cm[2] + cm[3];
-#pragma unroll
-                    for (int g = 0; g < NG; ++g) {
-                        float dg[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_f16(dg, ka[g][0][0], ka[g][0][1], ka[g][0][2], ka[g][0][3], qb[nt][g][0].x,
-                                qb[nt][g][0].y);
-                        mma_f16(dg, ka[g][1][0], ka[g][1][1], ka[g][1][2], ka[g][1][3], qb[nt][g][1].x,
-                                qb[nt][g][1].y);
-                        const float2 sa = f16x2_to_f32x2(ks0[g >> 1]), sb = f16x2_to_f32x2(ks1[g >> 1]);
-                        s0 = fmaf((g & 1) ? sa.y : sa.x, dg[0] + dg[1], s0);
-                        s1 = fmaf((g & 1) ? sb.y : sb.x, dg[2] + dg[3], s1);
-                    }
-                    s0 = fmaf(q0v[nt], k0a, s0);
-                    s1 = fmaf(q0v[nt], k0b, s1);
-                    if (gid >= nv) s0 = -INFINITY;
-                    if (gid + 8 >= nv) s1 = -INFINITY;
-                    float mx = fmaxf(s0, s1);
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    const float mnew = fmaxf(m_run[nt], mx);
-                    grow |= mnew > m_run[nt];
-                    const float mref = mnew == -INFINITY ? 0.0f : mnew;
-                    alpha[nt] = exp2f(m_run[nt] - mref);
-                    p0[nt] = exp2f(s0 - mref);
-                    p1[nt] = exp2f(s1 - mref);
-                    m_run[nt] = mnew;
-                }
-                if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                        for (int m = 0; m < NM; ++m) {
-                            oacc[nt][m][0] *= alpha[nt];
-                            oacc[nt][m][2] *= alpha[nt];
-                        }
-                        macc[nt][0] *= alpha[nt];
-                        macc[nt][2] *= alpha[nt];
-                    }
-                }
-
-                // ------------------------------------------------ value side
-                uint32_t vw[NG];
-                if constexpr (NG == 4) {
-                    const uint4 v = lds128(blk + Ly.vc + lane * 16);
-                    vw[0] = v.x; vw[1] = v.y; vw[2] = v.z; vw[3] = v.w;
-                } else {
-                    const uint2 v = lds64(blk + Ly.vc + lane * 8);
-                    vw[0] = v.x; vw[1] = v.y;
-                }
-                uint32_t vsa[NG], vsb[NG];   // scale pairs of tokens (2tig, 2tig+1) and (2tig+8, 2tig+9)
-                if constexpr (NG == 4) {
-                    const uint4 a = lds128(blk + Ly.vs + tig * 16), c = lds128(blk + Ly.vs + (tig + 4) * 16);
-                    vsa[0] = a.x; vsa[1] = a.y; vsa[2] = a.z; vsa[3] = a.w;
-                    vsb[0] = c.x; vsb[1] = c.y; vsb[2] = c.z; vsb[3] = c.w;
-                } else {
-                    const uint2 a = lds64(blk + Ly.vs + tig * 8), c = lds64(blk + Ly.vs + (tig + 4) * 8);
-                    vsa[0] = a.x; vsa[1] = a.y;
-                    vsb[0] = c.x; vsb[1] = c.y;
-                }
-                uint32_t vma = 0u, vmb = 0u;    // rows of the min / ones / channel-0 product
-                if (gid < NG) {
-                    vma = lds32(blk + Ly.vm + (tig * NG + gid) * 4);
-                    vmb = lds32(blk + Ly.vm + ((tig + 4) * NG + gid) * 4);
-                } else if (gid == NG) {
-                    vma = kOnes;
-                    vmb = kOnes;
-                } else if (gid == NG + 1 && p.v_ch0) {
-                    const uint32_t a = lds32(blk + Ly.v0 + tig * 4), c = lds32(blk + Ly.v0 + (tig + 4) * 4);
-                    vma = pack_f16x2(__uint_as_float(a << 16), __uint_as_float(a & 0xffff0000u));
-                    vmb = pack_f16x2(__uint_as_float(c << 16), __uint_as_float(c & 0xffff0000u));
-                }
-                if (nv < kPage) {
-                    // rows past the end of the sequence hold stale bytes: zero their weights' factors
-                    const uint32_t ma = (2 * tig < nv ? 0x0000ffffu : 0u) | (2 * tig + 1 < nv ? 0xffff0000u : 0u);
-                    const uint32_t mb = (2 * tig + 8 < nv ? 0x0000ffffu : 0u) | (2 * tig + 9 < nv ? 0xffff0000u : 0u);
-#pragma unroll
-                    for (int g = 0; g < NG; ++g) {
-                        vsa[g] &= ma;
-                        vsb[g] &= mb;
-                    }
-                    vma &= ma;
-                    vmb &= mb;
-                }
-
-                // P~ in the PV B-operand layout: column gid (even) = head gid/2 of the n-tile
-                uint32_t pb0[NT], pb1[NT];
-                const int srcA = (2 * tig) * 4 + (gid >> 1), srcB = srcA + 4;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const uint32_t pp = pack_f16x2(p0[nt], p1[nt]);   // lo: token gid, hi: token gid+8
-                    const uint32_t w0 = __shfl_sync(0xffffffffu, pp, srcA);
-                    const uint32_t w1 = __shfl_sync(0xffffffffu, pp, srcB);
-                    pb0[nt] = (gid & 1) ? 0u : prmt(w0, w1, 0x5410u);   // tokens 2tig, 2tig+1
-                    pb1[nt] = (gid & 1) ? 0u : prmt(w0, w1, 0x7632u);   // tokens 2tig+8, 2tig+9
-                    mma_f16(macc[nt], vma, 0u, vmb, 0u, pb0[nt], pb1[nt]);
-                }
-#pragma unroll
-                for (int w2 = 0; w2 < NG; ++w2) {       // word w2 holds m-tiles 2*w2 and 2*w2+1 (= group w2)
-                    const uint32_t x = vw[w2], xh = x >> 10;
-                    const uint32_t e0 = code_field<0>(x, xh), e2 = code_field<2>(x, xh);
-                    const uint32_t e1 = code_field<1>(x, xh), e3 = code_field<3>(x, xh);
-                    const uint32_t f0 = code_field<4>(x, xh), f2 = code_field<6>(x, xh);
-                    const uint32_t f1 = code_field<5>(x, xh), f3 = code_field<7>(x, xh);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint32_t b0 = hmul2(pb0[nt], vsa[w2]), b1 = hmul2(pb1[nt], vsb[w2]);
-                        mma_f16(oacc[nt][2 * w2], e0, e2, e1, e3, b0, b1);
-                        mma_f16(oacc[nt][2 * w2 + 1], f0, f2, f1, f3, b0, b1);
+                if (ub < u1) {
+                    if (ub >= run_end) switch_run(ub);
+                    const uint32_t s2[1] = {sa + pair_gap};
+                    if (vv >> 8) {
+                        if (ub == partial_u) consume<D, G, 1, true>(s2, nv_last, st, lane, lo, p.v_ch0);
+                        else consume<D, G, 1, false>(s2, kPage, st, lane, lo, p.v_ch0);
                     }
                 }
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        mbar_arrive_if(&empty[stage], lane == 0);
+        if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+        }
     }
     if (ok && cur_run >= 0) finish_run(cur_run);
 }
@@ -528,7 +613,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(128) k_combine(const int *__restrict__ seq_lens, int batch, int hq, int hkv,
-                                                 int hc, int pps, int nchunks, int num_ctas,
+                                                 int hc, int pw, int nchunks, int num_ctas,
                                                  const float *__restrict__ part, float *__restrict__ out) {
     __shared__ long long sh_U, sh_ur;
     __shared__ int sh_np;
@@ -567,21 +652,21 @@ __global__ void __launch_bounds__(128) k_combine(const int *__restrict__ seq_len
     float mstar = -INFINITY;
     for (int c = cf; c <= cl; ++c)
         if (has_units(c))
-            for (int s = 0; s < pps; ++s)
-                mstar = fmaxf(mstar, part[record_index(c + r, s, jl, hh, pps, hc, G) * (2 + D)]);
+            for (int s = 0; s < pw; ++s)
+                mstar = fmaxf(mstar, part[record_index(c + r, s, jl, hh, pw, hc, G) * (2 + D)]);
     float den = 0.0f;
     for (int c = cf; c <= cl; ++c)
         if (has_units(c))
-            for (int s = 0; s < pps; ++s) {
-            const float *rec = part + record_index(c + r, s, jl, hh, pps, hc, G) * (2 + D);
+            for (int s = 0; s < pw; ++s) {
+            const float *rec = part + record_index(c + r, s, jl, hh, pw, hc, G) * (2 + D);
             if (rec[0] != -INFINITY) den += rec[1] * exp2f(rec[0] - mstar);
         }
     for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
         float num = 0.0f;
         for (int c = cf; c <= cl; ++c)
             if (has_units(c))
-                for (int s = 0; s < pps; ++s) {
-                const float *rec = part + record_index(c + r, s, jl, hh, pps, hc, G) * (2 + D);
+                for (int s = 0; s < pw; ++s) {
+                const float *rec = part + record_index(c + r, s, jl, hh, pw, hc, G) * (2 + D);
                 if (rec[0] != -INFINITY) num += rec[2 + ch] * exp2f(rec[0] - mstar);
             }
         o[ch] = den > 0.0f ? num / den : 0.0f;

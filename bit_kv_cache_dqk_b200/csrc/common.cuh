@@ -22,8 +22,8 @@ struct Layout {
     int d, ng, kc, ks, km, k0, vc, vs, vm, v0, bytes;
 };
 
-__host__ __device__ __forceinline__ Layout make_layout(int d, int v_ch0) {
-    Layout L;
+__host__ __device__ constexpr Layout make_layout(int d, int v_ch0) {
+    Layout L{};
     L.d = d;
     L.ng = d / kGroup;
     L.kc = 0;
@@ -39,16 +39,20 @@ __host__ __device__ __forceinline__ Layout make_layout(int d, int v_ch0) {
 }
 
 // Key code of (token t, channel c): byte offset of its 32-bit word inside the
-// K code section and the bit of its 2-bit field.  The order is the A operand
-// of an m16n8k16 tile with tokens as rows and channels as columns: word W of
-// a lane holds group W (k-steps s = 0, 1) for token rows t%8 and t%8 + 8.
+// K code section and the bit of its 2-bit field.  The order is the u8 A
+// operand of m16n8k32 tiles with tokens as rows and the 32 channels of one
+// group as columns: register r (row t%8 + 8*(r&1), columns 16*(r>>1) +
+// 4*(lane%4) + byte) of group g sits in field g (NG = 4) of that byte, so one
+// AND with 0x03030303 << 2g yields the operand with values code * 4^g.  With
+// NG = 2 the registers r >= 2 take fields 2 and 3 of the words of r - 2.
 __host__ __device__ __forceinline__ void kcode_pos(int ng, int t, int c, int &word_off, int &bit) {
-    int g = c >> 5, cc = c & 31, s = cc >> 4, cb = (cc >> 3) & 1, tig = (cc & 7) >> 1, e = cc & 1;
-    int gid = t & 7, tr = t >> 3;
-    int lane = gid * 4 + tig;
-    int q = ((g * 2 + s) * 2 + cb) * 2 + tr;
-    word_off = (lane * ng + (q >> 3)) * 4;
-    bit = e * 16 + 2 * (q & 7);
+    const int g = c >> 5, cc = c & 31;
+    const int r = 2 * (cc >> 4) + (t >> 3);
+    const int lane = 4 * (t & 7) + ((cc & 15) >> 2);
+    const int j = cc & 3;
+    const int W = r % ng, f = g + ng * (r / ng);
+    word_off = (lane * ng + W) * 4;
+    bit = 8 * j + 2 * f;
 }
 
 // Value code of (token t, channel c): the A operand of an m16n8k16 tile with

@@ -44,11 +44,11 @@ int device_sms() {
 // Decode plan and workspace layout: [header | qf | qm | q0 | partial records],
 // every section 256-byte aligned.
 struct DecodePlan {
-    int d, G, NT, NG, hc, pps, nchunks, num_ctas, stages, bb;
-    size_t off_qf, off_qm, off_q0, off_part, bytes, smem;
+    int d, G, NT, NG, hc, pps, pw, nchunks, num_ctas, stages, bb;
+    size_t off_qf, off_qk, off_qm, off_q0, off_part, bytes, smem;
 };
 
-constexpr int kMaxAttendCtas = 320;
+constexpr int kMaxAttendCtas = 160;   // >= the 148 SMs of a B200; larger parts run 160 persistent CTAs
 
 bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.d = L->head_dim;
@@ -63,24 +63,29 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
         if (hkv % kConsumerWarps) return false;
         P.hc = kConsumerWarps;
     }
-    P.pps = kConsumerWarps / P.hc;
+    P.pps = kStageBlocks / P.hc;    // pages per stage
+    P.pw = kConsumerWarps / P.hc;   // warps per kv head (each takes 2 pages of a stage)
     P.nchunks = hkv / P.hc;
+    if ((long long)batch * P.nchunks * (L->num_pages + 1) >= (1LL << 31)) return false;
     // Records are sized for kMaxAttendCtas so the workspace size does not depend
     // on the device; the launch (check_decode) uses one CTA per SM up to that bound.
     P.num_ctas = kMaxAttendCtas;
     P.bb = make_layout(P.d, L->v_ch0_protect).bytes;
-    const size_t stage_bytes = (size_t)kConsumerWarps * P.bb;
-    const size_t per_stage = stage_bytes + 2 * sizeof(uint64_t) + 8;
-    const size_t budget = 227 * 1024 - 64;
-    P.stages = (int)std::min<size_t>(kMaxStages, budget / per_stage);
-    P.smem = P.stages * per_stage + 16;
+    // shared memory: ring stages | mbarriers | valid flags | abort flag
+    const size_t stage_bytes = (size_t)kStageBlocks * P.bb;
+    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * kStageBlocks + 16;
+    const size_t budget = 227 * 1024;
+    P.stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / stage_bytes);
+    if (P.stages < 2) return false;
+    P.smem = P.stages * stage_bytes + fixed;
     const size_t R = (size_t)batch * P.nchunks;
     const size_t bj = (size_t)batch * hkv;
     P.off_qf = 256;
-    P.off_qm = round_up(P.off_qf + bj * P.NT * P.NG * 2 * 32 * sizeof(uint2), 256);
+    P.off_qk = round_up(P.off_qf + bj * P.NT * P.NG * 32 * sizeof(uint2), 256);
+    P.off_qm = round_up(P.off_qk + bj * P.NT * P.NG * 4 * sizeof(float), 256);
     P.off_q0 = round_up(P.off_qm + bj * P.NT * 32 * sizeof(uint32_t), 256);
     P.off_part = round_up(P.off_q0 + (size_t)batch * L->num_q_heads * sizeof(float), 256);
-    const size_t records = ((size_t)kMaxAttendCtas + R - 1) * P.pps * P.hc * P.G;
+    const size_t records = ((size_t)kMaxAttendCtas + R - 1) * P.pw * P.hc * P.G;
     P.bytes = round_up(P.off_part + records * (2 + P.d) * sizeof(float), 256);
     return true;
 }
@@ -139,7 +144,7 @@ dqk_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 template <int D>
 dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
     const int G = P.G;
-    const size_t smem = (size_t)D * (D + 1) * 4 + (size_t)G * D * 4 + (size_t)G * P.NG * 4 + (size_t)G * D;
+    const size_t smem = (size_t)D * (D + 1) * 4 + (size_t)G * D * 4 + (size_t)G * P.NG * 8 + (size_t)G * D * 3;
     if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
@@ -147,8 +152,8 @@ dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
     const int threads = (G < 4 ? 4 : G) * 32;
     k_qprep<D><<<dim3(a.L->num_kv_heads, a.batch), threads, smem, a.stream>>>(
         a.L->t_q, a.q, a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qscale,
-        reinterpret_cast<uint2 *>(ws + P.off_qf), reinterpret_cast<uint32_t *>(ws + P.off_qm),
-        reinterpret_cast<float *>(ws + P.off_q0), a.sel_out);
+        reinterpret_cast<uint2 *>(ws + P.off_qf), reinterpret_cast<float *>(ws + P.off_qk),
+        reinterpret_cast<uint32_t *>(ws + P.off_qm), reinterpret_cast<float *>(ws + P.off_q0), a.sel_out);
     return launch_status();
 }
 
@@ -163,6 +168,7 @@ dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
     prm.seq_lens = a.seq_lens;
     prm.page_table = a.page_table;
     prm.qf = reinterpret_cast<const uint2 *>(ws + P.off_qf);
+    prm.qk = reinterpret_cast<const float *>(ws + P.off_qk);
     prm.qm = reinterpret_cast<const uint32_t *>(ws + P.off_qm);
     prm.q0 = reinterpret_cast<const float *>(ws + P.off_q0);
     prm.part = reinterpret_cast<float *>(ws + P.off_part);
@@ -171,6 +177,7 @@ dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
     prm.hkv = a.L->num_kv_heads;
     prm.hc = P.hc;
     prm.pps = P.pps;
+    prm.pw = P.pw;
     prm.nchunks = P.nchunks;
     prm.max_pages = a.max_pages;
     prm.bb = P.bb;
@@ -194,7 +201,7 @@ template <int D>
 dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
     char *ws = static_cast<char *>(a.ws);
     return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(D), 0, a.stream, a.seq_lens, a.batch,
-                      a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pps, P.nchunks, P.num_ctas,
+                      a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pw, P.nchunks, P.num_ctas,
                       reinterpret_cast<const float *>(ws + P.off_part), a.out);
 }
 

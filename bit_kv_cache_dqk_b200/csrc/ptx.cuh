@@ -78,6 +78,20 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D += A * B, m16n8k32, u8 x s8 operands, s32 accumulate.
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 1.5 * 2^23: an int32 accumulator started at its bit pattern (0x4B400000)
+// reads as the float kMagicF + sum, exactly, while |sum| < 2^22.
+constexpr int kMagicI = 0x4B400000;
+constexpr float kMagicF = 12582912.0f;
+
 // Two 2-bit codes at bit 2P of each 16-bit half of x -> an f16x2 holding the
 // exact values 0..3.  OR-ing the field into the mantissa of 2^(10-2P) gives
 // 2^(10-2P) + code (the field's weight equals one ulp there); subtracting
@@ -121,6 +135,62 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
+}
+
+// 2^x, MUFU approximation (relative error ~2^-22); -inf -> 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Non-negative fp16 values of an f16x2 word as fp32 numbers scaled by 2^-112:
+// the 15 value bits moved to bit 13 are a binary32 pattern whose exponent bias
+// differs by 127 - 15 = 112 (subnormal fp16 lands on subnormal fp32, so the
+// scaling is exact for every non-negative fp16).  Integer ops only.
+__device__ __forceinline__ float f16lo_scaled(uint32_t w) { return __uint_as_float((w << 13) & 0x0fffe000u); }
+__device__ __forceinline__ float f16hi_scaled(uint32_t w) { return __uint_as_float((w >> 3) & 0x0fffe000u); }
+constexpr float kTwoPow112 = 0x1p112f;
+
+// Shared-memory loads by 32-bit shared-window address.  volatile keeps them
+// after the mbarrier wait that makes the stage's bytes visible.
+__device__ __forceinline__ uint4 ld_s128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 ld_s64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_s32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_s16(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_s8(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
+__device__ __forceinline__ void st_s128(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+}
+
+// mbarrier arrive by the lanes where `pred` holds (predicated, no branch).
+__device__ __forceinline__ void mbar_arrive_if(uint64_t *bar, bool pred) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(
+            smem_addr(bar)),
+        "r"((uint32_t)pred)
+        : "memory");
 }
 
 __device__ __forceinline__ uint4 lds128(const void *p) { return *reinterpret_cast<const uint4 *>(p); }

@@ -48,21 +48,20 @@ __device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[E], in
     }
 }
 
-// Query fragments of one (sequence, kv head), consumed by k_attend:
-//   qf  [B*Hkv][NT][NG][2][32] uint2   per lane: the f16x2 pairs (b0b1, b2b3)
-//       of the QK B operand of k-step s of group g: rows = channels
-//       32g+16s+2*tig+{0,1} (and +8), column n = gid -> query head 4*nt + gid/2,
-//       gid even: fp16 high part, odd: low part of qs = q'_c * log2(e)/sqrt(d)
-//       on kept channels c >= 1, 0 elsewhere.
+// Query fragments of one (sequence, kv head), consumed by k_attend, with
+// qs = q'_c * log2(e)/sqrt(d) on kept channels c >= 1 (0 elsewhere):
+//   qf  [B*Hkv][NT][NG][32] uint2      per lane: the two s8x4 registers of the
+//       m16n8k32 B operand of group g: rows (channels of the group) 4*tig..+3
+//       and 16+4*tig..+3, column n = gid -> query head 4*nt + gid/2; gid even:
+//       Q1 = rne(qs/sigma), odd: Q2 = clamp(rne((qs/sigma - Q1)*256)), with
+//       sigma = max_g |qs| / 127 rounded up to 22 significant bits, so
+//       qs ~= sigma * (Q1 + Q2/256).
+//   qk  [B*Hkv][NT][NG][4] float       kappa = sigma / 4^g per head (the key
+//       operand of group g carries code * 4^g).
 //   qm  [B*Hkv][NT][32] uint32         per lane: rows 2*tig, 2*tig+1 of the
-//       min-term B operand: Qsum_{g,h} = sum of qs over the group's kept
-//       channels (hi/lo by column parity as above).
+//       fp16 min-term B operand: Qsum_{g,h} = sum of qs over the group's kept
+//       channels (high part for even gid, low part for odd gid).
 //   q0  [B][Hq] float                  qs of channel 0 (always kept).
-template <int D>
-struct QFrag {
-    static constexpr int NG = D / 32;
-};
-
 __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
     const __half hi = __float2half_rn(x);
     if (piece == 0) return __half_as_ushort(hi);
@@ -72,8 +71,9 @@ __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
 template <int D>
 __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, const void *__restrict__ q,
                                               int dtype, int hq, int hkv, int pct, float qscale,
-                                              uint2 *__restrict__ qf, uint32_t *__restrict__ qm,
-                                              float *__restrict__ q0, int16_t *__restrict__ sel_out) {
+                                              uint2 *__restrict__ qf, float *__restrict__ qk,
+                                              uint32_t *__restrict__ qm, float *__restrict__ q0,
+                                              int16_t *__restrict__ sel_out) {
     constexpr int NG = D / 32;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int G = hq / hkv;
@@ -81,7 +81,9 @@ __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, co
     float *tq = reinterpret_cast<float *>(smem_raw);                 // [D][D+1]
     float *qrow = tq + D * (D + 1);                                   // [G][D]  input, then qs
     float *qsum = qrow + G * D;                                       // [G][NG]
-    unsigned char *mask = reinterpret_cast<unsigned char *>(qsum + G * NG);  // [G][D]
+    float *sig = qsum + G * NG;                                       // [G][NG]  sigma
+    signed char *q8 = reinterpret_cast<signed char *>(sig + G * NG);  // [G][2][D] pieces
+    unsigned char *mask = reinterpret_cast<unsigned char *>(q8 + G * 2 * D);  // [G][D]
     const int j = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     grid_dependents_launch();   // the attend kernel may start streaming pages now
@@ -134,26 +136,48 @@ __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, co
             const float v = (keep && c != 0) ? qs : 0.0f;
             qrow[warp * D + c] = v;
             // group sums of the kept, scaled channels (channel 0 excluded)
-            float gs = v;
+            float gs = v, gm = fabsf(v);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+            for (int o = 16; o > 0; o >>= 1) {
+                gs += __shfl_xor_sync(0xffffffffu, gs, o);
+                gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+            }
             if (lane == 0) qsum[warp * NG + m] = gs;
+            // two int8 pieces relative to the group's largest |qs|; sigma rounded
+            // up to 22 significant bits (so 1.5 * 2^23 * sigma / 4^g is exact)
+            float sgm = gm / 127.0f;
+            sgm = __uint_as_float((__float_as_uint(sgm) + 3u) & ~3u);
+            int q1 = 0, q2 = 0;
+            if (sgm > 0.0f) {
+                const float x = v / sgm;
+                q1 = max(-127, min(127, __float2int_rn(x)));
+                q2 = max(-128, min(127, __float2int_rn((x - (float)q1) * 256.0f)));
+            }
+            q8[(warp * 2 + 0) * D + c] = (signed char)q1;
+            q8[(warp * 2 + 1) * D + c] = (signed char)q2;
+            if (lane == 0) sig[warp * NG + m] = sgm;
         }
     }
     __syncthreads();
     // lay out the B-operand fragments
     const size_t bj = (size_t)b * hkv + j;
-    for (int idx = threadIdx.x; idx < NT * NG * 2 * 32; idx += blockDim.x) {
-        const int L = idx & 31, s = (idx >> 5) & 1, g = (idx >> 6) % NG, nt = (idx >> 6) / NG;
+    for (int idx = threadIdx.x; idx < NT * NG * 32; idx += blockDim.x) {
+        const int L = idx & 31, g = (idx >> 5) % NG, nt = (idx >> 5) / NG;
         const int gid = L >> 2, tig = L & 3, hl = 4 * nt + (gid >> 1), piece = gid & 1;
-        const int c0 = 32 * g + 16 * s + 2 * tig;
         uint32_t w0 = 0, w1 = 0;
         if (hl < G) {
-            const float *r = &qrow[hl * D];
-            w0 = (uint32_t)f16_piece(r[c0], piece) | ((uint32_t)f16_piece(r[c0 + 1], piece) << 16);
-            w1 = (uint32_t)f16_piece(r[c0 + 8], piece) | ((uint32_t)f16_piece(r[c0 + 9], piece) << 16);
+            const unsigned char *r = reinterpret_cast<const unsigned char *>(&q8[(hl * 2 + piece) * D + 32 * g]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                w0 |= (uint32_t)r[4 * tig + i] << (8 * i);
+                w1 |= (uint32_t)r[16 + 4 * tig + i] << (8 * i);
+            }
         }
-        qf[(((bj * NT + nt) * NG + g) * 2 + s) * 32 + L] = make_uint2(w0, w1);
+        qf[((bj * NT + nt) * NG + g) * 32 + L] = make_uint2(w0, w1);
+    }
+    for (int idx = threadIdx.x; idx < NT * NG * 4; idx += blockDim.x) {
+        const int hh = idx & 3, g = (idx >> 2) % NG, nt = (idx >> 2) / NG, hl = 4 * nt + hh;
+        qk[((bj * NT + nt) * NG + g) * 4 + hh] = hl < G ? sig[hl * NG + g] * (1.0f / (float)(1 << (2 * g))) : 0.0f;
     }
     for (int idx = threadIdx.x; idx < NT * 32; idx += blockDim.x) {
         const int L = idx & 31, nt = idx >> 5;

@@ -95,9 +95,9 @@ typedef struct {
  * sections are in the operand order of the decode kernel's tensor-core
  * tiles, each lane of a warp reading 4*NG contiguous bytes):
  *   KC = 0            K codes, 4*d bytes: code of (token t, channel c) is in the
- *                     32-bit word at KC + 4*(lane*NG + W), bit 16*e + 2*i, with
- *                     g=c/32, s=(c%32)/16, cb=(c%16)/8, tig=(c%8)/2, e=c%2,
- *                     lane=4*(t%8)+tig, q=((2g+s)*2+cb)*2+t/8, W=q/8, i=q%8.
+ *                     32-bit word at KC + 4*(lane*NG + W), bit 8*j + 2*f, with
+ *                     g=c/32, cc=c%32, r=2*(cc/16)+t/8, lane=4*(t%8)+(cc%16)/4,
+ *                     j=cc%4, W=r%NG, f=g+NG*(r/NG).
  *   KS = 4d           K scale fp16 [t][g]
  *   KM = KS + 32*NG   K min   fp16 [t][g]
  *   K0 = KM + 32*NG   K channel 0 BF16, token t at index 2*(t%8) + t/8

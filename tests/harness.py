@@ -137,11 +137,12 @@ def _code_tables(d):
     vb = np.zeros((16, d), np.int64)
     for t in range(16):
         for c in range(d):
-            g, s, cb, tig, e = c // 32, (c % 32) // 16, (c % 16) // 8, (c % 8) // 2, c % 2
-            lane = 4 * (t % 8) + tig
-            q = ((2 * g + s) * 2 + cb) * 2 + t // 8
-            kw[t, c] = lane * ng + q // 8
-            kb[t, c] = 16 * e + 2 * (q % 8)
+            g, cc = c // 32, c % 32
+            r = 2 * (cc // 16) + t // 8
+            lane = 4 * (t % 8) + (cc % 16) // 4
+            j = cc % 4
+            kw[t, c] = lane * ng + r % ng
+            kb[t, c] = 8 * j + 2 * (g + ng * (r // ng))
             m, cr, tb, tig, e = c // 16, (c % 16) // 8, t // 8, (t % 8) // 2, t % 2
             lane = 4 * (c % 8) + tig
             q = (2 * m + cr) * 2 + tb
