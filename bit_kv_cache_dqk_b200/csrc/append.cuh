@@ -5,6 +5,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace dqk {
 
@@ -12,8 +13,8 @@ template <int D>
 struct AppendSmem {
     static constexpr int NG = D / kGroup;
     static constexpr int kMaxBlockBytes = 8 * D + 128 * NG + 64;
-    float tk[D * (D + 1)];           // T_K[j], rows padded by one float (bank-conflict free)
-    float x[kPage][D];               // one input row per warp
+    double tk[D * (D + 1)];          // T_K[j] in fp64, rows padded by one element
+    double x[kPage][D];              // one input row per warp, fp64
     uint8_t kcode[kPage][D];         // plain codes of the page being rewritten
     uint8_t vcode[kPage][D];
     uint16_t kscale[kPage][NG], kmin[kPage][NG], kch0[kPage];
@@ -173,9 +174,7 @@ __global__ void __launch_bounds__(512) k_quant_pack(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layout L = make_layout(D, v_ch0);
 
-    const float *T = t_k + (size_t)j * D * D;
-    for (int idx = threadIdx.x; idx < D * D; idx += blockDim.x)
-        S.tk[(idx / D) * (D + 1) + (idx % D)] = T[idx];
+    stage_f64_padded<D>(S.tk, t_k + (size_t)j * D * D);
     __syncthreads();
 
     const int items = batch * slots_per_seq;
@@ -203,17 +202,21 @@ __global__ void __launch_bounds__(512) k_quant_pack(
         if (pos >= L0 && pos < L0 + n) {
             const size_t base = ((size_t)(row0 + (pos - L0)) * hkv + j) * D;
 #pragma unroll
-            for (int m = 0; m < NG; ++m) S.x[warp][lane + 32 * m] = load_elem(kin, dtype, base + lane + 32 * m);
+            for (int m = 0; m < NG; ++m) S.x[warp][lane + 32 * m] = (double)load_elem(kin, dtype, base + lane + 32 * m);
             __syncwarp();
             float kp[NG];
+            double acc[NG];
 #pragma unroll
-            for (int m = 0; m < NG; ++m) {
-                const float *row = &S.tk[(lane + 32 * m) * (D + 1)];
-                double s = 0.0;
-#pragma unroll 8
-                for (int i = 0; i < D; ++i) s = fma((double)row[i], (double)S.x[warp][i], s);
-                kp[m] = __double2float_rn(s);
+            for (int m = 0; m < NG; ++m) acc[m] = 0.0;
+            // NG independent sequential sums (ascending i), interleaved
+#pragma unroll 4
+            for (int i = 0; i < D; ++i) {
+                const double xi = S.x[warp][i];
+#pragma unroll
+                for (int m = 0; m < NG; ++m) acc[m] = fma(S.tk[(lane + 32 * m) * (D + 1) + i], xi, acc[m]);
             }
+#pragma unroll
+            for (int m = 0; m < NG; ++m) kp[m] = __double2float_rn(acc[m]);
             quantize_warp<NG>(kp, true, lane, S.kcode[warp], S.kscale[warp], S.kmin[warp], &S.kch0[warp]);
             float vv[NG];
 #pragma unroll

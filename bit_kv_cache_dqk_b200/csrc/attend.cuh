@@ -32,10 +32,15 @@
 #include "common.cuh"
 #include "ptx.cuh"
 
+#ifndef ATTEND_BLOCKS_PER_WARP
+#define ATTEND_BLOCKS_PER_WARP 2
+#endif
+
 namespace dqk {
 
-constexpr int kConsumerWarps = 8;                           // one kv head each (chunks of <= 8 heads)
-constexpr int kStageBlocks = 2 * kConsumerWarps;            // (page, kv head) blocks per stage
+constexpr int kStageBlocks = 16;                            // (page, kv head) blocks per stage
+constexpr int kBlocksPerWarp = ATTEND_BLOCKS_PER_WARP;      // pages of its kv head a warp takes per stage
+constexpr int kConsumerWarps = kStageBlocks / kBlocksPerWarp;
 constexpr int kAttendThreads = (kConsumerWarps + 1) * 32;   // + 1 producer warp
 constexpr int kMaxStages = 8;                               // ring depth cap
 constexpr uint64_t kWaitLimitNs = 1000000000ull;            // 1 s: a stuck pipeline reports DQK_ERR_TIMEOUT
@@ -122,8 +127,6 @@ struct AttendTile {
 template <int D, int G>
 struct WarpState {
     using T = AttendTile<D, G>;
-    uint2 qbi[T::NT][T::NG];       // QK B fragments (s8 pieces Q1/Q2 of the kept, scaled q')
-    float4 kap[T::NT][T::NG];      // kappa, kappa/256, -M*kappa, -M*kappa/256 of this thread's head
     uint32_t qmin[T::NT];          // min-term B fragment
     float q0v[T::NT];              // scaled q'_0 of this thread's head
     float m_run[T::NT];            // running max (log2 units) of this thread's head
@@ -140,14 +143,16 @@ struct LaneOffsets {
     uint32_t tig16;    // (lane%4) * 16: V scale pairs of tokens 2tig.. (+64: 2tig+8..)
     uint32_t vmin;     // V min pair of row min(gid, NG-1), tokens 2tig, 2tig+1
     int srcA;          // lane holding p of (token 2tig, head gid/2); +4: token 2tig+1
+    uint32_t sq;       // shared address of this lane's QK B fragments: [NT][NG][32 lanes] uint2
+    uint32_t sk;       // shared address of this thread's head constants: [NT][NG][4 heads] float4
     uint32_t ones_lane, vmin_mask, kmin_mask;
 };
 
 // NB (page, kv head) blocks at shared addresses sb[]: 16 tokens x G query heads
 // each, same run.  MASKED (NB == 1 only): only the first nv tokens are valid.
-template <int D, int G, int NB, bool MASKED>
+template <int D, int G, bool VCH0, int NB, bool MASKED>
 __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpState<D, G> &st, int lane,
-                                        const LaneOffsets &o, int v_ch0) {
+                                        const LaneOffsets &o) {
     using T = AttendTile<D, G>;
     constexpr int NG = T::NG, NT = T::NT;
     constexpr Layout Ly = make_layout(D, 0);   // section offsets do not depend on v_ch0 (V0 is last)
@@ -186,8 +191,7 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
         for (int nt = 0; nt < NT; ++nt) {
             a0[b][nt] = 0.0f;
             a1[b][nt] = 0.0f;
-            cmin[b][nt][0] = cmin[b][nt][1] = cmin[b][nt][2] = cmin[b][nt][3] = 0.0f;
-            mma_f16(cmin[b][nt], km0[b], km1[b], 0u, 0u, st.qmin[nt], 0u);
+            mma_f16_zero(cmin[b][nt], km0[b], km1[b], 0u, 0u, st.qmin[nt], 0u);
         }
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
@@ -206,10 +210,13 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
             const float sbv = (g & 1) ? f16hi_scaled(ks1[b][g >> 1]) : f16lo_scaled(ks1[b][g >> 1]);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                int dg[4] = {kMagicI, kMagicI, kMagicI, kMagicI};
-                mma_u8s8(dg, A0, A1, A2, A3, st.qbi[nt][g].x, st.qbi[nt][g].y);
+                int dg[4];
+                const uint2 qb = ld_s64(o.sq + (nt * NG + g) * 256);
+                mma_u8s8(dg, A0, A1, A2, A3, qb.x, qb.y, kMagicI);
                 // (M + I) * kappa - M * kappa = I * kappa, one rounding
-                const float4 kp = st.kap[nt][g];
+                const uint4 kpu = ld_s128(o.sk + (nt * NG + g) * 64);
+                const float4 kp = make_float4(__uint_as_float(kpu.x), __uint_as_float(kpu.y),
+                                              __uint_as_float(kpu.z), __uint_as_float(kpu.w));
                 a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[0]), kp.x, kp.z), a0[b][nt]);
                 a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[1]), kp.y, kp.w), a0[b][nt]);
                 a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[2]), kp.x, kp.z), a1[b][nt]);
@@ -279,7 +286,7 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
         const uint32_t avm = sb[b] + o.vmin;
         uint32_t vma = (ld_s32(avm + Ly.vm) & o.vmin_mask) | o.ones_lane;
         uint32_t vmb = (ld_s32(avm + Ly.vm + 16 * NG) & o.vmin_mask) | o.ones_lane;
-        if (v_ch0) {
+        if constexpr (VCH0) {
             const Layout L1 = make_layout(D, 1);
             const uint32_t a = ld_s32(sb[b] + L1.v0 + tig * 4), c = ld_s32(sb[b] + L1.v0 + 16 + tig * 4);
             if (gid == NG + 1) {
@@ -329,7 +336,7 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
     }
 }
 
-template <int D, int G>
+template <int D, int G, bool VCH0>
 __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams p) {
     using T = AttendTile<D, G>;
     constexpr int NG = T::NG, NT = T::NT, NM = T::NM;
@@ -341,6 +348,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     uint64_t *empty = full + kMaxStages;
     unsigned char *valid = reinterpret_cast<unsigned char *>(empty + kMaxStages);   // [kMaxStages][kStageBlocks]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(valid + kMaxStages * kStageBlocks);
+    // per consumer warp: QK B fragments [NT][NG][32] uint2, head constants [NT][NG][4] float4
+    unsigned char *frag_mem = valid + kMaxStages * kStageBlocks + 16;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = p.batch * p.nchunks;
@@ -406,7 +415,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
             if (ubase + 32 < u1) off_next = fetch(ubase + 32);
             for (; it < iters && u0 + it * pps < ubase + 32; ++it) {
                 int good = 1;
-                if (lane == 0) good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs) && !*abort_flag;
+                if (lane == 0)
+                    good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs, 2000u) && !*abort_flag;
                 if (!__shfl_sync(0xffffffffu, good, 0)) {
                     if (lane == 0) {
                         *abort_flag = 1;
@@ -441,7 +451,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     }
 
     // ---------------------------------------------------------------- consumers
-    // warp: kv head jl of the chunk, page pair pi of each stage (pages 2pi, 2pi+1)
+    // warp: kv head jl of the chunk, page group pi of each stage (pages kBlocksPerWarp*pi + 0..)
     const int jl = warp % p.hc, pi = warp / p.hc;
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
@@ -486,6 +496,11 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     lo.tig16 = tig * 16;
     lo.vmin = (tig * NG + (gid < NG ? gid : 0)) * 4;
     lo.srcA = (2 * tig) * 4 + (gid >> 1);
+    {
+        unsigned char *mine = frag_mem + (size_t)warp * NT * NG * (32 * 8 + 4 * 16);
+        lo.sq = smem_addr(mine) + lane * 8;
+        lo.sk = smem_addr(mine + NT * NG * 32 * 8) + tig * 16;
+    }
     lo.ones_lane = gid == NG ? 0x3C003C00u : 0u;
     lo.vmin_mask = gid < NG ? 0xffffffffu : 0u;
     lo.kmin_mask = tig < NG / 2 ? 0xffffffffu : 0u;
@@ -498,11 +513,17 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
-                st.qbi[nt][g] = p.qf[((bj * NT + nt) * NG + g) * 32 + lane];
-                const float kappa = p.qk[((bj * NT + nt) * NG + g) * 4 + tig];
-                st.kap[nt][g] = make_float4(kappa, kappa * (1.0f / 256.0f), -kMagicF * kappa,
-                                            -kMagicF * kappa * (1.0f / 256.0f));
+                const uint2 qb = p.qf[((bj * NT + nt) * NG + g) * 32 + lane];
+                st_s64(lo.sq + (nt * NG + g) * 256, qb);
+                if (gid == 0) {
+                    const float kappa = p.qk[((bj * NT + nt) * NG + g) * 4 + tig];
+                    st_s128(lo.sk + (nt * NG + g) * 64,
+                            make_uint4(__float_as_uint(kappa), __float_as_uint(kappa * (1.0f / 256.0f)),
+                                       __float_as_uint(-kMagicF * kappa),
+                                       __float_as_uint(-kMagicF * kappa * (1.0f / 256.0f))));
+                }
             }
+            __syncwarp();
             st.qmin[nt] = p.qm[(bj * NT + nt) * 32 + lane];
             const int hh = 4 * nt + tig;
             st.q0v[nt] = hh < G ? p.q0[(size_t)b * p.hq + j * G + hh] : 0.0f;
@@ -536,7 +557,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
                 for (int m = 0; m < NM; ++m) {
                     const int c0 = 16 * m + gid, c1 = c0 + 8;
                     const float mt = minterm[m >> 1];
-                    rec[2 + c0] = (p.v_ch0 && c0 == 0) ? v0t : st.oacc[nt][m][0] + mt;
+                    rec[2 + c0] = (VCH0 && c0 == 0) ? v0t : st.oacc[nt][m][0] + mt;
                     rec[2 + c1] = st.oacc[nt][m][2] + mt;
                 }
             }
@@ -561,9 +582,9 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     bool ok = true;
     int stage = 0;
     uint32_t phase = 0;
-    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((2 * pi * p.hc + jl) * p.bb);
+    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((kBlocksPerWarp * pi * p.hc + jl) * p.bb);
     const uint32_t pair_gap = (uint32_t)(p.hc * p.bb);
-    const uint32_t valid_addr = smem_addr(valid) + 2 * pi;
+    const uint32_t valid_addr = smem_addr(valid) + kBlocksPerWarp * pi;
     for (int it = 0; it < iters; ++it) {
         if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
             if (lane == 0) {
@@ -573,27 +594,38 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
             ok = false;
             break;
         }
-        const int ua = u0 + it * pps + 2 * pi, ub = ua + 1;
+        const int ua = u0 + it * pps + kBlocksPerWarp * pi;
         if (ua < u1) {
-            const uint32_t vv = ld_s16(valid_addr + stage * kStageBlocks);   // flags of slots 2pi, 2pi+1 (even address)
-            if (ua >= run_end) switch_run(ua);
             const uint32_t sa = blk_a + (uint32_t)stage * stage_bytes;
-            if (ub < run_end && ub < u1 && ub != partial_u && vv == 0x0101u) {
-                const uint32_t sbb[2] = {sa, sa + pair_gap};
-                consume<D, G, 2, false>(sbb, kPage, st, lane, lo, p.v_ch0);
-            } else {
-                const uint32_t s1[1] = {sa};
-                if (vv & 0xffu) {
-                    if (ua == partial_u) consume<D, G, 1, true>(s1, nv_last, st, lane, lo, p.v_ch0);
-                    else consume<D, G, 1, false>(s1, kPage, st, lane, lo, p.v_ch0);
-                }
-                if (ub < u1) {
-                    if (ub >= run_end) switch_run(ub);
-                    const uint32_t s2[1] = {sa + pair_gap};
-                    if (vv >> 8) {
-                        if (ub == partial_u) consume<D, G, 1, true>(s2, nv_last, st, lane, lo, p.v_ch0);
-                        else consume<D, G, 1, false>(s2, kPage, st, lane, lo, p.v_ch0);
+            if constexpr (kBlocksPerWarp == 2) {
+                const int ub = ua + 1;
+                const uint32_t vv = ld_s16(valid_addr + stage * kStageBlocks);   // flags of slots 2pi, 2pi+1
+                if (ua >= run_end) switch_run(ua);
+                if (ub < run_end && ub < u1 && ub != partial_u && vv == 0x0101u) {
+                    const uint32_t sbb[2] = {sa, sa + pair_gap};
+                    consume<D, G, VCH0, 2, false>(sbb, kPage, st, lane, lo);
+                } else {
+                    const uint32_t s1[1] = {sa};
+                    if (vv & 0xffu) {
+                        if (ua == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
+                        else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);
                     }
+                    if (ub < u1) {
+                        if (ub >= run_end) switch_run(ub);
+                        const uint32_t s2[1] = {sa + pair_gap};
+                        if (vv >> 8) {
+                            if (ub == partial_u) consume<D, G, VCH0, 1, true>(s2, nv_last, st, lane, lo);
+                            else consume<D, G, VCH0, 1, false>(s2, kPage, st, lane, lo);
+                        }
+                    }
+                }
+            } else {
+                const uint32_t vv = ld_s8(valid_addr + stage * kStageBlocks);
+                if (ua >= run_end) switch_run(ua);
+                const uint32_t s1[1] = {sa};
+                if (vv) {
+                    if (ua == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
+                    else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);
                 }
             }
         }
@@ -611,17 +643,30 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
 // log-sum-exp combine: out[b][h] = sum_i o_i 2^(m_i - m*) / sum_i l_i 2^(m_i - m*)
 // over the records of every CTA (and page slot) that held pages of (b, h).
 // ---------------------------------------------------------------------------
+constexpr int kCombineChunk = 256;     // records weighted per pass
+constexpr int kCombineThreads = 512;   // channel x record-slice threads
+
+// One CTA per (sequence, query head).  Thread (slice, channel) accumulates the
+// records i = slice (mod slices) of its channel; slices are summed in a fixed
+// order, so the result does not depend on scheduling.
 template <int D>
-__global__ void __launch_bounds__(128) k_combine(const int *__restrict__ seq_lens, int batch, int hq, int hkv,
-                                                 int hc, int pw, int nchunks, int num_ctas,
-                                                 const float *__restrict__ part, float *__restrict__ out) {
+__global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restrict__ seq_lens, int batch, int hq,
+                                                             int hkv, int hc, int pw, int nchunks, int num_ctas,
+                                                             const float *__restrict__ part, float *__restrict__ out) {
+    constexpr int kSlices = kCombineThreads / D;
     __shared__ long long sh_U, sh_ur;
     __shared__ int sh_np;
+    __shared__ float sh_w[kCombineChunk];
+    __shared__ int sh_rec[kCombineChunk];
+    __shared__ float sh_dpart[kCombineThreads / 32];
+    __shared__ float sh_acc[kSlices][D];
+    __shared__ float sh_m;
     const int h = blockIdx.x, b = blockIdx.y;
     const int G = hq / hkv, j = h / G, chunk = j / hc, jl = j % hc, hh = h % G;
     const int r = b * nchunks + chunk, R = batch * nchunks;
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ch = threadIdx.x % D, slice = threadIdx.x / D;
+    if (warp == 0) {
         const long long U = warp_total_units(seq_lens, nchunks, R, lane);
         long long base = 0;   // start unit of run r
         for (int r0 = 0; r0 < r; r0 += 32) {
@@ -643,33 +688,63 @@ __global__ void __launch_bounds__(128) k_combine(const int *__restrict__ seq_len
     const int np = sh_np;
     float *o = out + ((size_t)b * hq + h) * D;
     if (np == 0) {
-        for (int c = threadIdx.x; c < D; c += blockDim.x) o[c] = 0.0f;
+        if (slice == 0) o[ch] = 0.0f;
         return;
     }
+    // records of this (run, head): CTAs cf..cl that own units of the run (CTAs
+    // with an empty unit range wrote none), each with pw warp-pair records
     const int cf = (int)cta_of_unit(ur, U, num_ctas), cl = (int)cta_of_unit(ur + np - 1, U, num_ctas);
-    // CTAs with an empty unit range (more CTAs than units) wrote no records
-    auto has_units = [&](int c) { return (long long)c * U / num_ctas < ((long long)c + 1) * U / num_ctas; };
-    float mstar = -INFINITY;
-    for (int c = cf; c <= cl; ++c)
-        if (has_units(c))
-            for (int s = 0; s < pw; ++s)
-                mstar = fmaxf(mstar, part[record_index(c + r, s, jl, hh, pw, hc, G) * (2 + D)]);
-    float den = 0.0f;
-    for (int c = cf; c <= cl; ++c)
-        if (has_units(c))
-            for (int s = 0; s < pw; ++s) {
-            const float *rec = part + record_index(c + r, s, jl, hh, pw, hc, G) * (2 + D);
-            if (rec[0] != -INFINITY) den += rec[1] * exp2f(rec[0] - mstar);
+    const int nrec = (cl - cf + 1) * pw;
+    auto rec_at = [&](int i, bool &ok) -> size_t {
+        const int c = cf + i / pw, s = i % pw;
+        ok = (long long)c * U / num_ctas < ((long long)c + 1) * U / num_ctas;
+        return record_index(c + r, s, jl, hh, pw, hc, G);
+    };
+    if (warp == 0) {       // global max over all records
+        float m = -INFINITY;
+        for (int i = lane; i < nrec; i += 32) {
+            bool ok;
+            const size_t ri = rec_at(i, ok);
+            if (ok) m = fmaxf(m, part[ri * (2 + D)]);
         }
-    for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0) sh_m = m;
+    }
+    __syncthreads();
+    const float mstar = sh_m;
+    float acc = 0.0f, dsum = 0.0f;
+    for (int i0 = 0; i0 < nrec; i0 += kCombineChunk) {
+        const int n = min(kCombineChunk, nrec - i0);
+        float dpart = 0.0f;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            bool ok;
+            const size_t ri = rec_at(i0 + i, ok);
+            const float mi = ok ? part[ri * (2 + D)] : -INFINITY;
+            const float w = mi == -INFINITY ? 0.0f : exp2f(mi - mstar);
+            sh_w[i] = w;
+            sh_rec[i] = ok ? (int)ri : -1;
+            if (w != 0.0f) dpart += w * part[ri * (2 + D) + 1];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dpart += __shfl_xor_sync(0xffffffffu, dpart, off);
+        if (lane == 0) sh_dpart[warp] = dpart;
+        __syncthreads();
+        for (int k = 0; k < kCombineThreads / 32; ++k) dsum += sh_dpart[k];   // fixed order
+#pragma unroll 4
+        for (int i = slice; i < n; i += kSlices) {
+            const float w = sh_w[i];
+            if (w != 0.0f) acc = fmaf(w, part[(size_t)sh_rec[i] * (2 + D) + 2 + ch], acc);
+        }
+        __syncthreads();
+    }
+    sh_acc[slice][ch] = acc;
+    __syncthreads();
+    if (slice == 0) {
         float num = 0.0f;
-        for (int c = cf; c <= cl; ++c)
-            if (has_units(c))
-                for (int s = 0; s < pw; ++s) {
-                const float *rec = part + record_index(c + r, s, jl, hh, pw, hc, G) * (2 + D);
-                if (rec[0] != -INFINITY) num += rec[2 + ch] * exp2f(rec[0] - mstar);
-            }
-        o[ch] = den > 0.0f ? num / den : 0.0f;
+#pragma unroll
+        for (int k = 0; k < kSlices; ++k) num += sh_acc[k][ch];
+        o[ch] = dsum > 0.0f ? num / dsum : 0.0f;
     }
 }
 

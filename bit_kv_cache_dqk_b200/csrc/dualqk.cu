@@ -71,9 +71,10 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     // on the device; the launch (check_decode) uses one CTA per SM up to that bound.
     P.num_ctas = kMaxAttendCtas;
     P.bb = make_layout(P.d, L->v_ch0_protect).bytes;
-    // shared memory: ring stages | mbarriers | valid flags | abort flag
+    // shared memory: ring stages | mbarriers | valid flags | abort flag | per-warp query fragments
     const size_t stage_bytes = (size_t)kStageBlocks * P.bb;
-    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * kStageBlocks + 16;
+    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * kStageBlocks + 16 +
+                         (size_t)kConsumerWarps * P.NT * P.NG * (32 * 8 + 4 * 16);
     const size_t budget = 227 * 1024;
     P.stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / stage_bytes);
     if (P.stages < 2) return false;
@@ -144,7 +145,8 @@ dqk_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 template <int D>
 dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
     const int G = P.G;
-    const size_t smem = (size_t)D * (D + 1) * 4 + (size_t)G * D * 4 + (size_t)G * P.NG * 8 + (size_t)G * D * 3;
+    const size_t smem = (size_t)D * (D + 1) * 8 + (size_t)G * D * 8 + (size_t)G * D * 4 + (size_t)G * P.NG * 8 +
+                        (size_t)G * D * 3;
     if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
@@ -157,9 +159,10 @@ dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
     return launch_status();
 }
 
-template <int D, int G>
+template <int D, int G, bool VCH0>
 dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
-    if (cudaFuncSetAttribute(k_attend<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_attend<D, G, VCH0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
+        cudaSuccess)
         return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
     AttendParams prm;
@@ -184,23 +187,29 @@ dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
     prm.v_ch0 = a.L->v_ch0_protect;
     prm.stages = P.stages;
     prm.num_ctas = P.num_ctas;
-    return launch_pdl(k_attend<D, G>, dim3(P.num_ctas), dim3(kAttendThreads), P.smem, a.stream, prm);
+    return launch_pdl(k_attend<D, G, VCH0>, dim3(P.num_ctas), dim3(kAttendThreads), P.smem, a.stream, prm);
+}
+
+template <int D, bool VCH0>
+dqk_status run_attend_v(const DecodeArgs &a, const DecodePlan &P) {
+    switch (P.G) {
+        case 1: return run_attend_g<D, 1, VCH0>(a, P);
+        case 2: return run_attend_g<D, 2, VCH0>(a, P);
+        case 4: return run_attend_g<D, 4, VCH0>(a, P);
+        default: return run_attend_g<D, 8, VCH0>(a, P);
+    }
 }
 
 template <int D>
 dqk_status run_attend(const DecodeArgs &a, const DecodePlan &P) {
-    switch (P.G) {
-        case 1: return run_attend_g<D, 1>(a, P);
-        case 2: return run_attend_g<D, 2>(a, P);
-        case 4: return run_attend_g<D, 4>(a, P);
-        default: return run_attend_g<D, 8>(a, P);
-    }
+    return a.L->v_ch0_protect ? run_attend_v<D, true>(a, P) : run_attend_v<D, false>(a, P);
 }
 
 template <int D>
 dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
     char *ws = static_cast<char *>(a.ws);
-    return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(D), 0, a.stream, a.seq_lens, a.batch,
+    return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(kCombineThreads), 0, a.stream, a.seq_lens,
+                      a.batch,
                       a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pw, P.nchunks, P.num_ctas,
                       reinterpret_cast<const float *>(ws + P.off_part), a.out);
 }
@@ -239,7 +248,7 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    long long gx = (2LL * sms + L->num_kv_heads - 1) / L->num_kv_heads;
+    long long gx = ((long long)sms + L->num_kv_heads - 1) / L->num_kv_heads;   // ~1 CTA per SM (fp64 T_K in smem)
     if (gx > items) gx = items;
     if (gx < 1) gx = 1;
     k_quant_pack<D><<<dim3((unsigned)gx, L->num_kv_heads), 512, smem, stream>>>(

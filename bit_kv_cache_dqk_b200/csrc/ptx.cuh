@@ -45,12 +45,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to `hint_ns` before returning.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase of `parity` to complete, giving up after `limit_ns`.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns,
+                                                  uint32_t hint_ns = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (hint_ns ? mbar_try_wait_hint(bar, parity, hint_ns) : mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
     }
 }
@@ -62,6 +76,42 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
             smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
+}
+
+// 4-byte asynchronous global -> shared copy (no register round trip), and the
+// wait for all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Stage a row-major [n][n] fp32 matrix into shared memory as fp64 (exact),
+// rows padded to n+1 doubles, so the sequential fp64 dot products read their
+// operands without per-use conversions.  n must be a multiple of 4.
+template <int n>
+__device__ __forceinline__ void stage_f64_padded(double *dst, const float *src) {
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    const int n4 = n * n / 4;
+    for (int base = threadIdx.x; base < n4; base += 4 * blockDim.x) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (base + u * blockDim.x < n4) v[u] = s4[base + u * blockDim.x];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int idx4 = base + u * blockDim.x;
+            if (idx4 < n4) {
+                const int e = idx4 * 4, row = e / n, col = e % n;
+                double *d = dst + row * (n + 1) + col;
+                d[0] = (double)v[u].x;
+                d[1] = (double)v[u].y;
+                d[2] = (double)v[u].z;
+                d[3] = (double)v[u].w;
+            }
+        }
+    }
 }
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -78,13 +128,24 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// D += A * B, m16n8k32, u8 x s8 operands, s32 accumulate.
+// D = A * B + C, m16n8k32, u8 x s8 operands, s32 accumulate; C is the same
+// value c in all four elements (kept in registers, no per-use copies).
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
+                                         uint32_t b0, uint32_t b1, int c) {
     asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        "{%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c));
+}
+
+// D = A * B (zero accumulator), m16n8k16 fp16, fp32 result.
+__device__ __forceinline__ void mma_f16_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    const float z = 0.0f;
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
 // 1.5 * 2^23: an int32 accumulator started at its bit pattern (0x4B400000)
@@ -180,6 +241,9 @@ __device__ __forceinline__ uint32_t ld_s8(uint32_t a) {
     return v;
 }
 
+__device__ __forceinline__ void st_s64(uint32_t a, uint2 v) {
+    asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(v.x), "r"(v.y));
+}
 __device__ __forceinline__ void st_s128(uint32_t a, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
 }

@@ -78,8 +78,9 @@ __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, co
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int G = hq / hkv;
     const int NT = G > 4 ? 2 : 1;
-    float *tq = reinterpret_cast<float *>(smem_raw);                 // [D][D+1]
-    float *qrow = tq + D * (D + 1);                                   // [G][D]  input, then qs
+    double *tq = reinterpret_cast<double *>(smem_raw);               // [D][D+1] fp64
+    double *qin = tq + D * (D + 1);                                   // [G][D]   input row, fp64
+    float *qrow = reinterpret_cast<float *>(qin + G * D);             // [G][D]   qs
     float *qsum = qrow + G * D;                                       // [G][NG]
     float *sig = qsum + G * NG;                                       // [G][NG]  sigma
     signed char *q8 = reinterpret_cast<signed char *>(sig + G * NG);  // [G][2][D] pieces
@@ -87,13 +88,12 @@ __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, co
     const int j = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     grid_dependents_launch();   // the attend kernel may start streaming pages now
-    const float *T = t_q + (size_t)j * D * D;
-    for (int idx = threadIdx.x; idx < D * D; idx += blockDim.x) tq[(idx / D) * (D + 1) + (idx % D)] = T[idx];
+    stage_f64_padded<D>(tq, t_q + (size_t)j * D * D);
     if (warp < G) {
         const size_t base = ((size_t)b * hq + j * G + warp) * D;
         for (int c = lane; c < D; c += 32) {
-            qrow[warp * D + c] = (dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[base + c])
-                                                     : reinterpret_cast<const float *>(q)[base + c];
+            qin[warp * D + c] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[base + c])
+                                                             : reinterpret_cast<const float *>(q)[base + c]);
             mask[warp * D + c] = 0;
         }
     }
@@ -106,10 +106,10 @@ __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, co
 #pragma unroll
         for (int m = 0; m < NG; ++m) {
             const int c = lane + 32 * m;
-            const float *row = &tq[c * (D + 1)];
+            const double *row = &tq[c * (D + 1)];
             double s = 0.0;
 #pragma unroll 8
-            for (int i = 0; i < D; ++i) s = fma((double)row[i], (double)qrow[warp * D + i], s);
+            for (int i = 0; i < D; ++i) s = fma(row[i], qin[warp * D + i], s);
             qp[m] = __double2float_rn(s);
             // descending |q'|, then ascending channel; channel 0 sorts last (key 0)
             key[m] = (c == 0) ? 0ull

@@ -240,4 +240,5 @@ def assert_outputs_close(out: np.ndarray, ref: np.ndarray, atol: float = ATOL, r
     ok = den > 0
     if ok.any():
         assert rel[ok].max() <= rtol_row, f"row relative error {rel[ok].max():.3e} > {rtol_row}"
+    print(f"[parity] max abs err {err.max():.3e}, max row rel err {rel[ok].max() if ok.any() else 0.0:.3e}")
     return float(err.max()), float(rel[ok].max()) if ok.any() else 0.0
