@@ -56,6 +56,12 @@ def aggregate(tokens_per_rank: int, elapsed_s: float, steps: int, n_ranks: int, 
     return {"value": tokens_per_rank * steps * n_ranks / t, "ms_per_step": 1e3 * t / steps, "elapsed_s": t}
 
 
+def rank_workload(w, rank: int):
+    """Weak scaling: every rank decodes its own independent batch of sequences
+    (same layer shapes, its own seeded contents); nothing crosses ranks."""
+    return w if rank == 0 else w.with_(seed=w.seed + 7919 * rank)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -243,7 +249,7 @@ def run_dqk(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     from bit_kv_cache_dqk_b200 import inputs as I
-    w = I.CONFIGS[args.workload]
+    w = rank_workload(I.CONFIGS[args.workload], rank)
     layer = Layer(w, dev)
     layer.prefill()
     tokens = int(layer.lens.sum())
