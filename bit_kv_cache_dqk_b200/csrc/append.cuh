@@ -14,7 +14,8 @@ struct AppendSmem {
     static constexpr int NG = D / kGroup;
     static constexpr int kMaxBlockBytes = 8 * D + 128 * NG + 64;
     double tk[D * (D + 1)];          // T_K[j] in fp64, rows padded by one element
-    double x[kPage][D];              // one input row per warp, fp64
+    double x[kPage][D];              // input K rows of the page's new slots, fp64
+    float kp[kPage][D];              // their transformed rows k' (fp32)
     uint8_t kcode[kPage][D];         // plain codes of the page being rewritten
     uint8_t vcode[kPage][D];
     uint16_t kscale[kPage][NG], kmin[kPage][NG], kch0[kPage];
@@ -22,34 +23,44 @@ struct AppendSmem {
     uint4 blk[kMaxBlockBytes / 16];  // the packed block
 };
 
+// One 32-channel group held by a warp (lane = channel of the group): group
+// min/max of the fp32 values by warp shuffles (with -0 read as +0), then fp64
+// arithmetic with single RNE roundings: scale = fp16((max - min) / 3), min =
+// fp16(min), code = clamp(rne((x - min) / scale), 0, 3) (0 when scale is 0).
+// excluded: this lane's value (channel 0 of a protected key) takes no part
+// and gets code 0.
+__device__ __forceinline__ int quantize_group(float xv, bool excluded, uint16_t &sh, uint16_t &mh) {
+    const float x = xv + 0.0f;
+    float lo = excluded ? __int_as_float(0x7f800000) : x;
+    float hi = excluded ? __int_as_float(0xff800000) : x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    sh = f64_to_f16_rne(((double)hi - (double)lo) / 3.0);
+    mh = f64_to_f16_rne((double)lo);
+    const double s = f16_to_f64(sh), mn = f16_to_f64(mh);
+    int code = 0;
+    if (!excluded && s != 0.0) {
+        const double r = rint(((double)x - mn) / s);
+        code = r < 0.0 ? 0 : (r > 3.0 ? 3 : (int)r);
+    }
+    return code;
+}
+
 // Quantize the D values a warp holds (lane owns channels lane + 32*m, i.e.
 // channel `lane` of group m) into codes / fp16 scale / fp16 min / BF16 ch0.
 // protect: channel 0 goes to BF16, is excluded from group 0's range and its
-// code is 0.  Group min/max of the fp32 values by warp shuffles (with -0
-// read as +0), then fp64 arithmetic with single RNE roundings.
+// code is 0.
 template <int NG>
 __device__ __forceinline__ void quantize_warp(const float (&vals)[NG], bool protect, int lane,
                                               uint8_t *codes, uint16_t *scale, uint16_t *minv,
                                               uint16_t *ch0) {
 #pragma unroll
     for (int m = 0; m < NG; ++m) {
-        const float x = vals[m] + 0.0f;
-        const bool excluded = protect && m == 0 && lane == 0;
-        float lo = excluded ? __int_as_float(0x7f800000) : x;
-        float hi = excluded ? __int_as_float(0xff800000) : x;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        }
-        const uint16_t sh = f64_to_f16_rne(((double)hi - (double)lo) / 3.0);
-        const uint16_t mh = f64_to_f16_rne((double)lo);
-        const double s = f16_to_f64(sh), mn = f16_to_f64(mh);
-        int code = 0;
-        if (!excluded && s != 0.0) {
-            const double r = rint(((double)x - mn) / s);
-            code = r < 0.0 ? 0 : (r > 3.0 ? 3 : (int)r);
-        }
+        uint16_t sh, mh;
+        const int code = quantize_group(vals[m], protect && m == 0 && lane == 0, sh, mh);
         codes[m * kGroup + lane] = (uint8_t)code;
         if (lane == 0) {
             scale[m] = sh;
@@ -158,21 +169,27 @@ __device__ void pack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
 }
 
 // Grid: x = work items (sequence, touched page) strided, y = kv head.
-// Block: 16 warps, warp w owns token slot w of the page being rewritten.
-// Each item: read the old block, overwrite the appended slots, write back
-// with 128-bit stores.  T_K[j] is staged once per CTA.
+// Block: 16 warps.  Each item: read the old block, overwrite the appended
+// slots, write it back with 128-bit stores.  T_K[j] is staged once per CTA;
+// the transforms of the new rows are spread over all threads (one (slot,
+// channel) sum each, four interleaved per thread), then warp w quantizes
+// token slot w.  early_release lets a kernel launched after this one with
+// programmatic stream serialization start at once (it must not read the
+// cache before its own grid-dependency wait).
 template <int D>
 __global__ void __launch_bounds__(512) k_quant_pack(
     const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin,
     int dtype, int batch, const int *__restrict__ new_lens, const int *__restrict__ seq_before,
     const int *__restrict__ page_table, int max_pages, int slots_per_seq, uint8_t *__restrict__ pool,
-    long long num_pages, int hkv, int v_ch0) {
+    long long num_pages, int hkv, int v_ch0, int early_release) {
     constexpr int NG = D / kGroup;
+    constexpr int kChains = 4;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     AppendSmem<D> &S = *reinterpret_cast<AppendSmem<D> *>(smem_raw);
     const int j = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layout L = make_layout(D, v_ch0);
+    if (early_release) grid_dependents_launch();
 
     stage_f64_padded<D>(S.tk, t_k + (size_t)j * D * D);
     __syncthreads();
@@ -192,32 +209,48 @@ __global__ void __launch_bounds__(512) k_quant_pack(
         long long row0 = 0;
         for (int bb = 0; bb < b; ++bb) row0 += new_lens[bb];
         uint4 *blk_g = reinterpret_cast<uint4 *>(pool + ((size_t)phys * hkv + j) * L.bytes);
+        // slots [s_lo, s_hi) of this page receive new rows
+        const int s_lo = max(0, L0 - page * kPage), s_hi = min(kPage, L0 + n - page * kPage);
+        const int total = (s_hi - s_lo) * D;
+        const long long row_of_slot = row0 + (long long)page * kPage - L0;   // input row of slot s: + s
 
         for (int o = threadIdx.x; o < L.bytes / 16; o += blockDim.x) S.blk[o] = blk_g[o];
+        for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+            const int sl = s_lo + idx / D, c = idx % D;
+            S.x[sl][c] = (double)load_elem(kin, dtype, ((size_t)(row_of_slot + sl) * hkv + j) * D + c);
+        }
         __syncthreads();
         unpack_block<D>(S, L, v_ch0);
-        __syncthreads();
-
-        const int pos = page * kPage + warp;
-        if (pos >= L0 && pos < L0 + n) {
-            const size_t base = ((size_t)(row0 + (pos - L0)) * hkv + j) * D;
+        // k'_c = sum_i T_K[c][i] x_i, ascending i, exact products summed in fp64
+        for (int k0 = threadIdx.x; k0 < total; k0 += kChains * blockDim.x) {
+            const double *row[kChains];
+            const double *xr[kChains];
+            double acc[kChains];
 #pragma unroll
-            for (int m = 0; m < NG; ++m) S.x[warp][lane + 32 * m] = (double)load_elem(kin, dtype, base + lane + 32 * m);
-            __syncwarp();
-            float kp[NG];
-            double acc[NG];
-#pragma unroll
-            for (int m = 0; m < NG; ++m) acc[m] = 0.0;
-            // NG independent sequential sums (ascending i), interleaved
-#pragma unroll 4
-            for (int i = 0; i < D; ++i) {
-                const double xi = S.x[warp][i];
-#pragma unroll
-                for (int m = 0; m < NG; ++m) acc[m] = fma(S.tk[(lane + 32 * m) * (D + 1) + i], xi, acc[m]);
+            for (int u = 0; u < kChains; ++u) {
+                const int k = min(k0 + u * (int)blockDim.x, total - 1);
+                const int sl = s_lo + k / D, c = k % D;
+                row[u] = &S.tk[c * (D + 1)];
+                xr[u] = &S.x[sl][0];
+                acc[u] = 0.0;
             }
+#pragma unroll 4
+            for (int i = 0; i < D; ++i)
 #pragma unroll
-            for (int m = 0; m < NG; ++m) kp[m] = __double2float_rn(acc[m]);
+                for (int u = 0; u < kChains; ++u) acc[u] = fma(row[u][i], xr[u][i], acc[u]);
+#pragma unroll
+            for (int u = 0; u < kChains; ++u) {
+                const int k = k0 + u * (int)blockDim.x;
+                if (k < total) S.kp[s_lo + k / D][k % D] = __double2float_rn(acc[u]);
+            }
+        }
+        __syncthreads();
+        if (warp >= s_lo && warp < s_hi) {
+            float kp[NG];
+#pragma unroll
+            for (int m = 0; m < NG; ++m) kp[m] = S.kp[warp][lane + 32 * m];
             quantize_warp<NG>(kp, true, lane, S.kcode[warp], S.kscale[warp], S.kmin[warp], &S.kch0[warp]);
+            const size_t base = ((size_t)(row_of_slot + warp) * hkv + j) * D;
             float vv[NG];
 #pragma unroll
             for (int m = 0; m < NG; ++m) vv[m] = load_elem(vin, dtype, base + lane + 32 * m);
@@ -228,6 +261,108 @@ __global__ void __launch_bounds__(512) k_quant_pack(
         __syncthreads();
         for (int o = threadIdx.x; o < L.bytes / 16; o += blockDim.x) blk_g[o] = S.blk[o];
         __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// k_append_rows: the decode-time append (a few rows per sequence).  One CTA
+// of D threads per (new row, kv head); thread c computes k'_c from T_K's row c
+// (read straight from global memory, all loads in flight at once) and warp g
+// quantizes group g.  Only the row's own fields of its (page, kv head) block
+// are written: its key code words (each holds codes of one token) with plain
+// stores, its value code fields (words shared with neighbouring tokens) with
+// atomic and/or, its scale/min/channel-0 entries with 16-bit stores.  Same
+// arithmetic, hence the same bytes, as k_quant_pack.
+// ---------------------------------------------------------------------------
+constexpr int kDirectMaxNew = 4;   // dqk_append uses k_append_rows up to this many rows per sequence
+
+template <int D>
+__global__ void __launch_bounds__(D) k_append_rows(
+    const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin, int dtype,
+    const int *__restrict__ new_lens, const int *__restrict__ seq_before, const int *__restrict__ page_table,
+    int max_pages, int max_new, uint8_t *__restrict__ pool, long long num_pages, int hkv, int v_ch0,
+    int early_release) {
+    constexpr int NG = D / kGroup;
+    __shared__ double xs[D];
+    __shared__ uint32_t kimg[D], kmask[D], vimg[D], vmask[D];   // code regions are D words each
+    const int j = blockIdx.y;
+    const int b = blockIdx.x / max_new, t = blockIdx.x - b * max_new;
+    const int c = threadIdx.x, warp = c >> 5, lane = c & 31;
+    if (early_release) grid_dependents_launch();
+    const int n = new_lens[b];
+    if (t >= n) return;                       // the whole CTA
+    const int L0 = seq_before[b];
+    const int pos = L0 + t;
+    const int page = pos / kPage, slot = pos - page * kPage;
+    // T_K row c, all loads in flight
+    const float4 *tr = reinterpret_cast<const float4 *>(t_k + ((size_t)j * D + c) * D);
+    float4 tv[D / 4];
+#pragma unroll
+    for (int u = 0; u < D / 4; ++u) tv[u] = tr[u];
+    int row0 = 0;                             // rows of sequences 0..b-1 come first
+    for (int bb = lane; bb < b; bb += 32) row0 += new_lens[bb];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) row0 += __shfl_xor_sync(0xffffffffu, row0, o);
+    const size_t base = (((size_t)row0 + t) * hkv + j) * D;
+    const float xk = load_elem(kin, dtype, base + c);
+    const float xv = load_elem(vin, dtype, base + c);
+    const int phys = (L0 >= 0 && page < max_pages) ? page_table[(size_t)b * max_pages + page] : -1;
+    xs[c] = (double)xk;
+    kimg[c] = 0u;
+    kmask[c] = 0u;
+    vimg[c] = 0u;
+    vmask[c] = 0u;
+    __syncthreads();
+    // k'_c = sum_i T_K[c][i] x_i, ascending i, exact products summed in fp64
+    double acc = 0.0;
+#pragma unroll
+    for (int u = 0; u < D / 4; ++u) {
+        acc = fma((double)tv[u].x, xs[4 * u + 0], acc);
+        acc = fma((double)tv[u].y, xs[4 * u + 1], acc);
+        acc = fma((double)tv[u].z, xs[4 * u + 2], acc);
+        acc = fma((double)tv[u].w, xs[4 * u + 3], acc);
+    }
+    const float kp = __double2float_rn(acc);
+    if (phys < 0 || phys >= num_pages) {      // the whole CTA
+        if (c == 0) dqk_flag_error(kErrBounds);
+        return;
+    }
+    const Layout L = make_layout(D, v_ch0);
+    uint8_t *blk = pool + ((size_t)phys * hkv + j) * L.bytes;
+    uint16_t *h16 = reinterpret_cast<uint16_t *>(blk);
+    uint16_t ksh, kmh, vsh, vmh;
+    const int kc = quantize_group(kp, c == 0, ksh, kmh);
+    const int vc = quantize_group(xv, v_ch0 != 0 && c == 0, vsh, vmh);
+    if (lane == 0) {
+        h16[(L.ks >> 1) + kscale_idx(NG, slot, warp)] = ksh;
+        h16[(L.km >> 1) + kscale_idx(NG, slot, warp)] = kmh;
+        h16[(L.vs >> 1) + vscale_idx(NG, slot, warp)] = vsh;
+        h16[(L.vm >> 1) + vscale_idx(NG, slot, warp)] = vmh;
+    }
+    if (c == 0) {
+        h16[(L.k0 >> 1) + k0_idx(slot)] = f32_to_bf16_rne(kp);
+        if (v_ch0) h16[(L.v0 >> 1) + slot] = f32_to_bf16_rne(xv);
+    }
+    int off, bit;
+    kcode_pos(NG, slot, c, off, bit);
+    atomicOr(&kimg[off >> 2], (uint32_t)kc << bit);
+    atomicOr(&kmask[off >> 2], 3u << bit);
+    vcode_pos(NG, slot, c, off, bit);
+    atomicOr(&vimg[off >> 2], (uint32_t)vc << bit);
+    atomicOr(&vmask[off >> 2], 3u << bit);
+    __syncthreads();
+    uint32_t *kw = reinterpret_cast<uint32_t *>(blk + L.kc);
+    uint32_t *vw = reinterpret_cast<uint32_t *>(blk + L.vc);
+    const uint32_t km = kmask[c], vm = vmask[c];
+    if (km == 0xffffffffu) {
+        kw[c] = kimg[c];                      // a key word holds codes of this token only
+    } else if (km) {
+        atomicAnd(&kw[c], ~km);
+        atomicOr(&kw[c], kimg[c]);
+    }
+    if (vm) {                                 // value words are shared with neighbouring tokens
+        atomicAnd(&vw[c], ~vm);
+        atomicOr(&vw[c], vimg[c]);
     }
 }
 

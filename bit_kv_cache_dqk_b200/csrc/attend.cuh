@@ -643,24 +643,26 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
 // log-sum-exp combine: out[b][h] = sum_i o_i 2^(m_i - m*) / sum_i l_i 2^(m_i - m*)
 // over the records of every CTA (and page slot) that held pages of (b, h).
 // ---------------------------------------------------------------------------
-constexpr int kCombineChunk = 256;     // records weighted per pass
-constexpr int kCombineThreads = 512;   // channel x record-slice threads
+constexpr int kCombineChunk = 64;      // records read per pass
+constexpr int kCombineThreads = 256;   // small enough to sit beside an attend CTA on its SM
 
-// One CTA per (sequence, query head).  Thread (slice, channel) accumulates the
-// records i = slice (mod slices) of its channel; slices are summed in a fixed
-// order, so the result does not depend on scheduling.
+// One CTA per (sequence, query head).  Each pass reads a chunk of records in
+// one round: (m_i, l_i) into shared memory, and thread (slice, channel) the
+// channel of records i = slice (mod slices).  The running max moves from
+// chunk to chunk with an exact rescale.  Every warp forms the chunk's max and
+// denominator with the same lane order and shuffle tree, and the slices are
+// summed in a fixed order, so the result does not depend on scheduling.
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restrict__ seq_lens, int batch, int hq,
                                                              int hkv, int hc, int pw, int nchunks, int num_ctas,
                                                              const float *__restrict__ part, float *__restrict__ out) {
     constexpr int kSlices = kCombineThreads / D;
+    constexpr int kPer = kCombineChunk / kSlices;   // records of a chunk per thread
     __shared__ long long sh_U, sh_ur;
     __shared__ int sh_np;
-    __shared__ float sh_w[kCombineChunk];
-    __shared__ int sh_rec[kCombineChunk];
-    __shared__ float sh_dpart[kCombineThreads / 32];
+    __shared__ int sh_rec[kCombineChunk];   // record index of slot i of the chunk, -1 for none
+    __shared__ float sh_m[kCombineChunk], sh_l[kCombineChunk];
     __shared__ float sh_acc[kSlices][D];
-    __shared__ float sh_m;
     const int h = blockIdx.x, b = blockIdx.y;
     const int G = hq / hkv, j = h / G, chunk = j / hc, jl = j % hc, hh = h % G;
     const int r = b * nchunks + chunk, R = batch * nchunks;
@@ -683,60 +685,79 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restri
         }
     }
     __syncthreads();
-    grid_dependency_wait();     // partial records come from k_attend
     const long long U = sh_U, ur = sh_ur;
     const int np = sh_np;
     float *o = out + ((size_t)b * hq + h) * D;
+    // records of this (run, head): CTAs cf..cl that own units of the run (CTAs
+    // with an empty unit range wrote none), each with pw page-slot records
+    const int cf = np > 0 ? (int)cta_of_unit(ur, U, num_ctas) : 0;
+    const int cl = np > 0 ? (int)cta_of_unit(ur + np - 1, U, num_ctas) : -1;
+    const int nrec = (cl - cf + 1) * pw;
+    // record slots of chunk i0 (known before the attend kernel has finished)
+    auto index_chunk = [&](int i0) {
+        for (int i = threadIdx.x; i < kCombineChunk; i += blockDim.x) {
+            int ri = -1;
+            if (i0 + i < nrec) {
+                const int c = cf + (i0 + i) / pw, s = (i0 + i) % pw;
+                if ((long long)c * U / num_ctas < ((long long)c + 1) * U / num_ctas)
+                    ri = (int)record_index(c + r, s, jl, hh, pw, hc, G);
+            }
+            sh_rec[i] = ri;
+        }
+    };
+    index_chunk(0);
+    __syncthreads();
+    grid_dependency_wait();     // partial records come from k_attend
     if (np == 0) {
         if (slice == 0) o[ch] = 0.0f;
         return;
     }
-    // records of this (run, head): CTAs cf..cl that own units of the run (CTAs
-    // with an empty unit range wrote none), each with pw warp-pair records
-    const int cf = (int)cta_of_unit(ur, U, num_ctas), cl = (int)cta_of_unit(ur + np - 1, U, num_ctas);
-    const int nrec = (cl - cf + 1) * pw;
-    auto rec_at = [&](int i, bool &ok) -> size_t {
-        const int c = cf + i / pw, s = i % pw;
-        ok = (long long)c * U / num_ctas < ((long long)c + 1) * U / num_ctas;
-        return record_index(c + r, s, jl, hh, pw, hc, G);
-    };
-    if (warp == 0) {       // global max over all records
-        float m = -INFINITY;
-        for (int i = lane; i < nrec; i += 32) {
-            bool ok;
-            const size_t ri = rec_at(i, ok);
-            if (ok) m = fmaxf(m, part[ri * (2 + D)]);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) sh_m = m;
-    }
-    __syncthreads();
-    const float mstar = sh_m;
-    float acc = 0.0f, dsum = 0.0f;
+    float mrun = -INFINITY, acc = 0.0f, dsum = 0.0f;
     for (int i0 = 0; i0 < nrec; i0 += kCombineChunk) {
         const int n = min(kCombineChunk, nrec - i0);
-        float dpart = 0.0f;
+        if (i0 > 0) {
+            __syncthreads();   // the previous chunk has been read
+            index_chunk(i0);
+            __syncthreads();
+        }
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            bool ok;
-            const size_t ri = rec_at(i0 + i, ok);
-            const float mi = ok ? part[ri * (2 + D)] : -INFINITY;
-            const float w = mi == -INFINITY ? 0.0f : exp2f(mi - mstar);
-            sh_w[i] = w;
-            sh_rec[i] = ok ? (int)ri : -1;
-            if (w != 0.0f) dpart += w * part[ri * (2 + D) + 1];
+            const int ri = sh_rec[i];
+            sh_m[i] = ri >= 0 ? part[(size_t)ri * (2 + D)] : -INFINITY;
+            sh_l[i] = ri >= 0 ? part[(size_t)ri * (2 + D) + 1] : 0.0f;
+        }
+        float ov[kPer];
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = slice + kSlices * k;
+            const int ri = i < n ? sh_rec[i] : -1;
+            ov[k] = ri >= 0 ? part[(size_t)ri * (2 + D) + 2 + ch] : 0.0f;
+        }
+        __syncthreads();
+        float cm = -INFINITY;
+        for (int i = lane; i < n; i += 32) cm = fmaxf(cm, sh_m[i]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+        const float mnew = fmaxf(mrun, cm);
+        if (mnew == -INFINITY) continue;   // no tokens yet
+        const float alpha = exp2f(mrun - mnew);   // 0 while mrun is -inf
+        float dpart = 0.0f;
+        for (int i = lane; i < n; i += 32) {
+            const float mi = sh_m[i];
+            if (mi != -INFINITY) dpart += exp2f(mi - mnew) * sh_l[i];
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) dpart += __shfl_xor_sync(0xffffffffu, dpart, off);
-        if (lane == 0) sh_dpart[warp] = dpart;
-        __syncthreads();
-        for (int k = 0; k < kCombineThreads / 32; ++k) dsum += sh_dpart[k];   // fixed order
-#pragma unroll 4
-        for (int i = slice; i < n; i += kSlices) {
-            const float w = sh_w[i];
-            if (w != 0.0f) acc = fmaf(w, part[(size_t)sh_rec[i] * (2 + D) + 2 + ch], acc);
+        dsum = dsum * alpha + dpart;
+        acc *= alpha;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = slice + kSlices * k;
+            if (i < n) {
+                const float mi = sh_m[i];
+                if (mi != -INFINITY) acc = fmaf(exp2f(mi - mnew), ov[k], acc);
+            }
         }
-        __syncthreads();
+        mrun = mnew;
     }
     sh_acc[slice][ch] = acc;
     __syncthreads();

@@ -144,19 +144,16 @@ dqk_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 
 template <int D>
 dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
-    const int G = P.G;
-    const size_t smem = (size_t)D * (D + 1) * 8 + (size_t)G * D * 8 + (size_t)G * D * 4 + (size_t)G * P.NG * 8 +
-                        (size_t)G * D * 3;
+    const size_t smem = qprep_smem_bytes(D, P.G);
     if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
     const float qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
-    const int threads = (G < 4 ? 4 : G) * 32;
-    k_qprep<D><<<dim3(a.L->num_kv_heads, a.batch), threads, smem, a.stream>>>(
-        a.L->t_q, a.q, a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qscale,
-        reinterpret_cast<uint2 *>(ws + P.off_qf), reinterpret_cast<float *>(ws + P.off_qk),
-        reinterpret_cast<uint32_t *>(ws + P.off_qm), reinterpret_cast<float *>(ws + P.off_q0), a.sel_out);
-    return launch_status();
+    return launch_pdl(k_qprep<D>, dim3(a.L->num_kv_heads, a.batch), dim3(kQprepThreads), smem, a.stream, a.L->t_q,
+                      a.q, (int)a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qscale,
+                      reinterpret_cast<uint2 *>(ws + P.off_qf), reinterpret_cast<float *>(ws + P.off_qk),
+                      reinterpret_cast<uint32_t *>(ws + P.off_qm), reinterpret_cast<float *>(ws + P.off_q0),
+                      a.sel_out);
 }
 
 template <int D, int G, bool VCH0>
@@ -239,7 +236,15 @@ dqk_status decode_stages(const DecodeArgs &a, int stages) {
 template <int D>
 dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk_dtype dtype, int batch,
                       const int *new_lens, const int *seq_before, int max_new, const int *page_table,
-                      int max_pages, cudaStream_t stream) {
+                      int max_pages, int early_release, cudaStream_t stream) {
+    if (max_new <= kDirectMaxNew) {
+        const long long gx = (long long)batch * max_new;
+        if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
+        k_append_rows<D><<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
+            L->t_k, k, v, dtype, new_lens, seq_before, page_table, max_pages, max_new,
+            static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
+        return launch_status();
+    }
     const size_t smem = sizeof(AppendSmem<D>);
     if (cudaFuncSetAttribute(k_quant_pack<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DQK_ERR_CUDA;
@@ -253,7 +258,7 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
     if (gx < 1) gx = 1;
     k_quant_pack<D><<<dim3((unsigned)gx, L->num_kv_heads), 512, smem, stream>>>(
         L->t_k, k, v, dtype, batch, new_lens, seq_before, page_table, max_pages, slots,
-        static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect);
+        static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
     return launch_status();
 }
 
@@ -267,20 +272,41 @@ size_t dqk_block_bytes(const dqk_layer_desc *layer) {
     return (size_t)make_layout(layer->head_dim, layer->v_ch0_protect).bytes;
 }
 
-dqk_status dqk_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
-                      const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
-                      int max_pages, dqk_stream_t stream) {
+}  // extern "C"
+
+namespace {
+dqk_status check_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
+                        const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
+                        int max_pages) {
     dqk_status st = check_layer(layer);
     if (st != DQK_OK) return st;
     if (!layer->t_k || !k || !v || !new_lens || !seq_lens_before || !page_table) return DQK_ERR_INVALID_ARG;
     if (dtype != DQK_F32 && dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
     if (batch <= 0 || max_pages <= 0 || max_new < 0) return DQK_ERR_INVALID_ARG;
     if (!aligned(k, 4) || !aligned(v, 4)) return DQK_ERR_INVALID_ARG;
-    if (max_new == 0) return DQK_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return layer->head_dim == 128
-               ? run_append<128>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages, s)
-               : run_append<64>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages, s);
+    return DQK_OK;
+}
+
+dqk_status launch_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
+                         const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
+                         int max_pages, int early_release, cudaStream_t s) {
+    return layer->head_dim == 128 ? run_append<128>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new,
+                                                    page_table, max_pages, early_release, s)
+                                  : run_append<64>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new,
+                                                   page_table, max_pages, early_release, s);
+}
+}  // namespace
+
+extern "C" {
+
+dqk_status dqk_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
+                      const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
+                      int max_pages, dqk_stream_t stream) {
+    dqk_status st = check_append(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages);
+    if (st != DQK_OK || max_new == 0) return st;
+    // whatever follows may read the cache at once: release it only at exit
+    return launch_append(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages, 0,
+                         static_cast<cudaStream_t>(stream));
 }
 
 size_t dqk_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max_pages) {
@@ -300,6 +326,28 @@ size_t dqk_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max
 
 dqk_status dqk_decode(DQK_DECODE_ARGS) {
     DQK_DECODE_PACK;
+    return decode_stages(a, kPrepare | kAttend | kCombine);
+}
+dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype kv_dtype,
+                           const int *new_lens, const int *seq_lens_before, int max_new, const void *q,
+                           dqk_dtype q_dtype, int batch, const int *seq_lens, const int *page_table, int max_pages,
+                           int sparsity_pct, float *out, int16_t *sel_out, void *workspace, size_t workspace_bytes,
+                           dqk_stream_t stream) {
+    dqk_status st = check_append(layer, k, v, kv_dtype, batch, new_lens, seq_lens_before, max_new, page_table,
+                                 max_pages);
+    if (st != DQK_OK) return st;
+    DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out, sel_out,
+                 workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};
+    DecodePlan P;
+    st = check_decode(a, P);
+    if (st != DQK_OK) return st;
+    if (max_new > 0) {
+        // the query kernel (next on the stream) may start at once: it reads only
+        // q and T_Q before its grid-dependency wait
+        st = launch_append(layer, k, v, kv_dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages,
+                           1, a.stream);
+        if (st != DQK_OK) return st;
+    }
     return decode_stages(a, kPrepare | kAttend | kCombine);
 }
 dqk_status dqk_decode_prepare(DQK_DECODE_ARGS) {

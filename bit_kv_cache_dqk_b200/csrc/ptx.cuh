@@ -92,15 +92,16 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // operands without per-use conversions.  n must be a multiple of 4.
 template <int n>
 __device__ __forceinline__ void stage_f64_padded(double *dst, const float *src) {
+    constexpr int kInFlight = 8;   // float4 loads a thread issues before converting
     const float4 *s4 = reinterpret_cast<const float4 *>(src);
-    const int n4 = n * n / 4;
-    for (int base = threadIdx.x; base < n4; base += 4 * blockDim.x) {
-        float4 v[4];
+    constexpr int n4 = n * n / 4;
+    for (int base = threadIdx.x; base < n4; base += kInFlight * blockDim.x) {
+        float4 v[kInFlight];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < kInFlight; ++u)
             if (base + u * blockDim.x < n4) v[u] = s4[base + u * blockDim.x];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kInFlight; ++u) {
             const int idx4 = base + u * blockDim.x;
             if (idx4 < n4) {
                 const int e = idx4 * 4, row = e / n, col = e % n;

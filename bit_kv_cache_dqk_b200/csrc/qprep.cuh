@@ -68,35 +68,65 @@ __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
     return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
 }
 
+constexpr int kQprepThreads = 256;
+
+// Shared memory of k_qprep for group size G.
+__host__ __device__ constexpr size_t qprep_smem_bytes(int D, int G) {
+    return (size_t)G * D * 8 + (size_t)G * D * 4 + (size_t)G * (D / 32) * 8 + (size_t)G * D * 3;
+}
+
+// Launched with programmatic stream serialization: it reads its inputs and
+// computes q' while an earlier append may still be running, waits for the
+// earlier work before writing anything, then releases the attend kernel.
 template <int D>
-__global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, const void *__restrict__ q,
-                                              int dtype, int hq, int hkv, int pct, float qscale,
-                                              uint2 *__restrict__ qf, float *__restrict__ qk,
-                                              uint32_t *__restrict__ qm, float *__restrict__ q0,
-                                              int16_t *__restrict__ sel_out) {
+__global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict__ t_q, const void *__restrict__ q,
+                                                        int dtype, int hq, int hkv, int pct, float qscale,
+                                                        uint2 *__restrict__ qf, float *__restrict__ qk,
+                                                        uint32_t *__restrict__ qm, float *__restrict__ q0,
+                                                        int16_t *__restrict__ sel_out) {
     constexpr int NG = D / 32;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int G = hq / hkv;
     const int NT = G > 4 ? 2 : 1;
-    double *tq = reinterpret_cast<double *>(smem_raw);               // [D][D+1] fp64
-    double *qin = tq + D * (D + 1);                                   // [G][D]   input row, fp64
-    float *qrow = reinterpret_cast<float *>(qin + G * D);             // [G][D]   qs
-    float *qsum = qrow + G * D;                                       // [G][NG]
+    double *qin = reinterpret_cast<double *>(smem_raw);               // [G][D]   input rows, fp64
+    float *qpv = reinterpret_cast<float *>(qin + G * D);              // [G][D]   q' (fp32)
+    float *qsum = qpv + G * D;                                        // [G][NG]
     float *sig = qsum + G * NG;                                       // [G][NG]  sigma
     signed char *q8 = reinterpret_cast<signed char *>(sig + G * NG);  // [G][2][D] pieces
     unsigned char *mask = reinterpret_cast<unsigned char *>(q8 + G * 2 * D);  // [G][D]
     const int j = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    grid_dependents_launch();   // the attend kernel may start streaming pages now
-    stage_f64_padded<D>(tq, t_q + (size_t)j * D * D);
-    if (warp < G) {
-        const size_t base = ((size_t)b * hq + j * G + warp) * D;
-        for (int c = lane; c < D; c += 32) {
-            qin[warp * D + c] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[base + c])
-                                                             : reinterpret_cast<const float *>(q)[base + c]);
-            mask[warp * D + c] = 0;
-        }
+    // thread: channel c of heads h0, h0 + hstep, ...; T_Q row c, all loads in flight
+    const int c = threadIdx.x % D, h0 = threadIdx.x / D, hstep = kQprepThreads / D;
+    float4 tv[D / 4];
+    if (h0 < G) {
+        const float4 *tr = reinterpret_cast<const float4 *>(t_q + ((size_t)j * D + c) * D);
+#pragma unroll
+        for (int u = 0; u < D / 4; ++u) tv[u] = tr[u];
     }
+    const size_t qbase = ((size_t)b * hq + (size_t)j * G) * D;
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        qin[idx] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[qbase + idx])
+                                                : reinterpret_cast<const float *>(q)[qbase + idx]);
+        mask[idx] = 0;
+    }
+    __syncthreads();
+    // q'_c = sum_i T_Q[c][i] q_i, ascending i, exact fp32 x fp32 products
+    // accumulated in fp64, rounded once to fp32
+    for (int h = h0; h < G; h += hstep) {
+        const double *x = &qin[h * D];
+        double acc = 0.0;
+#pragma unroll
+        for (int u = 0; u < D / 4; ++u) {
+            acc = fma((double)tv[u].x, x[4 * u + 0], acc);
+            acc = fma((double)tv[u].y, x[4 * u + 1], acc);
+            acc = fma((double)tv[u].z, x[4 * u + 2], acc);
+            acc = fma((double)tv[u].w, x[4 * u + 3], acc);
+        }
+        qpv[h * D + c] = __double2float_rn(acc);
+    }
+    grid_dependency_wait();     // earlier work on the stream (e.g. a cache append) is complete
+    grid_dependents_launch();   // the attend kernel may start streaming pages now
     __syncthreads();
     if (warp < G) {
         const int h = j * G + warp;
@@ -106,11 +136,7 @@ __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, co
 #pragma unroll
         for (int m = 0; m < NG; ++m) {
             const int c = lane + 32 * m;
-            const double *row = &tq[c * (D + 1)];
-            double s = 0.0;
-#pragma unroll 8
-            for (int i = 0; i < D; ++i) s = fma(row[i], qin[warp * D + i], s);
-            qp[m] = __double2float_rn(s);
+            qp[m] = qpv[warp * D + c];
             // descending |q'|, then ascending channel; channel 0 sorts last (key 0)
             key[m] = (c == 0) ? 0ull
                               : (((unsigned long long)(__float_as_uint(qp[m]) & 0x7fffffffu) << 32) |
@@ -134,7 +160,6 @@ __global__ void __launch_bounds__(256) k_qprep(const float *__restrict__ t_q, co
             const float qs = qp[m] * qscale;
             if (c == 0) q0[(size_t)b * hq + h] = qs;
             const float v = (keep && c != 0) ? qs : 0.0f;
-            qrow[warp * D + c] = v;
             // group sums of the kept, scaled channels (channel 0 excluded)
             float gs = v, gm = fabsf(v);
 #pragma unroll

@@ -24,7 +24,7 @@ DQK_ERR_CUDA, DQK_ERR_DEVICE_BOUNDS, DQK_ERR_TIMEOUT = 4, 5, 6
 DQK_F32, DQK_BF16 = 0, 1
 
 EXPORTED = ["dqk_block_bytes", "dqk_append", "dqk_decode_workspace_size", "dqk_decode",
-            "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine",
+            "dqk_decode_step", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine",
             "dqk_decode_noalloc", "dqk_last_device_error", "dqk_status_string"]
 
 DQK_NOALLOC_WORKSPACE_BYTES = 8 << 20
@@ -49,6 +49,9 @@ for _n in ("dqk_decode", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_
     getattr(_lib, _n).restype = C.c_int
     getattr(_lib, _n).argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P,
                                   C.c_size_t, _P]
+_lib.dqk_decode_step.restype = C.c_int
+_lib.dqk_decode_step.argtypes = [_D, _P, _P, C.c_int, _P, _P, C.c_int, _P, C.c_int, C.c_int, _P, _P, C.c_int,
+                                 C.c_int, _P, _P, _P, C.c_size_t, _P]
 _lib.dqk_decode_noalloc.restype = C.c_int
 _lib.dqk_decode_noalloc.argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P]
 _lib.dqk_last_device_error.restype = C.c_int
@@ -118,6 +121,16 @@ def dqk_decode(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsi
                workspace, workspace_bytes, stream=None, raise_on_error=True) -> int:
     return _decode(_lib.dqk_decode, "dqk_decode", layer, q, q_dtype, batch, seq_lens, page_table,
                    max_pages, sparsity_pct, out, sel_out, workspace, workspace_bytes, stream, raise_on_error)
+
+
+def dqk_decode_step(layer, k, v, kv_dtype, new_lens, seq_lens_before, max_new, q, q_dtype, batch, seq_lens,
+                    page_table, max_pages, sparsity_pct, out, sel_out, workspace, workspace_bytes, stream=None,
+                    raise_on_error=True) -> int:
+    st = _lib.dqk_decode_step(C.byref(layer), _addr(k), _addr(v), kv_dtype, _addr(new_lens),
+                              _addr(seq_lens_before), max_new, _addr(q), q_dtype, batch, _addr(seq_lens),
+                              _addr(page_table), max_pages, sparsity_pct, _addr(out), _addr(sel_out),
+                              _addr(workspace), workspace_bytes, _stream(stream))
+    return _check(st, "dqk_decode_step", raise_on_error)
 
 
 def dqk_decode_prepare(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out,

@@ -169,6 +169,25 @@ dqk_status dqk_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dt
                       int sparsity_pct, float *out, int16_t *sel_out, void *workspace,
                       size_t workspace_bytes, dqk_stream_t stream);
 
+/* dqk_decode_step -- one serving decode step of a layer: dqk_append of the
+ * step's new K/V rows, then dqk_decode.  Passage: the decode step whose
+ * throughput "Throughput on SGLang" reports (cache write + pruned attention).
+ *  Arguments: those of dqk_append (k, v, kv_dtype, new_lens, seq_lens_before,
+ *  max_new) and of dqk_decode (the rest), same layouts and ownership;
+ *  seq_lens must already count the new rows.  All arguments of both parts are
+ *  checked before anything is launched.
+ *  Result: the same bytes as dqk_append followed by dqk_decode on `stream`.
+ *  The difference is on the GPU: the query transform and selection run while
+ *  the append is still writing the cache (the query kernel reads only q and
+ *  T_Q before waiting for the append), and the attention kernel starts
+ *  streaming pages as soon as the append has finished. */
+dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const void *v,
+                           dqk_dtype kv_dtype, const int *new_lens, const int *seq_lens_before,
+                           int max_new, const void *q, dqk_dtype q_dtype, int batch,
+                           const int *seq_lens, const int *page_table, int max_pages,
+                           int sparsity_pct, float *out, int16_t *sel_out, void *workspace,
+                           size_t workspace_bytes, dqk_stream_t stream);
+
 /* The three stages of dqk_decode, exported so callers can place or time them
  * separately.  Same arguments; each uses the ones its stage needs. */
 dqk_status dqk_decode_prepare(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
