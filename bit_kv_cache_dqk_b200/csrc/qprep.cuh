@@ -68,16 +68,21 @@ __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
     return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
 }
 
-constexpr int kQprepThreads = 256;
+constexpr int kQprepThreads = 512;
 
-// Shared memory of k_qprep for group size G.
+// Shared memory of k_qprep: T_Q[j] in fp32 with rows padded to D+4 floats
+// (conflict-free 16-byte row reads), the query rows in fp64, per-head sort
+// buffers and the outputs before they are laid out.
 __host__ __device__ constexpr size_t qprep_smem_bytes(int D, int G) {
-    return (size_t)G * D * 8 + (size_t)G * D * 4 + (size_t)G * (D / 32) * 8 + (size_t)G * D * 3;
+    return (size_t)D * (D + 4) * 4 + (size_t)G * D * 8 + (size_t)kQprepThreads * 8 + (size_t)G * (D / 32) * 8 +
+           (size_t)G * D * 3 + 64;
 }
 
+// One thread per (query head, channel), kQprepThreads / D heads per pass.
 // Launched with programmatic stream serialization: it reads its inputs and
-// computes q' while an earlier append may still be running, waits for the
-// earlier work before writing anything, then releases the attend kernel.
+// computes q' and the selection while an earlier append may still be running,
+// waits for the earlier work before writing anything, then releases the
+// attend kernel.
 template <int D>
 __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict__ t_q, const void *__restrict__ q,
                                                         int dtype, int hq, int hkv, int pct, float qscale,
@@ -85,105 +90,146 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
                                                         uint32_t *__restrict__ qm, float *__restrict__ q0,
                                                         int16_t *__restrict__ sel_out) {
     constexpr int NG = D / 32;
+    constexpr int kRow = D + 4;                       // padded fp32 row of T_Q
+    constexpr int kHeadsPerPass = kQprepThreads / D;
+    constexpr int kWarpsPerHead = D / 32;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int G = hq / hkv;
     const int NT = G > 4 ? 2 : 1;
-    double *qin = reinterpret_cast<double *>(smem_raw);               // [G][D]   input rows, fp64
-    float *qpv = reinterpret_cast<float *>(qin + G * D);              // [G][D]   q' (fp32)
-    float *qsum = qpv + G * D;                                        // [G][NG]
-    float *sig = qsum + G * NG;                                       // [G][NG]  sigma
-    signed char *q8 = reinterpret_cast<signed char *>(sig + G * NG);  // [G][2][D] pieces
-    unsigned char *mask = reinterpret_cast<unsigned char *>(q8 + G * 2 * D);  // [G][D]
+    float *tq = reinterpret_cast<float *>(smem_raw);                                  // [D][D+4]
+    double *qin = reinterpret_cast<double *>(tq + D * kRow);                         // [G][D]
+    unsigned long long *xbuf = reinterpret_cast<unsigned long long *>(qin + G * D);  // [threads] sort exchange
+    float *qsum = reinterpret_cast<float *>(xbuf + kQprepThreads);                   // [G][NG]
+    float *sig = qsum + G * NG;                                                       // [G][NG]  sigma
+    signed char *q8 = reinterpret_cast<signed char *>(sig + G * NG);                 // [G][2][D] pieces
+    unsigned char *mask = reinterpret_cast<unsigned char *>(q8 + G * 2 * D);         // [G][D]
+    int *wcount = reinterpret_cast<int *>(mask + G * D + ((16 - (G * D) % 16) % 16)); // [threads/32] kept per warp
     const int j = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // thread: channel c of heads h0, h0 + hstep, ...; T_Q row c, all loads in flight
-    const int c = threadIdx.x % D, h0 = threadIdx.x / D, hstep = kQprepThreads / D;
-    float4 tv[D / 4];
-    if (h0 < G) {
-        const float4 *tr = reinterpret_cast<const float4 *>(t_q + ((size_t)j * D + c) * D);
+    const int c = threadIdx.x % D, hp = threadIdx.x / D;   // channel, head slot of the pass
+    const int nk = keep_count(D, pct);
+
+    {   // stage T_Q[j] (fp32, padded rows) and the query rows (fp64)
+        constexpr int n4 = D * D / 4, kIn = (n4 + kQprepThreads - 1) / kQprepThreads;
+        const float4 *src = reinterpret_cast<const float4 *>(t_q + (size_t)j * D * D);
+        float4 v[kIn];
 #pragma unroll
-        for (int u = 0; u < D / 4; ++u) tv[u] = tr[u];
-    }
-    const size_t qbase = ((size_t)b * hq + (size_t)j * G) * D;
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        qin[idx] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[qbase + idx])
-                                                : reinterpret_cast<const float *>(q)[qbase + idx]);
-        mask[idx] = 0;
+        for (int u = 0; u < kIn; ++u) {
+            const int i4 = threadIdx.x + u * kQprepThreads;
+            if (i4 < n4) v[u] = src[i4];
+        }
+        const size_t qbase = ((size_t)b * hq + (size_t)j * G) * D;
+        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x)
+            qin[idx] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[qbase + idx])
+                                                    : reinterpret_cast<const float *>(q)[qbase + idx]);
+#pragma unroll
+        for (int u = 0; u < kIn; ++u) {
+            const int i4 = threadIdx.x + u * kQprepThreads;
+            if (i4 < n4) {
+                const int e = 4 * i4, row = e / D, col = e % D;
+                *reinterpret_cast<float4 *>(&tq[row * kRow + col]) = v[u];
+            }
+        }
     }
     __syncthreads();
-    // q'_c = sum_i T_Q[c][i] q_i, ascending i, exact fp32 x fp32 products
-    // accumulated in fp64, rounded once to fp32
-    for (int h = h0; h < G; h += hstep) {
-        const double *x = &qin[h * D];
-        double acc = 0.0;
+
+    bool waited = false;
+    for (int h0 = 0; h0 < G; h0 += kHeadsPerPass) {
+        const int hl = h0 + hp;                 // local query head of this thread
+        const bool active = hl < G;
+        const int h = j * G + hl;
+        // q'_c = sum_i T_Q[c][i] q_i, ascending i, exact fp32 x fp32 products
+        // accumulated in fp64, rounded once to fp32
+        float qp = 0.0f;
+        if (active) {
+            const float *row = &tq[c * kRow];
+            const double *x = &qin[hl * D];
+            double acc = 0.0;
 #pragma unroll
-        for (int u = 0; u < D / 4; ++u) {
-            acc = fma((double)tv[u].x, x[4 * u + 0], acc);
-            acc = fma((double)tv[u].y, x[4 * u + 1], acc);
-            acc = fma((double)tv[u].z, x[4 * u + 2], acc);
-            acc = fma((double)tv[u].w, x[4 * u + 3], acc);
+            for (int i = 0; i < D; i += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(&row[i]);
+                acc = fma((double)t4.x, x[i + 0], acc);
+                acc = fma((double)t4.y, x[i + 1], acc);
+                acc = fma((double)t4.z, x[i + 2], acc);
+                acc = fma((double)t4.w, x[i + 3], acc);
+            }
+            qp = __double2float_rn(acc);
         }
-        qpv[h * D + c] = __double2float_rn(acc);
-    }
-    grid_dependency_wait();     // earlier work on the stream (e.g. a cache append) is complete
-    grid_dependents_launch();   // the attend kernel may start streaming pages now
-    __syncthreads();
-    if (warp < G) {
-        const int h = j * G + warp;
-        const int nk = keep_count(D, pct);
-        float qp[NG];
-        unsigned long long key[NG];
+        // selection: bitonic sort (descending) of the head's D keys, one per
+        // thread: |q'| bits, then ascending channel; channel 0 sorts last
+        unsigned long long key = (c == 0) ? 0ull
+                                          : (((unsigned long long)(__float_as_uint(qp) & 0x7fffffffu) << 32) |
+                                             (unsigned long long)(0xffffffffu - (unsigned)c));
 #pragma unroll
-        for (int m = 0; m < NG; ++m) {
-            const int c = lane + 32 * m;
-            qp[m] = qpv[warp * D + c];
-            // descending |q'|, then ascending channel; channel 0 sorts last (key 0)
-            key[m] = (c == 0) ? 0ull
-                              : (((unsigned long long)(__float_as_uint(qp[m]) & 0x7fffffffu) << 32) |
-                                 (unsigned long long)(0xffffffffu - (unsigned)c));
+        for (int k = 2; k <= D; k <<= 1) {
+#pragma unroll
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                unsigned long long o;
+                if (jj < 32) {
+                    o = __shfl_xor_sync(0xffffffffu, key, jj);
+                } else {
+                    xbuf[threadIdx.x] = key;
+                    __syncthreads();
+                    o = xbuf[threadIdx.x ^ jj];
+                    __syncthreads();
+                }
+                const bool keep_max = ((c & jj) == 0) == ((c & k) == 0);
+                key = keep_max ? (key > o ? key : o) : (key < o ? key : o);
+            }
         }
-        warp_bitonic_desc<NG>(key, lane);
+        // position c of the sorted order holds the c-th largest key
+        if (active) mask[hl * D + c] = 0;
+        __syncthreads();
+        if (active && c < nk - 1) mask[hl * D + (int)(0xffffffffu - (unsigned)(key & 0xffffffffull))] = 1;
+        if (active && c == 0) mask[hl * D] = 1;
+        __syncthreads();
+        const bool keep = active && mask[hl * D + c] != 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) wcount[warp] = __popc(bal);
+        // scaled q' on kept channels >= 1; group sums and two int8 pieces
+        // relative to the group's largest |qs| (warp = one group of one head),
+        // sigma rounded up to 22 significant bits (so 1.5 * 2^23 * sigma / 4^g
+        // is exact)
+        const float qs = qp * qscale;
+        const float v = (keep && c != 0) ? qs : 0.0f;
+        float gs = v, gm = fabsf(v);
 #pragma unroll
-        for (int e = 0; e < NG; ++e)
-            if (lane * NG + e < nk - 1) mask[warp * D + (int)(0xffffffffu - (unsigned)(key[e] & 0xffffffffull))] = 1;
-        if (lane == 0) mask[warp * D] = 1;
-        __syncwarp();
-        int written = 0;
-#pragma unroll
-        for (int m = 0; m < NG; ++m) {
-            const int c = lane + 32 * m;
-            const bool keep = mask[warp * D + c] != 0;
-            const unsigned bal = __ballot_sync(0xffffffffu, keep);
-            if (sel_out && keep)
-                sel_out[((size_t)b * hq + h) * nk + written + __popc(bal & ((1u << lane) - 1u))] = (int16_t)c;
-            written += __popc(bal);
-            const float qs = qp[m] * qscale;
+        for (int o = 16; o > 0; o >>= 1) {
+            gs += __shfl_xor_sync(0xffffffffu, gs, o);
+            gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+        }
+        float sgm = gm / 127.0f;
+        sgm = __uint_as_float((__float_as_uint(sgm) + 3u) & ~3u);
+        int q1 = 0, q2 = 0;
+        if (sgm > 0.0f) {
+            const float x = v / sgm;
+            q1 = max(-127, min(127, __float2int_rn(x)));
+            q2 = max(-128, min(127, __float2int_rn((x - (float)q1) * 256.0f)));
+        }
+        const int g = c >> 5;
+        if (active) {
+            q8[(hl * 2 + 0) * D + c] = (signed char)q1;
+            q8[(hl * 2 + 1) * D + c] = (signed char)q2;
+            if (lane == 0) {
+                qsum[hl * NG + g] = gs;
+                sig[hl * NG + g] = sgm;
+            }
+        }
+        __syncthreads();
+        if (!waited) {
+            grid_dependency_wait();     // earlier work on the stream (e.g. a cache append) is complete
+            grid_dependents_launch();   // the attend kernel may start streaming pages now
+            waited = true;
+        }
+        if (active) {
+            // kept channels before c: earlier warps of this head, then lanes below
+            int before = __popc(bal & ((1u << lane) - 1u));
+            for (int w = warp - (warp % kWarpsPerHead); w < warp; ++w) before += wcount[w];
+            if (sel_out && keep) sel_out[((size_t)b * hq + h) * nk + before] = (int16_t)c;
             if (c == 0) q0[(size_t)b * hq + h] = qs;
-            const float v = (keep && c != 0) ? qs : 0.0f;
-            // group sums of the kept, scaled channels (channel 0 excluded)
-            float gs = v, gm = fabsf(v);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                gs += __shfl_xor_sync(0xffffffffu, gs, o);
-                gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
-            }
-            if (lane == 0) qsum[warp * NG + m] = gs;
-            // two int8 pieces relative to the group's largest |qs|; sigma rounded
-            // up to 22 significant bits (so 1.5 * 2^23 * sigma / 4^g is exact)
-            float sgm = gm / 127.0f;
-            sgm = __uint_as_float((__float_as_uint(sgm) + 3u) & ~3u);
-            int q1 = 0, q2 = 0;
-            if (sgm > 0.0f) {
-                const float x = v / sgm;
-                q1 = max(-127, min(127, __float2int_rn(x)));
-                q2 = max(-128, min(127, __float2int_rn((x - (float)q1) * 256.0f)));
-            }
-            q8[(warp * 2 + 0) * D + c] = (signed char)q1;
-            q8[(warp * 2 + 1) * D + c] = (signed char)q2;
-            if (lane == 0) sig[warp * NG + m] = sgm;
         }
+        __syncthreads();
     }
-    __syncthreads();
     // lay out the B-operand fragments
     const size_t bj = (size_t)b * hkv + j;
     for (int idx = threadIdx.x; idx < NT * NG * 32; idx += blockDim.x) {
