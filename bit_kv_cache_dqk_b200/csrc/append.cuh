@@ -80,33 +80,25 @@ template <int D>
 __device__ void unpack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
     constexpr int NG = D / kGroup;
     const uint32_t *w = reinterpret_cast<const uint32_t *>(S.blk);
-    for (int idx = threadIdx.x; idx < 2 * 32 * NG; idx += blockDim.x) {
-        const bool is_v = idx >= 32 * NG;
-        const int widx = is_v ? idx - 32 * NG : idx;
+    for (int widx = threadIdx.x; widx < 32 * NG; widx += blockDim.x) {
         const int lane = widx / NG, W = widx % NG, gid = lane >> 2, tig = lane & 3;
-        const uint32_t word = w[((is_v ? L.vc : L.kc) >> 2) + widx];
-        if (!is_v) {
-            // byte j, field f: group g = f % NG, register r = W + NG * (f / NG)
+        const uint32_t word = w[(L.kc >> 2) + widx];
+        // byte j, field f: group g = f % NG, register r = W + NG * (f / NG)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int f = 0; f < 4; ++f) {
-                    const int g = f % NG, r = W + NG * (f / NG);
-                    S.kcode[gid + 8 * (r & 1)][32 * g + 16 * (r >> 1) + 4 * tig + j] =
-                        (uint8_t)((word >> (8 * j + 2 * f)) & 3u);
-                }
-            continue;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int q = W * 8 + i;
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const uint8_t code = (uint8_t)((word >> (16 * e + 2 * i)) & 3u);
-                const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
-                S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid] = code;
+            for (int f = 0; f < 4; ++f) {
+                const int g = f % NG, r = W + NG * (f / NG);
+                S.kcode[gid + 8 * (r & 1)][32 * g + 16 * (r >> 1) + 4 * tig + j] =
+                    (uint8_t)((word >> (8 * j + 2 * f)) & 3u);
             }
-        }
+    }
+    const uint8_t *vb = reinterpret_cast<const uint8_t *>(S.blk) + L.vc;
+    for (int idx = threadIdx.x; idx < kPage * D; idx += blockDim.x) {
+        const int t = idx / D, c = idx % D;
+        int off, bit;
+        vcode_pos(NG, t, c, off, bit);
+        S.vcode[t][c] = (uint8_t)((*reinterpret_cast<const uint32_t *>(vb + off) >> bit) & 3u);
     }
     const uint16_t *h = reinterpret_cast<const uint16_t *>(S.blk);
     for (int idx = threadIdx.x; idx < kPage * NG; idx += blockDim.x) {
@@ -126,33 +118,26 @@ template <int D>
 __device__ void pack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
     constexpr int NG = D / kGroup;
     uint32_t *w = reinterpret_cast<uint32_t *>(S.blk);
-    for (int idx = threadIdx.x; idx < 2 * 32 * NG; idx += blockDim.x) {
-        const bool is_v = idx >= 32 * NG;
-        const int widx = is_v ? idx - 32 * NG : idx;
+    for (int widx = threadIdx.x; widx < 32 * NG; widx += blockDim.x) {
         const int lane = widx / NG, W = widx % NG, gid = lane >> 2, tig = lane & 3;
         uint32_t word = 0;
-        if (!is_v) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int f = 0; f < 4; ++f) {
-                    const int g = f % NG, r = W + NG * (f / NG);
-                    word |= ((uint32_t)S.kcode[gid + 8 * (r & 1)][32 * g + 16 * (r >> 1) + 4 * tig + j] & 3u)
-                            << (8 * j + 2 * f);
-                }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int q = W * 8 + i;
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int tb = q & 1, cr = (q >> 1) & 1, m = q >> 2;
-                    word |= ((uint32_t)S.vcode[8 * tb + 2 * tig + e][16 * m + 8 * cr + gid] & 3u)
-                            << (16 * e + 2 * i);
-                }
+            for (int f = 0; f < 4; ++f) {
+                const int g = f % NG, r = W + NG * (f / NG);
+                word |= ((uint32_t)S.kcode[gid + 8 * (r & 1)][32 * g + 16 * (r >> 1) + 4 * tig + j] & 3u)
+                        << (8 * j + 2 * f);
             }
-        }
-        w[((is_v ? L.vc : L.kc) >> 2) + widx] = word;
+        w[(L.kc >> 2) + widx] = word;
+        w[(L.vc >> 2) + widx] = 0u;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < kPage * D; idx += blockDim.x) {
+        const int t = idx / D, c = idx % D;
+        int off, bit;
+        vcode_pos(NG, t, c, off, bit);
+        atomicOr(&w[(L.vc + off) >> 2], ((uint32_t)S.vcode[t][c] & 3u) << bit);
     }
     uint16_t *h = reinterpret_cast<uint16_t *>(S.blk);
     for (int idx = threadIdx.x; idx < kPage * NG; idx += blockDim.x) {

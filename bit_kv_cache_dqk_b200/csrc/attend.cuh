@@ -123,6 +123,14 @@ struct AttendTile {
     static constexpr int NM = D / 16;          // m-tiles of the PV product
 };
 
+// Factor that turns the PV accumulator of m-tile m into value units: 2^(24 - 2P)
+// for the subnormal operands of the NG = 4 layout, 1 otherwise.
+template <int NG>
+__device__ __forceinline__ float vfield_scale(int m) {
+    if constexpr (NG == 4) return __int_as_float((127 + 24 - 2 * (m <= 4 ? m : m - 5)) << 23);
+    else return 1.0f;
+}
+
 // Online-softmax state of one consumer warp for one (run, kv head).
 template <int D, int G>
 struct WarpState {
@@ -196,6 +204,15 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
         const uint32_t msk = 0x03030303u << (2 * g);   // group g's field in every byte: code * 4^g
+        uint2 qb[NT];
+        float4 kp[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            qb[nt] = ld_s64(o.sq + (nt * NG + g) * 256);
+            const uint4 kpu = ld_s128(o.sk + (nt * NG + g) * 64);
+            kp[nt] = make_float4(__uint_as_float(kpu.x), __uint_as_float(kpu.y), __uint_as_float(kpu.z),
+                                 __uint_as_float(kpu.w));
+        }
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
             uint32_t A0, A1, A2, A3;
@@ -211,16 +228,13 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 int dg[4];
-                const uint2 qb = ld_s64(o.sq + (nt * NG + g) * 256);
-                mma_u8s8(dg, A0, A1, A2, A3, qb.x, qb.y, kMagicI);
+                mma_u8s8(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y, kMagicI);
                 // (M + I) * kappa - M * kappa = I * kappa, one rounding
-                const uint4 kpu = ld_s128(o.sk + (nt * NG + g) * 64);
-                const float4 kp = make_float4(__uint_as_float(kpu.x), __uint_as_float(kpu.y),
-                                              __uint_as_float(kpu.z), __uint_as_float(kpu.w));
-                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[0]), kp.x, kp.z), a0[b][nt]);
-                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[1]), kp.y, kp.w), a0[b][nt]);
-                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[2]), kp.x, kp.z), a1[b][nt]);
-                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[3]), kp.y, kp.w), a1[b][nt]);
+                const float4 k4 = kp[nt];
+                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[0]), k4.x, k4.z), a0[b][nt]);
+                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[1]), k4.y, k4.w), a0[b][nt]);
+                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[2]), k4.x, k4.z), a1[b][nt]);
+                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[3]), k4.y, k4.w), a1[b][nt]);
             }
         }
     }
@@ -319,18 +333,41 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
             pb1[nt] = prmt(w0, w1, 0x7632u);   // tokens 2tig+8, 2tig+9
             mma_f16(st.macc[nt], vma, 0u, vmb, 0u, pb0[nt], pb1[nt]);
         }
+        if constexpr (NG == 4) {
+            // m-tile m is field m of the four words; as fp16 subnormals the
+            // fields read code * 4^P * 2^-24 (P = m, or m - 5 after >> 10),
+            // undone by vfield_scale when the run is finished
+            uint32_t vh[4];
 #pragma unroll
-        for (int w2 = 0; w2 < NG; ++w2) {       // word w2 holds m-tiles 2*w2, 2*w2+1 (= group w2)
-            const uint32_t x = vw[w2], xh = x >> 10;
-            const uint32_t e0 = code_field<0>(x, xh), e2 = code_field<2>(x, xh);
-            const uint32_t e1 = code_field<1>(x, xh), e3 = code_field<3>(x, xh);
-            const uint32_t f0 = code_field<4>(x, xh), f2 = code_field<6>(x, xh);
-            const uint32_t f1 = code_field<5>(x, xh), f3 = code_field<7>(x, xh);
+            for (int k = 0; k < 4; ++k) vh[k] = vw[k] >> 10;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint32_t b0 = hmul2(pb0[nt], vsa[w2]), b1 = hmul2(pb1[nt], vsb[w2]);
-                mma_f16(st.oacc[nt][2 * w2], e0, e2, e1, e3, b0, b1);
-                mma_f16(st.oacc[nt][2 * w2 + 1], f0, f2, f1, f3, b0, b1);
+            for (int g = 0; g < NG; ++g) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint32_t b0 = hmul2(pb0[nt], vsa[g]), b1 = hmul2(pb1[nt], vsb[g]);
+#pragma unroll
+                    for (int mm = 2 * g; mm < 2 * g + 2; ++mm) {
+                        const int P = mm <= 4 ? mm : mm - 5;
+                        const uint32_t msk = 0x00030003u << (2 * P);
+                        const uint32_t (&src)[4] = mm <= 4 ? vw : vh;
+                        mma_f16(st.oacc[nt][mm], src[0] & msk, src[1] & msk, src[2] & msk, src[3] & msk, b0, b1);
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int w2 = 0; w2 < NG; ++w2) {   // word w2 holds m-tiles 2*w2, 2*w2+1 (= group w2)
+                const uint32_t x = vw[w2], xh = x >> 10;
+                const uint32_t e0 = code_field<0>(x, xh), e2 = code_field<2>(x, xh);
+                const uint32_t e1 = code_field<1>(x, xh), e3 = code_field<3>(x, xh);
+                const uint32_t f0 = code_field<4>(x, xh), f2 = code_field<6>(x, xh);
+                const uint32_t f1 = code_field<5>(x, xh), f3 = code_field<7>(x, xh);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint32_t b0 = hmul2(pb0[nt], vsa[w2]), b1 = hmul2(pb1[nt], vsb[w2]);
+                    mma_f16(st.oacc[nt][2 * w2], e0, e2, e1, e3, b0, b1);
+                    mma_f16(st.oacc[nt][2 * w2 + 1], f0, f2, f1, f3, b0, b1);
+                }
             }
         }
     }
@@ -557,8 +594,9 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
                 for (int m = 0; m < NM; ++m) {
                     const int c0 = 16 * m + gid, c1 = c0 + 8;
                     const float mt = minterm[m >> 1];
-                    rec[2 + c0] = (VCH0 && c0 == 0) ? v0t : st.oacc[nt][m][0] + mt;
-                    rec[2 + c1] = st.oacc[nt][m][2] + mt;
+                    const float f = vfield_scale<NG>(m);
+                    rec[2 + c0] = (VCH0 && c0 == 0) ? v0t : fmaf(st.oacc[nt][m][0], f, mt);
+                    rec[2 + c1] = fmaf(st.oacc[nt][m][2], f, mt);
                 }
             }
         }

@@ -56,12 +56,21 @@ __host__ __device__ __forceinline__ void kcode_pos(int ng, int t, int c, int &wo
 }
 
 // Value code of (token t, channel c): the A operand of an m16n8k16 tile with
-// channels as rows and tokens as columns (O^T = V^T P).
+// channels as rows and tokens as columns (O^T = V^T P).  NG = 4: register k of
+// m-tile m (rows 16m + gid + 8*(k&1), columns 2*tig + 8*(k>>1) + e) is word k
+// of the lane, field m of half e, so each m-tile reads one field position of
+// all four words (one AND each, no shift for fields 0..4).  NG = 2: the
+// m-tiles' registers follow each other through the fields of the two words.
 __host__ __device__ __forceinline__ void vcode_pos(int ng, int t, int c, int &word_off, int &bit) {
-    int m = c >> 4, r = c & 15, cr = r >> 3, gid = r & 7;
-    int tb = t >> 3, tig = (t & 7) >> 1, e = t & 1;
-    int lane = gid * 4 + tig;
-    int q = (m * 2 + cr) * 2 + tb;
+    const int m = c >> 4, r = c & 15, cr = r >> 3, gid = r & 7;
+    const int tb = t >> 3, tig = (t & 7) >> 1, e = t & 1;
+    const int lane = gid * 4 + tig;
+    if (ng == 4) {
+        word_off = (lane * 4 + cr + 2 * tb) * 4;
+        bit = e * 16 + 2 * m;
+        return;
+    }
+    const int q = (m * 2 + cr) * 2 + tb;
     word_off = (lane * ng + (q >> 3)) * 4;
     bit = e * 16 + 2 * (q & 7);
 }

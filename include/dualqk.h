@@ -104,7 +104,8 @@ typedef struct {
  *   VC = K0 + 32      V codes, 4*d bytes: (t, c) is in the word at
  *                     VC + 4*(lane*NG + W), bit 16*e + 2*i, with m=c/16,
  *                     cr=(c%16)/8, tb=t/8, tig=(t%8)/2, e=t%2,
- *                     lane=4*(c%8)+tig, q=(2m+cr)*2+tb, W=q/8, i=q%8.
+ *                     lane=4*(c%8)+tig; NG=4: W=cr+2*tb, i=m;
+ *                     NG=2: q=(2m+cr)*2+tb, W=q/8, i=q%8.
  *   VS = VC + 4d      V scale fp16, (t, g) at index 2*(NG*(t/2) + g) + t%2
  *   VM = VS + 32*NG   V min fp16, same indexing
  *   V0 = VM + 32*NG   V channel 0 BF16 [t] (only with v_ch0_protect)

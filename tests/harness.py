@@ -145,9 +145,13 @@ def _code_tables(d):
             kb[t, c] = 8 * j + 2 * (g + ng * (r // ng))
             m, cr, tb, tig, e = c // 16, (c % 16) // 8, t // 8, (t % 8) // 2, t % 2
             lane = 4 * (c % 8) + tig
-            q = (2 * m + cr) * 2 + tb
-            vw[t, c] = lane * ng + q // 8
-            vb[t, c] = 16 * e + 2 * (q % 8)
+            if ng == 4:
+                vw[t, c] = lane * ng + cr + 2 * tb
+                vb[t, c] = 16 * e + 2 * m
+            else:
+                q = (2 * m + cr) * 2 + tb
+                vw[t, c] = lane * ng + q // 8
+                vb[t, c] = 16 * e + 2 * (q % 8)
     return kw, kb, vw, vb
 
 
