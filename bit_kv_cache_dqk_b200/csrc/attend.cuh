@@ -9,8 +9,9 @@
 // whatever the length mix.  A producer warp brings whole units in with 1-D bulk
 // async copies (one copy = 16 tokens x up to 8 kv heads, contiguous) into a
 // ring of shared-memory stages of 16 (page, kv head) blocks guarded by
-// mbarriers.  8 consumer warps each own one kv head and take two pages of it
-// per stage, processed together (two independent instruction streams).
+// mbarriers.  Consumer warps each own one kv head and take two pages of it per
+// stage, processed together (two independent instruction streams); a stage
+// holds two pages per consumer warp.
 //
 // Per consumer warp and page (16 tokens x G query heads), with
 // qs = q' * log2(e)/sqrt(d) on the kept channels:
@@ -26,22 +27,24 @@
 //        with p~ = fp16(p); one extra m16n8k16 gives sum_t p~ * vmin[t, g] and
 //        l = sum_t p~ (a row of ones), so numerator and denominator see the
 //        same rounded weights.
-// Value codes become exact fp16 operands with one LOP3 and one HSUB2 per pair.
+// Value codes become exact fp16 operands with one AND per register: with
+// head_dim 128 as subnormals (code * 4^P * 2^-24, P the field position, the
+// power of two removed when a run is finished), with head_dim 64 through a
+// magic exponent and one HSUB2.
 #pragma once
 
 #include "common.cuh"
 #include "ptx.cuh"
 
-#ifndef ATTEND_BLOCKS_PER_WARP
-#define ATTEND_BLOCKS_PER_WARP 2
-#endif
-
 namespace dqk {
 
-constexpr int kStageBlocks = 16;                            // (page, kv head) blocks per stage
-constexpr int kBlocksPerWarp = ATTEND_BLOCKS_PER_WARP;      // pages of its kv head a warp takes per stage
-constexpr int kConsumerWarps = kStageBlocks / kBlocksPerWarp;
-constexpr int kAttendThreads = (kConsumerWarps + 1) * 32;   // + 1 producer warp
+// CTA shape of k_attend: consumer warps each take two pages of one kv head per
+// stage, plus one producer warp.  16 consumer warps (two per kv head of a
+// chunk of 8) where the per-warp state fits 96 registers; 8 for G = 8, whose
+// two query-head tiles double that state.
+__host__ __device__ constexpr int attend_warps(int G) { return G > 4 ? 8 : 16; }
+__host__ __device__ constexpr int attend_stage_blocks(int G) { return 2 * attend_warps(G); }
+__host__ __device__ constexpr int attend_threads(int G) { return 32 * (attend_warps(G) + 1); }
 constexpr int kMaxStages = 8;                               // ring depth cap
 constexpr uint64_t kWaitLimitNs = 1000000000ull;            // 1 s: a stuck pipeline reports DQK_ERR_TIMEOUT
 
@@ -374,8 +377,9 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
 }
 
 template <int D, int G, bool VCH0>
-__global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams p) {
+__global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendParams p) {
     using T = AttendTile<D, G>;
+    constexpr int kConsumerWarps = attend_warps(G), kStageBlocks = attend_stage_blocks(G);
     constexpr int NG = T::NG, NT = T::NT, NM = T::NM;
     extern __shared__ __align__(128) unsigned char attend_smem[];
     const int S = p.stages;
@@ -488,7 +492,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     }
 
     // ---------------------------------------------------------------- consumers
-    // warp: kv head jl of the chunk, page group pi of each stage (pages kBlocksPerWarp*pi + 0..)
+    // warp: kv head jl of the chunk, page pair pi of each stage (pages 2*pi, 2*pi + 1)
     const int jl = warp % p.hc, pi = warp / p.hc;
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
@@ -620,9 +624,9 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
     bool ok = true;
     int stage = 0;
     uint32_t phase = 0;
-    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((kBlocksPerWarp * pi * p.hc + jl) * p.bb);
+    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((2 * pi * p.hc + jl) * p.bb);
     const uint32_t pair_gap = (uint32_t)(p.hc * p.bb);
-    const uint32_t valid_addr = smem_addr(valid) + kBlocksPerWarp * pi;
+    const uint32_t valid_addr = smem_addr(valid) + 2 * pi;
     for (int it = 0; it < iters; ++it) {
         if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
             if (lane == 0) {
@@ -632,38 +636,28 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
             ok = false;
             break;
         }
-        const int ua = u0 + it * pps + kBlocksPerWarp * pi;
+        const int ua = u0 + it * pps + 2 * pi;
         if (ua < u1) {
             const uint32_t sa = blk_a + (uint32_t)stage * stage_bytes;
-            if constexpr (kBlocksPerWarp == 2) {
-                const int ub = ua + 1;
-                const uint32_t vv = ld_s16(valid_addr + stage * kStageBlocks);   // flags of slots 2pi, 2pi+1
-                if (ua >= run_end) switch_run(ua);
-                if (ub < run_end && ub < u1 && ub != partial_u && vv == 0x0101u) {
-                    const uint32_t sbb[2] = {sa, sa + pair_gap};
-                    consume<D, G, VCH0, 2, false>(sbb, kPage, st, lane, lo);
-                } else {
-                    const uint32_t s1[1] = {sa};
-                    if (vv & 0xffu) {
-                        if (ua == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
-                        else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);
-                    }
-                    if (ub < u1) {
-                        if (ub >= run_end) switch_run(ub);
-                        const uint32_t s2[1] = {sa + pair_gap};
-                        if (vv >> 8) {
-                            if (ub == partial_u) consume<D, G, VCH0, 1, true>(s2, nv_last, st, lane, lo);
-                            else consume<D, G, VCH0, 1, false>(s2, kPage, st, lane, lo);
-                        }
-                    }
-                }
+            const int ub = ua + 1;
+            const uint32_t vv = ld_s16(valid_addr + stage * kStageBlocks);   // flags of slots 2pi, 2pi+1
+            if (ua >= run_end) switch_run(ua);
+            if (ub < run_end && ub < u1 && ub != partial_u && vv == 0x0101u) {
+                const uint32_t sbb[2] = {sa, sa + pair_gap};
+                consume<D, G, VCH0, 2, false>(sbb, kPage, st, lane, lo);
             } else {
-                const uint32_t vv = ld_s8(valid_addr + stage * kStageBlocks);
-                if (ua >= run_end) switch_run(ua);
                 const uint32_t s1[1] = {sa};
-                if (vv) {
+                if (vv & 0xffu) {
                     if (ua == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
                     else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);
+                }
+                if (ub < u1) {
+                    if (ub >= run_end) switch_run(ub);
+                    const uint32_t s2[1] = {sa + pair_gap};
+                    if (vv >> 8) {
+                        if (ub == partial_u) consume<D, G, VCH0, 1, true>(s2, nv_last, st, lane, lo);
+                        else consume<D, G, VCH0, 1, false>(s2, kPage, st, lane, lo);
+                    }
                 }
             }
         }
@@ -681,25 +675,30 @@ __global__ void __launch_bounds__(kAttendThreads, 1) k_attend(const AttendParams
 // log-sum-exp combine: out[b][h] = sum_i o_i 2^(m_i - m*) / sum_i l_i 2^(m_i - m*)
 // over the records of every CTA (and page slot) that held pages of (b, h).
 // ---------------------------------------------------------------------------
-constexpr int kCombineChunk = 64;      // records read per pass
-constexpr int kCombineThreads = 256;   // small enough to sit beside an attend CTA on its SM
+constexpr int kCombineChunk = 96;      // records read per pass
+constexpr int kCombineThreads = 256;
 
-// One CTA per (sequence, query head).  Each pass reads a chunk of records in
-// one round: (m_i, l_i) into shared memory, and thread (slice, channel) the
-// channel of records i = slice (mod slices).  The running max moves from
-// chunk to chunk with an exact rescale.  Every warp forms the chunk's max and
-// denominator with the same lane order and shuffle tree, and the slices are
-// summed in a fixed order, so the result does not depend on scheduling.
+// One CTA per (sequence, query head).  The record indices are worked out
+// before the attend kernel has finished.  Each pass then reads a chunk of
+// records in one round -- (m_i, l_i) into shared memory, and thread (slice,
+// channel) the channel of records i = slice (mod slices) into registers --
+// forms the weights 2^(m_i - m*) once per record, and accumulates.  The
+// running max moves from chunk to chunk with an exact rescale.  Maxima and
+// denominators are reduced in a fixed order, so the result does not depend on
+// scheduling.
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restrict__ seq_lens, int batch, int hq,
                                                              int hkv, int hc, int pw, int nchunks, int num_ctas,
                                                              const float *__restrict__ part, float *__restrict__ out) {
     constexpr int kSlices = kCombineThreads / D;
     constexpr int kPer = kCombineChunk / kSlices;   // records of a chunk per thread
+    constexpr int kWarps = kCombineThreads / 32;
+    static_assert(kCombineChunk <= kCombineThreads, "one record per thread when forming weights");
     __shared__ long long sh_U, sh_ur;
     __shared__ int sh_np;
     __shared__ int sh_rec[kCombineChunk];   // record index of slot i of the chunk, -1 for none
-    __shared__ float sh_m[kCombineChunk], sh_l[kCombineChunk];
+    __shared__ float sh_m[kCombineChunk], sh_l[kCombineChunk], sh_w[kCombineChunk];
+    __shared__ float sh_red[kWarps];
     __shared__ float sh_acc[kSlices][D];
     const int h = blockIdx.x, b = blockIdx.y;
     const int G = hq / hkv, j = h / G, chunk = j / hc, jl = j % hc, hh = h % G;
@@ -731,7 +730,6 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restri
     const int cf = np > 0 ? (int)cta_of_unit(ur, U, num_ctas) : 0;
     const int cl = np > 0 ? (int)cta_of_unit(ur + np - 1, U, num_ctas) : -1;
     const int nrec = (cl - cf + 1) * pw;
-    // record slots of chunk i0 (known before the attend kernel has finished)
     auto index_chunk = [&](int i0) {
         for (int i = threadIdx.x; i < kCombineChunk; i += blockDim.x) {
             int ri = -1;
@@ -771,28 +769,36 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restri
             ov[k] = ri >= 0 ? part[(size_t)ri * (2 + D) + 2 + ch] : 0.0f;
         }
         __syncthreads();
+        // chunk max (every warp, same order), weights once per record
         float cm = -INFINITY;
         for (int i = lane; i < n; i += 32) cm = fmaxf(cm, sh_m[i]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
         const float mnew = fmaxf(mrun, cm);
-        if (mnew == -INFINITY) continue;   // no tokens yet
-        const float alpha = exp2f(mrun - mnew);   // 0 while mrun is -inf
+        if (mnew == -INFINITY) continue;   // no tokens yet (uniform)
         float dpart = 0.0f;
-        for (int i = lane; i < n; i += 32) {
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
             const float mi = sh_m[i];
-            if (mi != -INFINITY) dpart += exp2f(mi - mnew) * sh_l[i];
+            const float wi = mi == -INFINITY ? 0.0f : exp2f(mi - mnew);
+            sh_w[i] = wi;
+            dpart = fmaf(wi, sh_l[i], dpart);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) dpart += __shfl_xor_sync(0xffffffffu, dpart, off);
-        dsum = dsum * alpha + dpart;
+        if (lane == 0) sh_red[warp] = dpart;
+        __syncthreads();
+        float dchunk = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) dchunk += sh_red[k];
+        const float alpha = exp2f(mrun - mnew);   // 0 while mrun is -inf
+        dsum = dsum * alpha + dchunk;
         acc *= alpha;
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
             const int i = slice + kSlices * k;
             if (i < n) {
-                const float mi = sh_m[i];
-                if (mi != -INFINITY) acc = fmaf(exp2f(mi - mnew), ov[k], acc);
+                const float wi = sh_w[i];
+                if (wi != 0.0f) acc = fmaf(wi, ov[k], acc);   // empty records hold no o values
             }
         }
         mrun = mnew;

@@ -56,15 +56,16 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.NT = P.G > 4 ? 2 : 1;
     P.NG = P.d / kGroup;
     const int hkv = L->num_kv_heads;
-    if (hkv <= kConsumerWarps) {
-        if (kConsumerWarps % hkv) return false;
+    const int warps = attend_warps(P.G), stage_blocks = attend_stage_blocks(P.G);
+    if (hkv <= warps) {
+        if (warps % hkv) return false;
         P.hc = hkv;
     } else {
-        if (hkv % kConsumerWarps) return false;
-        P.hc = kConsumerWarps;
+        if (hkv % warps) return false;
+        P.hc = warps;
     }
-    P.pps = kStageBlocks / P.hc;    // pages per stage
-    P.pw = kConsumerWarps / P.hc;   // warps per kv head (each takes 2 pages of a stage)
+    P.pps = stage_blocks / P.hc;    // pages per stage
+    P.pw = warps / P.hc;            // warps per kv head (each takes 2 pages of a stage)
     P.nchunks = hkv / P.hc;
     if ((long long)batch * P.nchunks * (L->num_pages + 1) >= (1LL << 31)) return false;
     // Records are sized for kMaxAttendCtas so the workspace size does not depend
@@ -72,9 +73,9 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.num_ctas = kMaxAttendCtas;
     P.bb = make_layout(P.d, L->v_ch0_protect).bytes;
     // shared memory: ring stages | mbarriers | valid flags | abort flag | per-warp query fragments
-    const size_t stage_bytes = (size_t)kStageBlocks * P.bb;
-    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * kStageBlocks + 16 +
-                         (size_t)kConsumerWarps * P.NT * P.NG * (32 * 8 + 4 * 16);
+    const size_t stage_bytes = (size_t)stage_blocks * P.bb;
+    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * stage_blocks + 16 +
+                         (size_t)warps * P.NT * P.NG * (32 * 8 + 4 * 16);
     const size_t budget = 227 * 1024;
     P.stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / stage_bytes);
     if (P.stages < 2) return false;
@@ -184,7 +185,7 @@ dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
     prm.v_ch0 = a.L->v_ch0_protect;
     prm.stages = P.stages;
     prm.num_ctas = P.num_ctas;
-    return launch_pdl(k_attend<D, G, VCH0>, dim3(P.num_ctas), dim3(kAttendThreads), P.smem, a.stream, prm);
+    return launch_pdl(k_attend<D, G, VCH0>, dim3(P.num_ctas), dim3(attend_threads(G)), P.smem, a.stream, prm);
 }
 
 template <int D, bool VCH0>
