@@ -376,6 +376,115 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
     }
 }
 
+// Every (run, page slot, kv head) record a consumer warp could own starts
+// empty (m = -inf, l = 0): a run shorter than the page slots of a stage
+// leaves some warps without a page of it.
+__device__ __forceinline__ void init_records(const AttendParams &p, int u0, int u1, int slot_base, int pi, int jl,
+                                             int G, int D, int lane) {
+    const int R = p.batch * p.nchunks;
+    int r;
+    long long urll;
+    warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
+    int ur = (int)urll;
+    int np = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
+    while (r < R && ur < u1) {
+        if (np > 0 && lane < G) {
+            float *rec = p.part + record_index(slot_base + r, pi, jl, lane, p.pw, p.hc, G) * (2 + D);
+            rec[0] = -INFINITY;
+            rec[1] = 0.0f;
+        }
+        ur += np;
+        ++r;
+        np = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
+    }
+}
+
+// The producer warp of the attend kernels: brings the CTA's units [u0, u1)
+// into the ring, pps pages (each hc blocks, one bulk copy) per stage, marks
+// which page slots of a stage hold a page, and never leaves with copies in
+// flight.  Waits are bounded; a stuck pipeline sets the abort flag.
+__device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned char *stage_mem, uint64_t *full,
+                                                uint64_t *empty, unsigned char *valid, volatile int *abort_flag,
+                                                int S, uint32_t stage_bytes, int kStageBlocks, int u0, int u1,
+                                                int iters, int lane) {
+    const int R = p.batch * p.nchunks;
+    const int pps = p.pps;
+    grid_dependents_launch();   // the combine kernel may start its prologue
+    if (iters == 0) return;
+    int r;
+    long long urll;
+    warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
+    int ur = (int)urll;
+    int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
+    const uint32_t copy_bytes = (uint32_t)(p.hc * p.bb);
+    // pool byte offset of unit ubase + lane (or -1); moves the cursor to unit ubase + 32
+    auto fetch = [&](int ubase) -> long long {
+        const int u = ubase + lane;
+        int rr = r, st = ur, np = npr;
+        while (rr < R && u >= st + np) {
+            st += np;
+            ++rr;
+            np = rr < R ? run_pages(p.seq_lens, p.nchunks, rr) : 0;
+        }
+        long long off = -1;
+        if (u < u1 && rr < R) {
+            const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
+            const int page = u - st;
+            if (page < p.max_pages) {
+                const int phys = p.page_table[(size_t)b * p.max_pages + page];
+                if (phys >= 0 && phys < p.num_pages)
+                    off = ((long long)phys * p.hkv + (long long)chunk * p.hc) * p.bb;
+            }
+            if (off < 0) dqk_flag_error(kErrBounds);
+        }
+        r = __shfl_sync(0xffffffffu, rr, 31);
+        ur = __shfl_sync(0xffffffffu, st, 31);
+        npr = __shfl_sync(0xffffffffu, np, 31);
+        return off;
+    };
+    long long off_next = fetch(u0);
+    int it = 0, stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int ubase = u0; ubase < u1 && ok; ubase += 32) {
+        const long long off_cur = off_next;
+        if (ubase + 32 < u1) off_next = fetch(ubase + 32);
+        for (; it < iters && u0 + it * pps < ubase + 32; ++it) {
+            int good = 1;
+            if (lane == 0)
+                good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs, 2000u) && !*abort_flag;
+            if (!__shfl_sync(0xffffffffu, good, 0)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    dqk_flag_error(kErrTimeout);
+                }
+                ok = false;
+                break;
+            }
+            // lane k < pps fills page slot k of this stage
+            const int uk = u0 + it * pps + lane;
+            const long long off = __shfl_sync(0xffffffffu, off_cur, (uk - ubase) & 31);
+            const bool have = lane < pps && uk < u1 && off >= 0;
+            const unsigned ballot = __ballot_sync(0xffffffffu, have);
+            if (lane < pps) valid[stage * kStageBlocks + lane] = have ? 1 : 0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(ballot) * copy_bytes);
+            __syncwarp();
+            if (have)
+                bulk_copy_g2s(stage_mem + (size_t)stage * stage_bytes + (size_t)lane * copy_bytes, p.pool + off,
+                              copy_bytes, &full[stage]);
+            if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+    // never leave with copies in flight (exit path: wait, bounded, for the last round of each stage)
+    if (lane == 0)
+        for (int k = it - 1; k >= 0 && k >= it - S; --k)
+            (void)mbar_wait_bounded(&full[k % S], (uint32_t)(k / S) & 1u, kWaitLimitNs);
+}
+
 template <int D, int G, bool VCH0>
 __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendParams p) {
     using T = AttendTile<D, G>;
@@ -413,81 +522,8 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const int iters = (nunits + pps - 1) / pps;
 
     if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        grid_dependents_launch();   // the combine kernel may start its prologue
-        if (iters == 0) return;
-        int r;
-        long long urll;
-        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
-        int ur = (int)urll;
-        int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-        const uint32_t copy_bytes = (uint32_t)(p.hc * p.bb);
-        // pool byte offset of unit ubase + lane (or -1); moves the cursor to unit ubase + 32
-        auto fetch = [&](int ubase) -> long long {
-            const int u = ubase + lane;
-            int rr = r, st = ur, np = npr;
-            while (rr < R && u >= st + np) {
-                st += np;
-                ++rr;
-                np = rr < R ? run_pages(p.seq_lens, p.nchunks, rr) : 0;
-            }
-            long long off = -1;
-            if (u < u1 && rr < R) {
-                const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
-                const int page = u - st;
-                if (page < p.max_pages) {
-                    const int phys = p.page_table[(size_t)b * p.max_pages + page];
-                    if (phys >= 0 && phys < p.num_pages)
-                        off = ((long long)phys * p.hkv + (long long)chunk * p.hc) * p.bb;
-                }
-                if (off < 0) dqk_flag_error(kErrBounds);
-            }
-            r = __shfl_sync(0xffffffffu, rr, 31);
-            ur = __shfl_sync(0xffffffffu, st, 31);
-            npr = __shfl_sync(0xffffffffu, np, 31);
-            return off;
-        };
-        long long off_next = fetch(u0);
-        int it = 0, stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        for (int ubase = u0; ubase < u1 && ok; ubase += 32) {
-            const long long off_cur = off_next;
-            if (ubase + 32 < u1) off_next = fetch(ubase + 32);
-            for (; it < iters && u0 + it * pps < ubase + 32; ++it) {
-                int good = 1;
-                if (lane == 0)
-                    good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs, 2000u) && !*abort_flag;
-                if (!__shfl_sync(0xffffffffu, good, 0)) {
-                    if (lane == 0) {
-                        *abort_flag = 1;
-                        dqk_flag_error(kErrTimeout);
-                    }
-                    ok = false;
-                    break;
-                }
-                // lane k < pps fills page slot k of this stage
-                const int uk = u0 + it * pps + lane;
-                const long long off = __shfl_sync(0xffffffffu, off_cur, (uk - ubase) & 31);
-                const bool have = lane < pps && uk < u1 && off >= 0;
-                const unsigned ballot = __ballot_sync(0xffffffffu, have);
-                if (lane < pps) valid[stage * kStageBlocks + lane] = have ? 1 : 0;
-                __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(ballot) * copy_bytes);
-                __syncwarp();
-                if (have)
-                    bulk_copy_g2s(stage_mem + (size_t)stage * stage_bytes + (size_t)lane * copy_bytes, p.pool + off,
-                                  copy_bytes, &full[stage]);
-                if (++stage == S) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-        // never leave with copies in flight (exit path: wait, bounded, for the last round of each stage)
-        if (lane == 0)
-            for (int k = it - 1; k >= 0 && k >= it - S; --k)
-                (void)mbar_wait_bounded(&full[k % S], (uint32_t)(k / S) & 1u, kWaitLimitNs);
+        attend_producer(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kStageBlocks, u0, u1, iters,
+                        lane);
         return;
     }
 
@@ -497,25 +533,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
 
-    // Every (run, pair, kv head) record this warp could own starts empty: a run
-    // shorter than the page slots leaves some warps without a page.
-    if (nunits > 0) {
-        int r;
-        long long urll;
-        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
-        int ur = (int)urll;
-        int np = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-        while (r < R && ur < u1) {
-            if (np > 0 && lane < G) {
-                float *rec = p.part + record_index(slot_base + r, pi, jl, lane, p.pw, p.hc, G) * (2 + D);
-                rec[0] = -INFINITY;
-                rec[1] = 0.0f;
-            }
-            ur += np;
-            ++r;
-            np = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-        }
-    }
+    if (nunits > 0) init_records(p, u0, u1, slot_base, pi, jl, G, D, lane);
     if (iters == 0) return;
     grid_dependency_wait();     // query fragments come from k_qprep
 

@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "append.cuh"
 #include "attend.cuh"
+#include "bf16.cuh"
 #include "qprep.cuh"
 
 namespace {
@@ -436,6 +437,166 @@ const char *dqk_status_string(dqk_status s) {
         case DQK_ERR_TIMEOUT: return "DQK_ERR_TIMEOUT";
     }
     return "DQK_UNKNOWN_STATUS";
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// The BF16 comparison decode (paged BF16 cache, no transform / quantization /
+// pruning): append, workspace size, decode.
+// ---------------------------------------------------------------------------
+namespace {
+
+dqk_status check_layer_b16(const dqk_layer_desc *L) {
+    if (!L) return DQK_ERR_INVALID_ARG;
+    if (L->head_dim != 64 && L->head_dim != 128) return DQK_ERR_UNSUPPORTED;
+    if (L->num_kv_heads <= 0 || L->num_q_heads <= 0 || L->num_q_heads % L->num_kv_heads)
+        return DQK_ERR_INVALID_ARG;
+    const int G = L->num_q_heads / L->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return DQK_ERR_UNSUPPORTED;
+    if (L->page_size != kPage) return DQK_ERR_UNSUPPORTED;
+    if (!L->pool || !aligned(L->pool, 16) || L->num_pages <= 0) return DQK_ERR_INVALID_ARG;
+    return DQK_OK;
+}
+
+bool plan_b16(const dqk_layer_desc *L, int batch, DecodePlan &P) {
+    P.d = L->head_dim;
+    P.G = L->num_q_heads / L->num_kv_heads;
+    P.NT = P.G > 4 ? 2 : 1;
+    P.NG = P.d / kGroup;
+    const int hkv = L->num_kv_heads;
+    if (hkv <= kB16Warps) {
+        if (kB16Warps % hkv) return false;
+        P.hc = hkv;
+    } else {
+        if (hkv % kB16Warps) return false;
+        P.hc = kB16Warps;
+    }
+    P.pps = kB16StageBlocks / P.hc;
+    P.pw = kB16Warps / P.hc;
+    P.nchunks = hkv / P.hc;
+    if ((long long)batch * P.nchunks * (L->num_pages + 1) >= (1LL << 31)) return false;
+    P.num_ctas = kMaxAttendCtas;
+    P.bb = b16_block_bytes(P.d);
+    const size_t stage_bytes = (size_t)kB16StageBlocks * P.bb;
+    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * kB16StageBlocks + 16;
+    P.stages = (int)std::min<size_t>(kMaxStages, (227 * 1024 - fixed) / stage_bytes);
+    if (P.stages < 2) return false;
+    P.smem = P.stages * stage_bytes + fixed;
+    const size_t R = (size_t)batch * P.nchunks;
+    const size_t bj = (size_t)batch * hkv;
+    P.off_qf = 256;
+    P.off_qk = P.off_qm = P.off_q0 = 0;
+    P.off_part = round_up(P.off_qf + bj * P.NT * (P.d / 16) * 32 * sizeof(uint2), 256);
+    const size_t records = ((size_t)kMaxAttendCtas + R - 1) * P.pw * P.hc * P.G;
+    P.bytes = round_up(P.off_part + records * (2 + P.d) * sizeof(float), 256);
+    return true;
+}
+
+template <int D, int G>
+dqk_status run_attend_b16(const DecodeArgs &a, const DecodePlan &P) {
+    if (cudaFuncSetAttribute(k_attend_b16<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
+        cudaSuccess)
+        return DQK_ERR_CUDA;
+    char *ws = static_cast<char *>(a.ws);
+    AttendParams prm = {};
+    prm.pool = static_cast<const uint8_t *>(a.L->pool);
+    prm.num_pages = a.L->num_pages;
+    prm.seq_lens = a.seq_lens;
+    prm.page_table = a.page_table;
+    prm.qf = reinterpret_cast<const uint2 *>(ws + P.off_qf);
+    prm.part = reinterpret_cast<float *>(ws + P.off_part);
+    prm.batch = a.batch;
+    prm.hq = a.L->num_q_heads;
+    prm.hkv = a.L->num_kv_heads;
+    prm.hc = P.hc;
+    prm.pps = P.pps;
+    prm.pw = P.pw;
+    prm.nchunks = P.nchunks;
+    prm.max_pages = a.max_pages;
+    prm.bb = P.bb;
+    prm.v_ch0 = 0;
+    prm.stages = P.stages;
+    prm.num_ctas = P.num_ctas;
+    return launch_pdl(k_attend_b16<D, G>, dim3(P.num_ctas), dim3(kB16Threads), P.smem, a.stream, prm);
+}
+
+template <int D>
+dqk_status run_decode_b16(const DecodeArgs &a, const DecodePlan &P) {
+    char *ws = static_cast<char *>(a.ws);
+    const float qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
+    k_qprep_b16<D><<<dim3(a.L->num_kv_heads, a.batch), 128, 0, a.stream>>>(
+        a.q, (int)a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, qscale, reinterpret_cast<uint2 *>(ws + P.off_qf));
+    dqk_status st = launch_status();
+    if (st != DQK_OK) return st;
+    switch (P.G) {
+        case 1: st = run_attend_b16<D, 1>(a, P); break;
+        case 2: st = run_attend_b16<D, 2>(a, P); break;
+        case 4: st = run_attend_b16<D, 4>(a, P); break;
+        default: st = run_attend_b16<D, 8>(a, P); break;
+    }
+    if (st != DQK_OK) return st;
+    return run_combine<D>(a, P);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dqk_bf16_block_bytes(const dqk_layer_desc *layer) {
+    if (!layer || (layer->head_dim != 64 && layer->head_dim != 128)) return 0;
+    return (size_t)b16_block_bytes(layer->head_dim);
+}
+
+dqk_status dqk_bf16_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
+                           const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
+                           int max_pages, dqk_stream_t stream) {
+    dqk_status st = check_layer_b16(layer);
+    if (st != DQK_OK) return st;
+    if (!k || !v || !new_lens || !seq_lens_before || !page_table) return DQK_ERR_INVALID_ARG;
+    if (dtype != DQK_F32 && dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
+    if (batch <= 0 || max_pages <= 0 || max_new < 0) return DQK_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16)) return DQK_ERR_INVALID_ARG;
+    if (max_new == 0) return DQK_OK;
+    const long long gx = (long long)batch * max_new;
+    if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *pool = static_cast<uint8_t *>(layer->pool);
+    if (layer->head_dim == 128)
+        k_append_b16<128><<<dim3((unsigned)gx, layer->num_kv_heads), 2 * 128 / 8, 0, s>>>(
+            k, v, dtype, new_lens, seq_lens_before, page_table, max_pages, max_new, pool, layer->num_pages,
+            layer->num_kv_heads);
+    else
+        k_append_b16<64><<<dim3((unsigned)gx, layer->num_kv_heads), 2 * 64 / 8, 0, s>>>(
+            k, v, dtype, new_lens, seq_lens_before, page_table, max_pages, max_new, pool, layer->num_pages,
+            layer->num_kv_heads);
+    return launch_status();
+}
+
+size_t dqk_bf16_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max_pages) {
+    if (check_layer_b16(layer) != DQK_OK || batch <= 0 || max_pages <= 0) return 0;
+    DecodePlan P;
+    if (!plan_b16(layer, batch, P)) return 0;
+    return P.bytes;
+}
+
+dqk_status dqk_bf16_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype, int batch,
+                           const int *seq_lens, const int *page_table, int max_pages, float *out, void *workspace,
+                           size_t workspace_bytes, dqk_stream_t stream) {
+    dqk_status st = check_layer_b16(layer);
+    if (st != DQK_OK) return st;
+    if (!q || !seq_lens || !page_table || !out || !workspace) return DQK_ERR_INVALID_ARG;
+    if (q_dtype != DQK_F32 && q_dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
+    if (batch <= 0 || max_pages <= 0) return DQK_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || !aligned(out, 16)) return DQK_ERR_INVALID_ARG;
+    DecodePlan P;
+    if (!plan_b16(layer, batch, P)) return DQK_ERR_UNSUPPORTED;
+    if (workspace_bytes < P.bytes) return DQK_ERR_WORKSPACE_TOO_SMALL;
+    P.num_ctas = std::min(device_sms(), kMaxAttendCtas);
+    if (P.num_ctas <= 0) return DQK_ERR_CUDA;
+    DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, 0, out, nullptr,
+                 workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};
+    return layer->head_dim == 128 ? run_decode_b16<128>(a, P) : run_decode_b16<64>(a, P);
 }
 
 }  // extern "C"

@@ -25,7 +25,8 @@ DQK_F32, DQK_BF16 = 0, 1
 
 EXPORTED = ["dqk_block_bytes", "dqk_append", "dqk_decode_workspace_size", "dqk_decode",
             "dqk_decode_step", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine",
-            "dqk_decode_noalloc", "dqk_last_device_error", "dqk_status_string"]
+            "dqk_decode_noalloc", "dqk_bf16_block_bytes", "dqk_bf16_append",
+            "dqk_bf16_decode_workspace_size", "dqk_bf16_decode", "dqk_last_device_error", "dqk_status_string"]
 
 DQK_NOALLOC_WORKSPACE_BYTES = 8 << 20
 
@@ -54,6 +55,14 @@ _lib.dqk_decode_step.argtypes = [_D, _P, _P, C.c_int, _P, _P, C.c_int, _P, C.c_i
                                  C.c_int, _P, _P, _P, C.c_size_t, _P]
 _lib.dqk_decode_noalloc.restype = C.c_int
 _lib.dqk_decode_noalloc.argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P]
+_lib.dqk_bf16_block_bytes.restype = C.c_size_t
+_lib.dqk_bf16_block_bytes.argtypes = [_D]
+_lib.dqk_bf16_append.restype = C.c_int
+_lib.dqk_bf16_append.argtypes = [_D, _P, _P, C.c_int, C.c_int, _P, _P, C.c_int, _P, C.c_int, _P]
+_lib.dqk_bf16_decode_workspace_size.restype = C.c_size_t
+_lib.dqk_bf16_decode_workspace_size.argtypes = [_D, C.c_int, C.c_int]
+_lib.dqk_bf16_decode.restype = C.c_int
+_lib.dqk_bf16_decode.argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, _P, _P, C.c_size_t, _P]
 _lib.dqk_last_device_error.restype = C.c_int
 _lib.dqk_last_device_error.argtypes = [_P]
 _lib.dqk_status_string.restype = C.c_char_p
@@ -161,6 +170,28 @@ def dqk_decode_noalloc(layer, q, q_dtype, batch, seq_lens, page_table, max_pages
     st = _lib.dqk_decode_noalloc(C.byref(layer), _addr(q), q_dtype, batch, _addr(seq_lens), _addr(page_table),
                                  max_pages, sparsity_pct, _addr(out), _addr(sel_out), _stream(stream))
     return _check(st, "dqk_decode_noalloc", raise_on_error)
+
+
+def dqk_bf16_block_bytes(layer: dqk_layer_desc) -> int:
+    return int(_lib.dqk_bf16_block_bytes(C.byref(layer)))
+
+
+def dqk_bf16_append(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages,
+                    stream=None, raise_on_error=True) -> int:
+    st = _lib.dqk_bf16_append(C.byref(layer), _addr(k), _addr(v), dtype, batch, _addr(new_lens),
+                              _addr(seq_lens_before), max_new, _addr(page_table), max_pages, _stream(stream))
+    return _check(st, "dqk_bf16_append", raise_on_error)
+
+
+def dqk_bf16_decode_workspace_size(layer, batch, max_pages) -> int:
+    return int(_lib.dqk_bf16_decode_workspace_size(C.byref(layer), batch, max_pages))
+
+
+def dqk_bf16_decode(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, out, workspace, workspace_bytes,
+                    stream=None, raise_on_error=True) -> int:
+    st = _lib.dqk_bf16_decode(C.byref(layer), _addr(q), q_dtype, batch, _addr(seq_lens), _addr(page_table),
+                              max_pages, _addr(out), _addr(workspace), workspace_bytes, _stream(stream))
+    return _check(st, "dqk_bf16_decode", raise_on_error)
 
 
 def dqk_last_device_error(stream=None) -> int:

@@ -232,6 +232,36 @@ dqk_status dqk_decode_noalloc(const dqk_layer_desc *layer, const void *q, dqk_dt
                               int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
                               dqk_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * The BF16 comparison decode: plain attention over a paged BF16 K/V cache, no
+ * transform, no quantization, no channel pruning -- the baseline the decode
+ * speedup of "Throughput on SGLang" (3.75x over BF16) is quoted against.  It
+ * uses the same dqk_layer_desc (t_k, t_q, group_size and v_ch0_protect are
+ * ignored; pool holds BF16 blocks) and the same page tables.
+ *
+ * Block of (page, kv head), 64*d bytes (8192 at d = 128): K [16][d] then
+ * V [16][d] BF16, token-major; the 16-byte chunk x (channels 8x..8x+7) of
+ * token t is stored at chunk position x ^ (t % 8) of its row.
+ * ------------------------------------------------------------------------- */
+size_t dqk_bf16_block_bytes(const dqk_layer_desc *layer);
+
+/* Copy new K/V rows into the BF16 cache; arguments as dqk_append (k and v
+ * 16-byte aligned; fp32 rows are rounded to BF16, RNE). */
+dqk_status dqk_bf16_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype,
+                           int batch, const int *new_lens, const int *seq_lens_before, int max_new,
+                           const int *page_table, int max_pages, dqk_stream_t stream);
+
+/* Workspace of dqk_bf16_decode (0 = unsupported). */
+size_t dqk_bf16_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max_pages);
+
+/* out = softmax(q.k / sqrt(d)) . v over the first seq_lens[b] cached tokens,
+ * every channel kept; arguments as dqk_decode (no sparsity, no sel_out).
+ * Query pieces and softmax weights are carried as BF16 hi + lo pairs
+ * (about 16 significant bits), accumulation in fp32. */
+dqk_status dqk_bf16_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype, int batch,
+                           const int *seq_lens, const int *page_table, int max_pages, float *out,
+                           void *workspace, size_t workspace_bytes, dqk_stream_t stream);
+
 /* Synchronizes `stream`, then reads and clears the current device's error
  * word: DQK_OK, DQK_ERR_DEVICE_BOUNDS or DQK_ERR_TIMEOUT (DQK_ERR_CUDA if the
  * stream itself reports an error).  All calls on a device share the word. */

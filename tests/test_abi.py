@@ -21,7 +21,7 @@ def Q():
 def header_functions():
     text = open(os.path.join(ROOT, "include", "dualqk.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(dqk_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(dqk_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_function_is_exported(Q):
