@@ -228,23 +228,25 @@ class Layer:
         self.out_host.copy_(self.out, non_blocking=True)
 
     def algorithmic_bytes(self) -> tuple[float, float]:
-        """Bytes the attend kernel must touch per launch (retained-channel key
-        codes for the union of the GQA group's kept channels, K scale/min of
-        touched groups, K channel 0, V codes, V scale/min) and per token-kv-head."""
-        w = self.w
-        sel = self.sel.cpu().numpy()
-        G, ng = w.group, w.d // 32
-        total = 0.0
-        for b in range(w.batch):
-            for j in range(w.hkv):
-                kept = np.zeros(w.d, bool)
-                kept[sel[b, j * G:(j + 1) * G].ravel()] = True
-                kept[0] = False
-                u = int(kept.sum())
-                groups = int(kept.reshape(ng, 32).any(axis=1).sum())
-                per_tok = -(-u // 4) + 4 * groups + 2 + w.d // 4 + 4 * ng
-                total += per_tok * int(self.lens[b])
-        return total, total / (w.hkv * float(self.lens.sum()))
+        return algorithmic_bytes(self.w, self.sel.cpu().numpy(), self.lens)
+
+
+def algorithmic_bytes(w, sel: np.ndarray, lens: np.ndarray) -> tuple[float, float]:
+    """Bytes the attend kernel must touch per launch (retained-channel key
+    codes for the union of the GQA group's kept channels, K scale/min of
+    touched groups, K channel 0, V codes, V scale/min) and per token-kv-head."""
+    G, ng = w.group, w.d // 32
+    total = 0.0
+    for b in range(len(lens)):
+        for j in range(w.hkv):
+            kept = np.zeros(w.d, bool)
+            kept[sel[b, j * G:(j + 1) * G].ravel()] = True
+            kept[0] = False
+            u = int(kept.sum())
+            groups = int(kept.reshape(ng, 32).any(axis=1).sum())
+            per_tok = -(-u // 4) + 4 * groups + 2 + w.d // 4 + 4 * ng
+            total += per_tok * int(lens[b])
+    return total, total / (w.hkv * float(np.sum(lens)))
 
 
 def run_dqk(args):
@@ -421,6 +423,130 @@ def run_reference(args):
     }), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# the sparsity x batch x context sweep against the BF16 comparison decode, and
+# the 64-row append of the ragged Qwen-shaped workload
+# ----------------------------------------------------------------------------
+def _event_time_us(torch, fn, reps, flush):
+    ts = []
+    for r in range(reps):
+        flush.fill_(r & 255)             # L2 flush: 256 MB write
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.median(ts)
+
+
+def run_sweep(args):
+    import torch
+    from bit_kv_cache_dqk_b200 import dualqk as Q
+    from bit_kv_cache_dqk_b200 import inputs as I
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = I.CONFIGS["sweep"]
+    Bmax, Lmax = w.batch, w.ctx
+    lens = np.full(Bmax, Lmax, np.int32)
+    table, num_pages = I.page_table(w, lens)
+    max_pages = table.shape[1]
+    tk, tq, _, _ = I.transforms(w)
+    t_k, t_q = torch.from_numpy(tk).to(dev), torch.from_numpy(tq).to(dev)
+    probe = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, 0, 1)
+    pool = torch.empty(num_pages * w.hkv * Q.dqk_block_bytes(probe), dtype=torch.uint8, device=dev)
+    pool_b = torch.empty(num_pages * w.hkv * Q.dqk_bf16_block_bytes(probe), dtype=torch.uint8, device=dev)
+    desc = Q.layer_desc(w.d, w.hq, w.hkv, t_k, t_q, pool, num_pages)
+    desc_b = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, pool_b, num_pages)
+    table_d = torch.from_numpy(table).to(dev)
+    chunk = 4096
+    new_d = torch.full((Bmax,), chunk, dtype=torch.int32, device=dev)
+    for t0 in range(0, Lmax, chunk):
+        k, v = I.kv_rows_device(w, range(Bmax), t0, t0 + chunk, dev)
+        before = torch.full((Bmax,), t0, dtype=torch.int32, device=dev)
+        Q.dqk_append(desc, k, v, Q.DQK_BF16, Bmax, new_d, before, chunk, table_d, max_pages)
+        Q.dqk_bf16_append(desc_b, k, v, Q.DQK_BF16, Bmax, new_d, before, chunk, table_d, max_pages)
+    torch.cuda.synchronize(dev)
+    q = torch.from_numpy(I.queries(w, lens)).to(torch.bfloat16).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak, peak_kind = measured_peaks()
+    points = []
+    for B in (1, 4, 16):
+        ws_bytes = max(Q.dqk_decode_workspace_size(desc, B, max_pages),
+                       Q.dqk_bf16_decode_workspace_size(desc_b, B, max_pages))
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        out = torch.empty((B, w.hq, w.d), dtype=torch.float32, device=dev)
+        for L in (8192, 32768, 131072):
+            lens_d = torch.full((B,), L, dtype=torch.int32, device=dev)
+            t_b16 = _event_time_us(torch, lambda: Q.dqk_bf16_decode(desc_b, q, Q.DQK_BF16, B, lens_d, table_d,
+                                                                     max_pages, out, ws, ws_bytes), args.reps, flush)
+            b16_bytes = B * L * w.hkv * Q.dqk_bf16_block_bytes(probe) / 16
+            for pct in (0, 20, 40, 60):
+                keep = w.d - (pct * w.d) // 100
+                sel = torch.empty((B, w.hq, keep), dtype=torch.int16, device=dev)
+                t_dqk = _event_time_us(torch, lambda: Q.dqk_decode(desc, q, Q.DQK_BF16, B, lens_d, table_d,
+                                                                   max_pages, pct, out, sel, ws, ws_bytes),
+                                       args.reps, flush)
+                algo, per_tok = algorithmic_bytes(w, sel.cpu().numpy(), np.full(B, L))
+                points.append({"batch": B, "context": L, "sparsity_pct": pct, "dqk_decode_us": t_dqk,
+                               "bf16_decode_us": t_b16, "speedup": t_b16 / t_dqk,
+                               "dqk_kv_tokens_per_s": B * L / (t_dqk * 1e-6),
+                               "dqk_algorithmic_gbs": algo / (t_dqk * 1e-6) / 1e9,
+                               "dqk_bytes_per_token_kv_head": per_tok,
+                               "bf16_gbs": b16_bytes / (t_b16 * 1e-6) / 1e9})
+    print(json.dumps({"metric": "decode time vs BF16 decode over sparsity x batch x context", "unit": "us",
+                      "peak_hbm_gbs": peak, "peak_kind": peak_kind, "reps": args.reps,
+                      "timing": "median of CUDA-event times of one dqk_decode / dqk_bf16_decode call each, "
+                                "256 MB L2 flush before every call",
+                      "data": "synthetic, drawn on the device (torch Philox), random page order",
+                      "config": {"workload": "sweep: 32/8 heads, head_dim 128, BF16 K/V, batch {1,4,16} x "
+                                             "context {8K,32K,128K} x sparsity {0,20,40,60}%"},
+                      "points": points}), flush=True)
+
+
+def run_append64(args):
+    """dqk_append of 64 rows per sequence on the ragged Qwen-shaped layer
+    (batch 16, lengths 4K..64K, Student-t keys), timed alone."""
+    import torch
+    from bit_kv_cache_dqk_b200 import dualqk as Q
+    from bit_kv_cache_dqk_b200 import inputs as I
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = I.CONFIGS["qwen"]
+    lens = I.lengths(w)
+    table, num_pages = I.page_table(w, lens)
+    max_pages = table.shape[1]
+    tk, tq, _, _ = I.transforms(w)
+    t_k, t_q = torch.from_numpy(tk).to(dev), torch.from_numpy(tq).to(dev)
+    probe = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, 0, 1)
+    bb = Q.dqk_block_bytes(probe)
+    pool = torch.empty(num_pages * w.hkv * bb, dtype=torch.uint8, device=dev)
+    desc = Q.layer_desc(w.d, w.hq, w.hkv, t_k, t_q, pool, num_pages)
+    table_d = torch.from_numpy(table).to(dev)
+    n = w.append_new
+    before = (lens - n).astype(np.int32)
+    ks, vs = zip(*[I.kv_rows(w, b, int(before[b]), int(lens[b])) for b in range(w.batch)])
+    k = torch.from_numpy(np.concatenate(ks)).to(torch.bfloat16).to(dev)
+    v = torch.from_numpy(np.concatenate(vs)).to(torch.bfloat16).to(dev)
+    new_d = torch.full((w.batch,), n, dtype=torch.int32, device=dev)
+    before_d = torch.from_numpy(before).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    call = lambda: Q.dqk_append(desc, k, v, Q.DQK_BF16, w.batch, new_d, before_d, n, table_d, max_pages)
+    for _ in range(3):
+        call()
+    t = _event_time_us(torch, call, args.reps, flush)
+    rows = w.batch * n * w.hkv
+    pages_touched = int(sum(((int(lens[b]) - 1) // 16) - (int(before[b]) // 16) + 1 for b in range(w.batch)))
+    print(json.dumps({"metric": "append of 64 rows per sequence (transform + INT2 pack)", "value": t, "unit": "us",
+                      "rows_per_s": rows / (t * 1e-6),
+                      "bytes_in": rows * w.d * 2 * 2, "bytes_out": pages_touched * w.hkv * bb,
+                      "achieved_gbs": (rows * w.d * 4 + 2 * pages_touched * w.hkv * bb) / (t * 1e-6) / 1e9,
+                      "reps": args.reps, "timing": "median of CUDA-event times, 256 MB L2 flush before each call",
+                      "config": {"workload": f"qwen: batch {w.batch}, 32/8 heads, head_dim 128, lengths "
+                                             f"{int(lens.min())}..{int(lens.max())}, {n} rows appended per "
+                                             f"sequence"}}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -431,11 +557,18 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-ctx", type=int, default=16384)
+    ap.add_argument("--sweep", action="store_true", help="sparsity x batch x context sweep vs the BF16 decode")
+    ap.add_argument("--append64", action="store_true", help="time the 64-row append of the qwen workload")
+    ap.add_argument("--reps", type=int, default=10)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
+    elif args.append64:
+        run_append64(args)
     else:
         run_dqk(args)
 

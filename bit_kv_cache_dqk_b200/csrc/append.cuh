@@ -250,35 +250,38 @@ __global__ void __launch_bounds__(512) k_quant_pack(
 }
 
 // ---------------------------------------------------------------------------
-// k_append_rows: the decode-time append (a few rows per sequence).  One CTA
-// of D threads per (new row, kv head); thread c computes k'_c from T_K's row c
-// (read straight from global memory, all loads in flight at once) and warp g
-// quantizes group g.  Only the row's own fields of its (page, kv head) block
-// are written: its key code words (each holds codes of one token) with plain
-// stores, its value code fields (words shared with neighbouring tokens) with
-// atomic and/or, its scale/min/channel-0 entries with 16-bit stores.  Same
-// arithmetic, hence the same bytes, as k_quant_pack.
+// k_append_rows: appends of up to a few dozen rows per sequence (decode steps,
+// speculative or chunked appends).  One CTA of D threads per (group of kRows
+// consecutive new rows of a sequence, kv head); thread c holds T_K's row c in
+// registers (read straight from global memory, all loads in flight at once)
+// and computes k'_c of every row of the group as interleaved independent
+// sums; warp g quantizes group g of each row.  Only the rows' own fields of
+// their (page, kv head) blocks are written: key code words (each holds codes
+// of one token) with plain stores, value code fields (words shared with
+// neighbouring tokens) with atomic and/or, scale/min/channel-0 entries with
+// 16-bit stores.  Same arithmetic, hence the same bytes, as k_quant_pack.
 // ---------------------------------------------------------------------------
-constexpr int kDirectMaxNew = 4;   // dqk_append uses k_append_rows up to this many rows per sequence
+constexpr int kDirectMaxNew = 64;   // dqk_append uses k_append_rows up to this many rows per sequence
+constexpr int kRowsPerCta = 4;
 
 template <int D>
 __global__ void __launch_bounds__(D) k_append_rows(
     const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin, int dtype,
     const int *__restrict__ new_lens, const int *__restrict__ seq_before, const int *__restrict__ page_table,
-    int max_pages, int max_new, uint8_t *__restrict__ pool, long long num_pages, int hkv, int v_ch0,
+    int max_pages, int groups_per_seq, uint8_t *__restrict__ pool, long long num_pages, int hkv, int v_ch0,
     int early_release) {
     constexpr int NG = D / kGroup;
-    __shared__ double xs[D];
-    __shared__ uint32_t kimg[D], kmask[D], vimg[D], vmask[D];   // code regions are D words each
+    constexpr int RW = kRowsPerCta;
+    __shared__ double xs[RW][D];
+    __shared__ uint32_t kimg[RW][D], kmask[RW][D], vimg[RW][D], vmask[RW][D];   // code regions: D words each
     const int j = blockIdx.y;
-    const int b = blockIdx.x / max_new, t = blockIdx.x - b * max_new;
+    const int b = blockIdx.x / groups_per_seq, t0 = (blockIdx.x - b * groups_per_seq) * RW;
     const int c = threadIdx.x, warp = c >> 5, lane = c & 31;
     if (early_release) grid_dependents_launch();
     const int n = new_lens[b];
-    if (t >= n) return;                       // the whole CTA
+    if (t0 >= n) return;                      // the whole CTA
+    const int nr = min(RW, n - t0);           // rows of this CTA
     const int L0 = seq_before[b];
-    const int pos = L0 + t;
-    const int page = pos / kPage, slot = pos - page * kPage;
     // T_K row c, all loads in flight
     const float4 *tr = reinterpret_cast<const float4 *>(t_k + ((size_t)j * D + c) * D);
     float4 tv[D / 4];
@@ -288,66 +291,85 @@ __global__ void __launch_bounds__(D) k_append_rows(
     for (int bb = lane; bb < b; bb += 32) row0 += new_lens[bb];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) row0 += __shfl_xor_sync(0xffffffffu, row0, o);
-    const size_t base = (((size_t)row0 + t) * hkv + j) * D;
-    const float xk = load_elem(kin, dtype, base + c);
-    const float xv = load_elem(vin, dtype, base + c);
-    const int phys = (L0 >= 0 && page < max_pages) ? page_table[(size_t)b * max_pages + page] : -1;
-    xs[c] = (double)xk;
-    kimg[c] = 0u;
-    kmask[c] = 0u;
-    vimg[c] = 0u;
-    vmask[c] = 0u;
+    float xv[RW];
+    int phys[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        const int t = t0 + (i < nr ? i : 0);
+        const size_t base = (((size_t)row0 + t) * hkv + j) * D;
+        xs[i][c] = (double)load_elem(kin, dtype, base + c);
+        xv[i] = load_elem(vin, dtype, base + c);
+        const int page = (L0 + t) / kPage;
+        phys[i] = (L0 >= 0 && page < max_pages) ? page_table[(size_t)b * max_pages + page] : -1;
+        kimg[i][c] = 0u;
+        kmask[i][c] = 0u;
+        vimg[i][c] = 0u;
+        vmask[i][c] = 0u;
+    }
     __syncthreads();
     // k'_c = sum_i T_K[c][i] x_i, ascending i, exact products summed in fp64
-    double acc = 0.0;
+    double acc[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) acc[i] = 0.0;
 #pragma unroll
     for (int u = 0; u < D / 4; ++u) {
-        acc = fma((double)tv[u].x, xs[4 * u + 0], acc);
-        acc = fma((double)tv[u].y, xs[4 * u + 1], acc);
-        acc = fma((double)tv[u].z, xs[4 * u + 2], acc);
-        acc = fma((double)tv[u].w, xs[4 * u + 3], acc);
-    }
-    const float kp = __double2float_rn(acc);
-    if (phys < 0 || phys >= num_pages) {      // the whole CTA
-        if (c == 0) dqk_flag_error(kErrBounds);
-        return;
+        const double t4[4] = {(double)tv[u].x, (double)tv[u].y, (double)tv[u].z, (double)tv[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int i = 0; i < RW; ++i) acc[i] = fma(t4[e], xs[i][4 * u + e], acc[i]);
     }
     const Layout L = make_layout(D, v_ch0);
-    uint8_t *blk = pool + ((size_t)phys * hkv + j) * L.bytes;
-    uint16_t *h16 = reinterpret_cast<uint16_t *>(blk);
-    uint16_t ksh, kmh, vsh, vmh;
-    const int kc = quantize_group(kp, c == 0, ksh, kmh);
-    const int vc = quantize_group(xv, v_ch0 != 0 && c == 0, vsh, vmh);
-    if (lane == 0) {
-        h16[(L.ks >> 1) + kscale_idx(NG, slot, warp)] = ksh;
-        h16[(L.km >> 1) + kscale_idx(NG, slot, warp)] = kmh;
-        h16[(L.vs >> 1) + vscale_idx(NG, slot, warp)] = vsh;
-        h16[(L.vm >> 1) + vscale_idx(NG, slot, warp)] = vmh;
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        if (i >= nr) break;                   // uniform
+        const float kp = __double2float_rn(acc[i]);
+        if (phys[i] < 0 || phys[i] >= num_pages) {   // uniform
+            if (c == 0) dqk_flag_error(kErrBounds);
+            continue;
+        }
+        const int slot = (L0 + t0 + i) % kPage;
+        uint16_t *h16 = reinterpret_cast<uint16_t *>(pool + ((size_t)phys[i] * hkv + j) * L.bytes);
+        uint16_t ksh, kmh, vsh, vmh;
+        const int kc = quantize_group(kp, c == 0, ksh, kmh);
+        const int vc = quantize_group(xv[i], v_ch0 != 0 && c == 0, vsh, vmh);
+        if (lane == 0) {
+            h16[(L.ks >> 1) + kscale_idx(NG, slot, warp)] = ksh;
+            h16[(L.km >> 1) + kscale_idx(NG, slot, warp)] = kmh;
+            h16[(L.vs >> 1) + vscale_idx(NG, slot, warp)] = vsh;
+            h16[(L.vm >> 1) + vscale_idx(NG, slot, warp)] = vmh;
+        }
+        if (c == 0) {
+            h16[(L.k0 >> 1) + k0_idx(slot)] = f32_to_bf16_rne(kp);
+            if (v_ch0) h16[(L.v0 >> 1) + slot] = f32_to_bf16_rne(xv[i]);
+        }
+        int off, bit;
+        kcode_pos(NG, slot, c, off, bit);
+        atomicOr(&kimg[i][off >> 2], (uint32_t)kc << bit);
+        atomicOr(&kmask[i][off >> 2], 3u << bit);
+        vcode_pos(NG, slot, c, off, bit);
+        atomicOr(&vimg[i][off >> 2], (uint32_t)vc << bit);
+        atomicOr(&vmask[i][off >> 2], 3u << bit);
     }
-    if (c == 0) {
-        h16[(L.k0 >> 1) + k0_idx(slot)] = f32_to_bf16_rne(kp);
-        if (v_ch0) h16[(L.v0 >> 1) + slot] = f32_to_bf16_rne(xv);
-    }
-    int off, bit;
-    kcode_pos(NG, slot, c, off, bit);
-    atomicOr(&kimg[off >> 2], (uint32_t)kc << bit);
-    atomicOr(&kmask[off >> 2], 3u << bit);
-    vcode_pos(NG, slot, c, off, bit);
-    atomicOr(&vimg[off >> 2], (uint32_t)vc << bit);
-    atomicOr(&vmask[off >> 2], 3u << bit);
     __syncthreads();
-    uint32_t *kw = reinterpret_cast<uint32_t *>(blk + L.kc);
-    uint32_t *vw = reinterpret_cast<uint32_t *>(blk + L.vc);
-    const uint32_t km = kmask[c], vm = vmask[c];
-    if (km == 0xffffffffu) {
-        kw[c] = kimg[c];                      // a key word holds codes of this token only
-    } else if (km) {
-        atomicAnd(&kw[c], ~km);
-        atomicOr(&kw[c], kimg[c]);
-    }
-    if (vm) {                                 // value words are shared with neighbouring tokens
-        atomicAnd(&vw[c], ~vm);
-        atomicOr(&vw[c], vimg[c]);
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        if (i >= nr) break;
+        if (phys[i] < 0 || phys[i] >= num_pages) continue;
+        uint8_t *blk = pool + ((size_t)phys[i] * hkv + j) * L.bytes;
+        uint32_t *kw = reinterpret_cast<uint32_t *>(blk + L.kc);
+        uint32_t *vw = reinterpret_cast<uint32_t *>(blk + L.vc);
+        const uint32_t km = kmask[i][c], vm = vmask[i][c];
+        if (km == 0xffffffffu) {
+            kw[c] = kimg[i][c];               // a key word holds codes of this token only
+        } else if (km) {
+            atomicAnd(&kw[c], ~km);
+            atomicOr(&kw[c], kimg[i][c]);
+        }
+        if (vm) {                             // value words are shared with neighbouring tokens
+            atomicAnd(&vw[c], ~vm);
+            atomicOr(&vw[c], vimg[i][c]);
+        }
     }
 }
 

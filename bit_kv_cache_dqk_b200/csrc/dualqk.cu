@@ -240,10 +240,11 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
                       const int *new_lens, const int *seq_before, int max_new, const int *page_table,
                       int max_pages, int early_release, cudaStream_t stream) {
     if (max_new <= kDirectMaxNew) {
-        const long long gx = (long long)batch * max_new;
+        const int groups = (max_new + kRowsPerCta - 1) / kRowsPerCta;
+        const long long gx = (long long)batch * groups;
         if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
         k_append_rows<D><<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
-            L->t_k, k, v, dtype, new_lens, seq_before, page_table, max_pages, max_new,
+            L->t_k, k, v, dtype, new_lens, seq_before, page_table, max_pages, groups,
             static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
         return launch_status();
     }

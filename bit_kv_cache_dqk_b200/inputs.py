@@ -257,6 +257,39 @@ def kv_rows(w: Workload, b: int, t0: int, t1: int, threads: int = 8):
     return k, v
 
 
+def kv_rows_device(w: Workload, seqs, t0: int, t1: int, device):
+    """Large-sweep stand-in for ``kv_rows``: keys and values of sequences
+    ``seqs``, positions [t0, t1), drawn on the device with torch's Philox
+    generator (seeded by (seed, chunk)), same distributions as ``kv_rows``
+    (N(0,1) or Student-t(3) keys times the outlier gains, N(0,1) values,
+    rotate-half RoPE, model dtype).  Returns two tensors [len(seqs)*(t1-t0)]
+    [hkv][d], sequence-major.  Not bit-identical to ``kv_rows``; used where the
+    CPU draw would take minutes and no oracle comparison is made."""
+    import torch
+    n = t1 - t0
+    g = torch.Generator(device=device)
+    g.manual_seed(int(w.seed) * 1000003 + int(t0))
+    shape = (len(seqs), n, w.hkv, w.d)
+    if w.k_dist == "t3":
+        z = torch.randn(shape, generator=g, device=device)
+        chi = torch.randn((3,) + shape, generator=g, device=device).pow(2).sum(0)
+        k = z / torch.sqrt(chi / 3.0)
+    else:
+        k = torch.randn(shape, generator=g, device=device)
+    v = torch.randn(shape, generator=g, device=device)
+    k = k * torch.from_numpy(_outlier_gain(w)).to(device)[None, None]
+    if w.rope_theta is not None:
+        half = w.d // 2
+        inv = torch.tensor(w.rope_theta ** (-np.arange(half, dtype=np.float64) * 2.0 / w.d), device=device)
+        ang = torch.arange(t0, t1, device=device, dtype=torch.float64)[:, None] * inv[None, :]
+        c = torch.cos(ang).float()[None, :, None, :]
+        sn = torch.sin(ang).float()[None, :, None, :]
+        k1, k2 = k[..., :half], k[..., half:]
+        k = torch.cat([k1 * c - k2 * sn, k2 * c + k1 * sn], dim=-1)
+    dt = torch.bfloat16 if w.kv_dtype == "bf16" else torch.float32
+    return k.to(dt).reshape(-1, w.hkv, w.d).contiguous(), v.to(dt).reshape(-1, w.hkv, w.d).contiguous()
+
+
 def queries(w: Workload, lens: np.ndarray, step: int = 0) -> np.ndarray:
     """Decode queries [batch][hq][d] (fp32 holding model-dtype values), RoPE'd
     at position L_b - 1.  ``step`` selects an independent draw."""
@@ -282,4 +315,4 @@ def ceil_div(a: int, b: int) -> int:
 
 
 __all__ = ["Workload", "CONFIGS", "PAGE", "lengths", "page_table", "transforms",
-           "kv_rows", "queries", "describe", "ceil_div"]
+           "kv_rows", "kv_rows_device", "queries", "describe", "ceil_div"]
