@@ -9,9 +9,8 @@
 // whatever the length mix.  A producer warp brings whole units in with 1-D bulk
 // async copies (one copy = 16 tokens x up to 8 kv heads, contiguous) into a
 // ring of shared-memory stages of 16 (page, kv head) blocks guarded by
-// mbarriers.  Consumer warps each own one kv head and take two pages of it per
-// stage, processed together (two independent instruction streams); a stage
-// holds two pages per consumer warp.
+// mbarriers.  Consumer warps each own one kv head and take two or four pages
+// of it per stage, processed together (independent instruction streams).
 //
 // Per consumer warp and page (16 tokens x G query heads), with
 // qs = q' * log2(e)/sqrt(d) on the kept channels:
@@ -38,12 +37,14 @@
 
 namespace dqk {
 
-// CTA shape of k_attend: consumer warps each take two pages of one kv head per
-// stage, plus one producer warp.  16 consumer warps (two per kv head of a
-// chunk of 8) where the per-warp state fits 96 registers; 8 for G = 8, whose
-// two query-head tiles double that state.
-__host__ __device__ constexpr int attend_warps(int G) { return G > 4 ? 8 : 16; }
-__host__ __device__ constexpr int attend_stage_blocks(int G) { return 2 * attend_warps(G); }
+// CTA shape of k_attend: 8 consumer warps, each owning one kv head of a chunk
+// of 8 and taking attend_pages_per_warp pages of it per stage (processed as
+// independent instruction streams), plus one producer warp.  Four pages per
+// warp where the per-warp state allows (G <= 4), two for G = 8, whose two
+// query-head tiles double that state.
+__host__ __device__ constexpr int attend_warps(int G) { return 8; }
+__host__ __device__ constexpr int attend_pages_per_warp(int G) { return G > 4 ? 2 : 4; }
+__host__ __device__ constexpr int attend_stage_blocks(int G) { return attend_pages_per_warp(G) * attend_warps(G); }
 __host__ __device__ constexpr int attend_threads(int G) { return 32 * (attend_warps(G) + 1); }
 constexpr int kMaxStages = 8;                               // ring depth cap
 constexpr uint64_t kWaitLimitNs = 1000000000ull;            // 1 s: a stuck pipeline reports DQK_ERR_TIMEOUT
@@ -489,6 +490,8 @@ template <int D, int G, bool VCH0>
 __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendParams p) {
     using T = AttendTile<D, G>;
     constexpr int kConsumerWarps = attend_warps(G), kStageBlocks = attend_stage_blocks(G);
+    constexpr int BPW = attend_pages_per_warp(G);
+    static_assert(BPW == 2 || BPW == 4, "pages per warp");
     constexpr int NG = T::NG, NT = T::NT, NM = T::NM;
     extern __shared__ __align__(128) unsigned char attend_smem[];
     const int S = p.stages;
@@ -528,7 +531,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     }
 
     // ---------------------------------------------------------------- consumers
-    // warp: kv head jl of the chunk, page pair pi of each stage (pages 2*pi, 2*pi + 1)
+    // warp: kv head jl of the chunk, page group pi of each stage (slots BPW*pi ..)
     const int jl = warp % p.hc, pi = warp / p.hc;
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
@@ -642,9 +645,10 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     bool ok = true;
     int stage = 0;
     uint32_t phase = 0;
-    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((2 * pi * p.hc + jl) * p.bb);
-    const uint32_t pair_gap = (uint32_t)(p.hc * p.bb);
-    const uint32_t valid_addr = smem_addr(valid) + 2 * pi;
+    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((BPW * pi * p.hc + jl) * p.bb);
+    const uint32_t page_gap = (uint32_t)(p.hc * p.bb);
+    const uint32_t valid_addr = smem_addr(valid) + BPW * pi;
+    constexpr uint32_t kAllValid = BPW == 4 ? 0x01010101u : 0x0101u;
     for (int it = 0; it < iters; ++it) {
         if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
             if (lane == 0) {
@@ -654,27 +658,29 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
             ok = false;
             break;
         }
-        const int ua = u0 + it * pps + 2 * pi;
+        const int ua = u0 + it * pps + BPW * pi;
         if (ua < u1) {
             const uint32_t sa = blk_a + (uint32_t)stage * stage_bytes;
-            const int ub = ua + 1;
-            const uint32_t vv = ld_s16(valid_addr + stage * kStageBlocks);   // flags of slots 2pi, 2pi+1
+            const int ul = ua + BPW - 1;
+            // flags of the warp's page slots (one byte each)
+            const uint32_t vv = BPW == 4 ? ld_s32(valid_addr + stage * kStageBlocks)
+                                         : ld_s16(valid_addr + stage * kStageBlocks);
             if (ua >= run_end) switch_run(ua);
-            if (ub < run_end && ub < u1 && ub != partial_u && vv == 0x0101u) {
-                const uint32_t sbb[2] = {sa, sa + pair_gap};
-                consume<D, G, VCH0, 2, false>(sbb, kPage, st, lane, lo);
+            if (ul < run_end && ul < u1 && !(partial_u >= ua && partial_u <= ul) && vv == kAllValid) {
+                uint32_t sbb[BPW];
+#pragma unroll
+                for (int q = 0; q < BPW; ++q) sbb[q] = sa + q * page_gap;
+                consume<D, G, VCH0, BPW, false>(sbb, kPage, st, lane, lo);
             } else {
-                const uint32_t s1[1] = {sa};
-                if (vv & 0xffu) {
-                    if (ua == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
-                    else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);
-                }
-                if (ub < u1) {
-                    if (ub >= run_end) switch_run(ub);
-                    const uint32_t s2[1] = {sa + pair_gap};
-                    if (vv >> 8) {
-                        if (ub == partial_u) consume<D, G, VCH0, 1, true>(s2, nv_last, st, lane, lo);
-                        else consume<D, G, VCH0, 1, false>(s2, kPage, st, lane, lo);
+#pragma unroll
+                for (int q = 0; q < BPW; ++q) {
+                    const int uq = ua + q;
+                    if (uq >= u1) break;
+                    if (uq >= run_end) switch_run(uq);
+                    if ((vv >> (8 * q)) & 1u) {
+                        const uint32_t s1[1] = {sa + q * page_gap};
+                        if (uq == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
+                        else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);
                     }
                 }
             }
