@@ -112,6 +112,41 @@ __host__ __device__ __forceinline__ long long cta_of_unit(long long u, long long
     return ((u + 1) * C - 1) / U;
 }
 
+// The CTA's unit range [u0, u1) out of U units, the run r holding u0 and the
+// unit ur where that run starts (r = R past the last unit).  One warp, one
+// pass over the run lengths when there are at most 32 runs.
+struct CtaUnits {
+    int U, u0, u1, r, ur;
+};
+
+__device__ __forceinline__ CtaUnits cta_units(const int *seq_lens, int nchunks, int R, int cta, int num_ctas,
+                                              int lane) {
+    CtaUnits cu;
+    if (R <= 32) {
+        const int np = lane < R ? run_pages(seq_lens, nchunks, lane) : 0;
+        int incl = np;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        cu.U = __shfl_sync(0xffffffffu, incl, 31);
+        cu.u0 = (int)((long long)cta * cu.U / num_ctas);
+        cu.u1 = (int)(((long long)cta + 1) * cu.U / num_ctas);
+        const unsigned m = __ballot_sync(0xffffffffu, np > 0 && incl - np <= cu.u0 && cu.u0 < incl);
+        cu.r = m ? __ffs(m) - 1 : R;
+        cu.ur = m ? __shfl_sync(0xffffffffu, incl - np, cu.r) : cu.U;
+    } else {
+        cu.U = (int)warp_total_units(seq_lens, nchunks, R, lane);
+        cu.u0 = (int)((long long)cta * cu.U / num_ctas);
+        cu.u1 = (int)(((long long)cta + 1) * cu.U / num_ctas);
+        long long urll;
+        warp_locate(seq_lens, nchunks, R, cu.u0, lane, cu.r, urll);
+        cu.ur = (int)urll;
+    }
+    return cu;
+}
+
 // Partial record of (slot = CTA + run, warp pair index pi, kv head jl, query head hh).
 __host__ __device__ __forceinline__ size_t record_index(int slot, int pi, int jl, int hh, int pw, int hc, int G) {
     return (((size_t)slot * pw + pi) * hc + jl) * G + hh;
@@ -380,13 +415,11 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
 // Every (run, page slot, kv head) record a consumer warp could own starts
 // empty (m = -inf, l = 0): a run shorter than the page slots of a stage
 // leaves some warps without a page of it.
-__device__ __forceinline__ void init_records(const AttendParams &p, int u0, int u1, int slot_base, int pi, int jl,
-                                             int G, int D, int lane) {
+__device__ __forceinline__ void init_records(const AttendParams &p, const CtaUnits &cu, int slot_base, int pi,
+                                             int jl, int G, int D, int lane) {
     const int R = p.batch * p.nchunks;
-    int r;
-    long long urll;
-    warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
-    int ur = (int)urll;
+    const int u1 = cu.u1;
+    int r = cu.r, ur = cu.ur;
     int np = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     while (r < R && ur < u1) {
         if (np > 0 && lane < G) {
@@ -406,16 +439,14 @@ __device__ __forceinline__ void init_records(const AttendParams &p, int u0, int 
 // flight.  Waits are bounded; a stuck pipeline sets the abort flag.
 __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned char *stage_mem, uint64_t *full,
                                                 uint64_t *empty, unsigned char *valid, volatile int *abort_flag,
-                                                int S, uint32_t stage_bytes, int kStageBlocks, int u0, int u1,
+                                                int S, uint32_t stage_bytes, int kStageBlocks, const CtaUnits &cu,
                                                 int iters, int lane) {
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
+    const int u0 = cu.u0, u1 = cu.u1;
     grid_dependents_launch();   // the combine kernel may start its prologue
     if (iters == 0) return;
-    int r;
-    long long urll;
-    warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
-    int ur = (int)urll;
+    int r = cu.r, ur = cu.ur;
     int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     const uint32_t copy_bytes = (uint32_t)(p.hc * p.bb);
     // pool byte offset of unit ubase + lane (or -1); moves the cursor to unit ubase + 32
@@ -508,6 +539,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
 
+    __shared__ CtaUnits sh_cu;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
@@ -516,17 +548,18 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == 0) {
+        const CtaUnits c = cta_units(p.seq_lens, p.nchunks, R, blockIdx.x, p.num_ctas, lane);
+        if (lane == 0) sh_cu = c;
+    }
     __syncthreads();
-
-    const int U = (int)warp_total_units(p.seq_lens, p.nchunks, R, lane);
-    const int u0 = (int)((long long)blockIdx.x * U / p.num_ctas);
-    const int u1 = (int)(((long long)blockIdx.x + 1) * U / p.num_ctas);
+    const CtaUnits cu = sh_cu;
+    const int u0 = cu.u0, u1 = cu.u1;
     const int nunits = u1 - u0;
     const int iters = (nunits + pps - 1) / pps;
 
     if (warp == kConsumerWarps) {
-        attend_producer(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kStageBlocks, u0, u1, iters,
-                        lane);
+        attend_producer(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kStageBlocks, cu, iters, lane);
         return;
     }
 
@@ -536,17 +569,12 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
 
-    if (nunits > 0) init_records(p, u0, u1, slot_base, pi, jl, G, D, lane);
+    if (nunits > 0) init_records(p, cu, slot_base, pi, jl, G, D, lane);
     if (iters == 0) return;
     grid_dependency_wait();     // query fragments come from k_qprep
 
-    int r, ur, npr;
-    {
-        long long urll;
-        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
-        ur = (int)urll;
-        npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-    }
+    int r = cu.r, ur = cu.ur;
+    int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     int cur_run = -1, run_end = -1, partial_u = -1, nv_last = kPage;
 
     WarpState<D, G> st;

@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
+    __shared__ CtaUnits sh_cu;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
@@ -232,13 +233,16 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == 0) {
+        const CtaUnits c = cta_units(p.seq_lens, p.nchunks, R, blockIdx.x, p.num_ctas, lane);
+        if (lane == 0) sh_cu = c;
+    }
     __syncthreads();
-    const int U = (int)warp_total_units(p.seq_lens, p.nchunks, R, lane);
-    const int u0 = (int)((long long)blockIdx.x * U / p.num_ctas);
-    const int u1 = (int)(((long long)blockIdx.x + 1) * U / p.num_ctas);
+    const CtaUnits cu = sh_cu;
+    const int u0 = cu.u0, u1 = cu.u1;
     const int iters = (u1 - u0 + pps - 1) / pps;
     if (warp == kB16Warps) {
-        attend_producer(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kB16StageBlocks, u0, u1, iters,
+        attend_producer(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kB16StageBlocks, cu, iters,
                         lane);
         return;
     }
@@ -246,17 +250,12 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     const int jl = warp % p.hc, pi = warp / p.hc;
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
-    if (u1 > u0) init_records(p, u0, u1, slot_base, pi, jl, G, D, lane);
+    if (u1 > u0) init_records(p, cu, slot_base, pi, jl, G, D, lane);
     if (iters == 0) return;
     grid_dependency_wait();     // query fragments come from k_qprep_b16
 
-    int r, ur, npr;
-    {
-        long long urll;
-        warp_locate(p.seq_lens, p.nchunks, R, u0, lane, r, urll);
-        ur = (int)urll;
-        npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-    }
+    int r = cu.r, ur = cu.ur;
+    int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     int cur_run = -1, run_end = -1, partial_u = -1, nv_last = kPage;
     St st;
     auto start_run = [&](int rr) {
