@@ -192,21 +192,24 @@ struct LaneOffsets {
     int srcA;          // lane holding p of (token 2tig, head gid/2); +4: token 2tig+1
     uint32_t sq;       // shared address of this lane's QK B fragments: [NT][NG][32 lanes] uint2
     uint32_t sk;       // shared address of this thread's head constants: [NT][NG][4 heads] float4
-    uint32_t ones_lane, vmin_mask, kmin_mask;
+    uint32_t ones_lane, vmin_mask;
 };
 
-// NB (page, kv head) blocks at shared addresses sb[]: 16 tokens x G query heads
-// each, same run.  MASKED (NB == 1 only): only the first nv tokens are valid.
-template <int D, int G, bool VCH0, int NB, bool MASKED>
-__device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpState<D, G> &st, int lane,
-                                        const LaneOffsets &o) {
+// A page is consumed in three steps: qk_scores (scores of its 16 tokens for
+// the warp's G query heads), max_update (the lazy running max) and pv_accum
+// (softmax weights and the value accumulation).  NB (page, kv head) blocks at
+// shared addresses sb[], same run; MASKED (NB == 1 only): only the first nv
+// tokens are valid.
+template <int D, int G, int NB, bool MASKED>
+__device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, const WarpState<D, G> &st, int lane,
+                                          const LaneOffsets &o, float (&s0)[NB][AttendTile<D, G>::NT],
+                                          float (&s1)[NB][AttendTile<D, G>::NT]) {
     using T = AttendTile<D, G>;
     constexpr int NG = T::NG, NT = T::NT;
     constexpr Layout Ly = make_layout(D, 0);   // section offsets do not depend on v_ch0 (V0 is last)
     static_assert(NB == 1 || !MASKED, "masked blocks are processed alone");
-    const int gid = lane >> 2, tig = lane & 3;
+    const int gid = lane >> 2;
 
-    // ---------------------------------------------------------------- keys
     uint32_t kw[NB][NG], ks0[NB][NG / 2], ks1[NB][NG / 2], km0[NB], km1[NB];
     float k0a[NB], k0b[NB];
 #pragma unroll
@@ -225,8 +228,10 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
             ks1[b][0] = ld_s32(a + Ly.ks + 32);
         }
         const uint32_t akm = sb[b] + o.kmin;
-        km0[b] = ld_s32(akm + Ly.km) & o.kmin_mask;
-        km1[b] = ld_s32(akm + Ly.km + 16 * NG) & o.kmin_mask;
+        // lanes past the groups read this token's other mins; the min-term B
+        // operand is zero in those rows
+        km0[b] = ld_s32(akm + Ly.km);
+        km1[b] = ld_s32(akm + Ly.km + 16 * NG);
         const uint32_t k0w = ld_s32(sb[b] + o.gid4 + Ly.k0);
         k0a[b] = __uint_as_float(k0w << 16);
         k0b[b] = __uint_as_float(k0w & 0xffff0000u);
@@ -261,9 +266,9 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
                 A0 = kw[b][0] & msk; A1 = kw[b][1] & msk;
                 A2 = (kw[b][0] >> 4) & msk; A3 = (kw[b][1] >> 4) & msk;
             }
-            // key scales * 2^-112 (integer ops only)
-            const float sa = (g & 1) ? f16hi_scaled(ks0[b][g >> 1]) : f16lo_scaled(ks0[b][g >> 1]);
-            const float sbv = (g & 1) ? f16hi_scaled(ks1[b][g >> 1]) : f16lo_scaled(ks1[b][g >> 1]);
+            // key scales of tokens gid and gid + 8
+            const float sa = (g & 1) ? f16hi_to_f32(ks0[b][g >> 1]) : f16lo_to_f32(ks0[b][g >> 1]);
+            const float sbv = (g & 1) ? f16hi_to_f32(ks1[b][g >> 1]) : f16lo_to_f32(ks1[b][g >> 1]);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 int dg[4];
@@ -277,22 +282,31 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
             }
         }
     }
-    float s0[NB][NT], s1[NB][NT];
-    bool grow = false;
 #pragma unroll
     for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            s0[b][nt] = fmaf(a0[b][nt], kTwoPow112, fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0] + cmin[b][nt][1]));
-            s1[b][nt] = fmaf(a1[b][nt], kTwoPow112, fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2] + cmin[b][nt][3]));
+            s0[b][nt] = a0[b][nt] + fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0] + cmin[b][nt][1]);
+            s1[b][nt] = a1[b][nt] + fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2] + cmin[b][nt][3]);
             if constexpr (MASKED) {
                 if (gid >= nv) s0[b][nt] = -INFINITY;
                 if (gid + 8 >= nv) s1[b][nt] = -INFINITY;
             }
-            grow |= (s0[b][nt] > st.m_run[nt]) | (s1[b][nt] > st.m_run[nt]);
         }
-    // The running max only moves when a score exceeds it (rare after the first
-    // pages): then take the exact max over these pages and rescale.
+}
+
+// The running max only moves when a score exceeds it (rare after the first
+// pages): then take the exact max over these pages and rescale.
+template <int D, int G, int NB>
+__device__ __forceinline__ void max_update(WarpState<D, G> &st, const float (&s0)[NB][AttendTile<D, G>::NT],
+                                           const float (&s1)[NB][AttendTile<D, G>::NT]) {
+    using T = AttendTile<D, G>;
+    constexpr int NT = T::NT;
+    bool grow = false;
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) grow |= (s0[b][nt] > st.m_run[nt]) | (s1[b][nt] > st.m_run[nt]);
     if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -314,8 +328,16 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
             st.m_run[nt] = mnew;
         }
     }
+}
 
-    // ---------------------------------------------------------------- values
+template <int D, int G, bool VCH0, int NB, bool MASKED>
+__device__ __forceinline__ void pv_accum(const uint32_t (&sb)[NB], int nv, WarpState<D, G> &st, int lane,
+                                         const LaneOffsets &o, const float (&s0)[NB][AttendTile<D, G>::NT],
+                                         const float (&s1)[NB][AttendTile<D, G>::NT]) {
+    using T = AttendTile<D, G>;
+    constexpr int NG = T::NG, NT = T::NT;
+    constexpr Layout Ly = make_layout(D, 0);
+    const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
         uint32_t vw[NG], vsa[NG], vsb[NG];   // vsa/vsb: scale pairs of tokens (2tig, 2tig+1) and (+8, +9)
@@ -410,6 +432,16 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
             }
         }
     }
+}
+
+template <int D, int G, bool VCH0, int NB, bool MASKED>
+__device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpState<D, G> &st, int lane,
+                                        const LaneOffsets &o) {
+    constexpr int NT = AttendTile<D, G>::NT;
+    float s0[NB][NT], s1[NB][NT];
+    qk_scores<D, G, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
+    max_update<D, G, NB>(st, s0, s1);
+    pv_accum<D, G, VCH0, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
 }
 
 // Every (run, page slot, kv head) record a consumer warp could own starts
@@ -581,7 +613,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     LaneOffsets lo;
     lo.lane16 = lane * 16;
     lo.gid8 = gid * 8;
-    lo.kmin = gid * 2 * NG + (tig & (NG / 2 - 1)) * 4;   // in range for every lane; kmin_mask zeroes the rest
+    lo.kmin = gid * 2 * NG + (tig & (NG / 2 - 1)) * 4;   // in range for every lane (B rows past NG are 0)
     lo.gid4 = gid * 4;
     lo.tig16 = tig * 16;
     lo.vmin = (tig * NG + (gid < NG ? gid : 0)) * 4;
@@ -593,7 +625,6 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     }
     lo.ones_lane = gid == NG ? 0x3C003C00u : 0u;
     lo.vmin_mask = gid < NG ? 0xffffffffu : 0u;
-    lo.kmin_mask = tig < NG / 2 ? 0xffffffffu : 0u;
 
     auto start_run = [&](int rr) {
         const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;

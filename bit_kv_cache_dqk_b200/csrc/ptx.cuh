@@ -242,6 +242,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
 __device__ __forceinline__ float f16lo_scaled(uint32_t w) { return __uint_as_float((w << 13) & 0x0fffe000u); }
 __device__ __forceinline__ float f16hi_scaled(uint32_t w) { return __uint_as_float((w >> 3) & 0x0fffe000u); }
 constexpr float kTwoPow112 = 0x1p112f;
+// fp16 halves of a word as fp32 (exact; one conversion each)
+__device__ __forceinline__ float f16lo_to_f32(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
+__device__ __forceinline__ float f16hi_to_f32(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
 // Shared-memory loads by 32-bit shared-window address.  volatile keeps them
 // after the mbarrier wait that makes the stage's bytes visible.
