@@ -174,6 +174,9 @@ __device__ __forceinline__ float vfield_scale(int m) {
 template <int D, int G>
 struct WarpState {
     using T = AttendTile<D, G>;
+    static constexpr bool kRegFrags = T::NT == 1;   // score fragments in registers (else per-warp shared memory)
+    uint2 qb[kRegFrags ? T::NG : 1];                // score B fragments of group g
+    float4 kp[kRegFrags ? T::NG : 1];               // kappa, kappa/256, -M kappa, -M kappa/256 of group g
     uint32_t qmin[T::NT];          // min-term B fragment
     float q0v[T::NT];              // scaled q'_0 of this thread's head
     float m_run[T::NT];            // running max (log2 units) of this thread's head
@@ -250,12 +253,17 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
         const uint32_t msk = 0x03030303u << (2 * g);   // group g's field in every byte: code * 4^g
         uint2 qb[NT];
         float4 kp[NT];
+        if constexpr (WarpState<D, G>::kRegFrags) {
+            qb[0] = st.qb[g];
+            kp[0] = st.kp[g];
+        } else {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            qb[nt] = ld_s64(o.sq + (nt * NG + g) * 256);
-            const uint4 kpu = ld_s128(o.sk + (nt * NG + g) * 64);
-            kp[nt] = make_float4(__uint_as_float(kpu.x), __uint_as_float(kpu.y), __uint_as_float(kpu.z),
-                                 __uint_as_float(kpu.w));
+            for (int nt = 0; nt < NT; ++nt) {
+                qb[nt] = ld_s64(o.sq + (nt * NG + g) * 256);
+                const uint4 kpu = ld_s128(o.sk + (nt * NG + g) * 64);
+                kp[nt] = make_float4(__uint_as_float(kpu.x), __uint_as_float(kpu.y), __uint_as_float(kpu.z),
+                                     __uint_as_float(kpu.w));
+            }
         }
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
@@ -635,13 +643,17 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
                 const uint2 qb = p.qf[((bj * NT + nt) * NG + g) * 32 + lane];
-                st_s64(lo.sq + (nt * NG + g) * 256, qb);
-                if (gid == 0) {
-                    const float kappa = p.qk[((bj * NT + nt) * NG + g) * 4 + tig];
-                    st_s128(lo.sk + (nt * NG + g) * 64,
-                            make_uint4(__float_as_uint(kappa), __float_as_uint(kappa * (1.0f / 256.0f)),
-                                       __float_as_uint(-kMagicF * kappa),
-                                       __float_as_uint(-kMagicF * kappa * (1.0f / 256.0f))));
+                const float kappa = p.qk[((bj * NT + nt) * NG + g) * 4 + tig];
+                const float4 kp = make_float4(kappa, kappa * (1.0f / 256.0f), -kMagicF * kappa,
+                                              -kMagicF * kappa * (1.0f / 256.0f));
+                if constexpr (WarpState<D, G>::kRegFrags) {
+                    st.qb[g] = qb;
+                    st.kp[g] = kp;
+                } else {
+                    st_s64(lo.sq + (nt * NG + g) * 256, qb);
+                    if (gid == 0)
+                        st_s128(lo.sk + (nt * NG + g) * 64, make_uint4(__float_as_uint(kp.x), __float_as_uint(kp.y),
+                                                                       __float_as_uint(kp.z), __float_as_uint(kp.w)));
                 }
             }
             __syncwarp();
@@ -700,6 +712,9 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
         partial_u = (Lb & (kPage - 1)) ? run_end - 1 : -1;
         nv_last = Lb - (npr - 1) * kPage;
     };
+
+    // the first run's query fragments load while the first pages are in flight
+    switch_run(u0 + BPW * pi < u1 ? u0 + BPW * pi : u0);
 
     bool ok = true;
     int stage = 0;
