@@ -125,6 +125,19 @@ dqk_status check_decode(const DecodeArgs &a, DecodePlan &P) {
     return DQK_OK;
 }
 
+// Every kernel of the path prefers the largest shared-memory carveout, so that
+// consecutive kernels do not make the SMs switch their L1 / shared split.
+// Attributes are per function; setting one twice is harmless.
+template <typename Kern>
+void prefer_max_shared(Kern kernel) {
+    static bool done = false;
+    if (!done) {
+        (void)cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                   (int)cudaSharedmemCarveoutMaxShared);
+        done = true;
+    }
+}
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream finishes; it orders itself with
 // griddepcontrol.wait before touching that kernel's outputs.
@@ -147,6 +160,7 @@ dqk_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 template <int D>
 dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
     const size_t smem = qprep_smem_bytes(D, P.G);
+    prefer_max_shared(k_qprep<D>);
     if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
@@ -160,6 +174,7 @@ dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
 
 template <int D, int G, bool VCH0>
 dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
+    prefer_max_shared(k_attend<D, G, VCH0>);
     if (cudaFuncSetAttribute(k_attend<D, G, VCH0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
         cudaSuccess)
         return DQK_ERR_CUDA;
@@ -207,6 +222,7 @@ dqk_status run_attend(const DecodeArgs &a, const DecodePlan &P) {
 template <int D>
 dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
     char *ws = static_cast<char *>(a.ws);
+    prefer_max_shared(k_combine<D>);
     return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(kCombineThreads), 0, a.stream, a.seq_lens,
                       a.batch,
                       a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pw, P.nchunks, P.num_ctas,
@@ -240,6 +256,7 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
                       const int *new_lens, const int *seq_before, int max_new, const int *page_table,
                       int max_pages, int early_release, cudaStream_t stream) {
     if (max_new <= kDirectMaxNew) {
+        prefer_max_shared(k_append_rows<D>);
         const int groups = (max_new + kRowsPerCta - 1) / kRowsPerCta;
         const long long gx = (long long)batch * groups;
         if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
