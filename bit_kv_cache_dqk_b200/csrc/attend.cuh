@@ -562,7 +562,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     using T = AttendTile<D, G>;
     constexpr int kConsumerWarps = attend_warps(G), kStageBlocks = attend_stage_blocks(G);
     constexpr int BPW = attend_pages_per_warp(G);
-    static_assert(BPW == 2 || BPW == 4, "pages per warp");
+    static_assert(BPW >= 2 && BPW <= 8, "pages per warp");
     constexpr int NG = T::NG, NT = T::NT, NM = T::NM;
     extern __shared__ __align__(128) unsigned char attend_smem[];
     const int S = p.stages;
@@ -722,7 +722,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((BPW * pi * p.hc + jl) * p.bb);
     const uint32_t page_gap = (uint32_t)(p.hc * p.bb);
     const uint32_t valid_addr = smem_addr(valid) + BPW * pi;
-    constexpr uint32_t kAllValid = BPW == 4 ? 0x01010101u : 0x0101u;
+    constexpr uint32_t kAllValid = (1u << BPW) - 1u;
     for (int it = 0; it < iters; ++it) {
         if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
             if (lane == 0) {
@@ -736,9 +736,19 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
         if (ua < u1) {
             const uint32_t sa = blk_a + (uint32_t)stage * stage_bytes;
             const int ul = ua + BPW - 1;
-            // flags of the warp's page slots (one byte each)
-            const uint32_t vv = BPW == 4 ? ld_s32(valid_addr + stage * kStageBlocks)
-                                         : ld_s16(valid_addr + stage * kStageBlocks);
+            // flags of the warp's page slots (one byte each), as a bit mask
+            const uint32_t va = valid_addr + stage * kStageBlocks;
+            uint32_t vv = 0;
+            if constexpr (BPW == 4) {
+                const uint32_t w = ld_s32(va);
+                vv = (w & 1u) | ((w >> 7) & 2u) | ((w >> 14) & 4u) | ((w >> 21) & 8u);
+            } else if constexpr (BPW == 2) {
+                const uint32_t w = ld_s16(va);
+                vv = (w & 1u) | ((w >> 7) & 2u);
+            } else {
+#pragma unroll
+                for (int q = 0; q < BPW; ++q) vv |= ld_s8(va + q) << q;
+            }
             if (ua >= run_end) switch_run(ua);
             if (ul < run_end && ul < u1 && !(partial_u >= ua && partial_u <= ul) && vv == kAllValid) {
                 uint32_t sbb[BPW];
@@ -751,7 +761,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
                     const int uq = ua + q;
                     if (uq >= u1) break;
                     if (uq >= run_end) switch_run(uq);
-                    if ((vv >> (8 * q)) & 1u) {
+                    if ((vv >> q) & 1u) {
                         const uint32_t s1[1] = {sa + q * page_gap};
                         if (uq == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
                         else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);

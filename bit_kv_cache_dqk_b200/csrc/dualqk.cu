@@ -75,8 +75,9 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.bb = make_layout(P.d, L->v_ch0_protect).bytes;
     // shared memory: ring stages | mbarriers | valid flags | abort flag | per-warp query fragments
     const size_t stage_bytes = (size_t)stage_blocks * P.bb;
+    // (score fragments live in shared memory only for two query-head tiles)
     const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * stage_blocks + 16 +
-                         (size_t)warps * P.NT * P.NG * (32 * 8 + 4 * 16);
+                         (P.NT > 1 ? (size_t)warps * P.NT * P.NG * (32 * 8 + 4 * 16) : 0);
     const size_t budget = 227 * 1024;
     P.stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / stage_bytes);
     if (P.stages < 2) return false;
