@@ -155,7 +155,8 @@ class Layer:
         self.lens = I.lengths(w)
         self.table, self.num_pages = I.page_table(w, self.lens)
         self.max_pages = self.table.shape[1]
-        tk, tq, _, _ = I.transforms(w)
+        from bit_kv_cache_dqk_b200 import calibrate as Cb
+        tk, tq, _, _ = Cb.layer_transforms(w)
         self.t_k = torch.from_numpy(tk).to(dev)
         self.t_q = torch.from_numpy(tq).to(dev)
         probe = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, 0, 1)
@@ -363,7 +364,8 @@ class OracleSample:
         from bit_kv_cache_dqk_b200 import inputs as I
         from oracle import oracle as O
         self.O, self.w, self.ctx = O, w, ctx
-        tk, tq, _, _ = I.transforms(w)
+        from bit_kv_cache_dqk_b200 import calibrate as Cb
+        tk, tq, _, _ = Cb.layer_transforms(w)
         self.tq = tq
         k, v = I.kv_rows(w, 0, 0, ctx)
         with ThreadPoolExecutor(min(w.hkv, os.cpu_count() or 1)) as ex:

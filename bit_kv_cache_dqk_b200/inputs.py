@@ -42,6 +42,7 @@ CHUNK = 1024       # tokens per independently seeded K/V draw
 
 # stream ids (second word of every seed sequence)
 _S_KV, _S_Q, _S_T, _S_OUTL, _S_LEN, _S_PERM = 11, 12, 13, 14, 15, 16
+_S_QBASIS, _S_CAL = 17, 18
 
 
 @dataclasses.dataclass(frozen=True)
@@ -56,7 +57,9 @@ class Workload:
     kv_dtype: str = "bf16"       # "bf16" or "f32"
     k_dist: str = "normal"       # "normal" or "t3"
     outliers: str = "random4"    # "fixed_3_17", "random4" or "none"
-    transform: str = "whiten"    # "whiten" (Cov^-1/4) or "noise" (I + 0.1 N)
+    transform: str = "whiten"    # "whiten" (Cov^-1/4), "noise" (I + 0.1 N) or "calibrated" (built by the
+                                 # caller from calibration_rows; see bit_kv_cache_dqk_b200.calibrate)
+    q_dist: str = "normal"       # "normal" or "lowrank" (queries near a rank-8 subspace per kv head)
     rope_theta: float | None = 5e5
     pct: int = 40
     page_order: str = "random"   # "sequential", "random" or "shared"
@@ -83,6 +86,9 @@ CONFIGS = {
     "qwen": Workload("qwen", batch=16, hq=32, hkv=8, d=128, ctx=None, seed=4,
                      k_dist="t3", outliers="none", rope_theta=1e6, append_new=64),
     "sweep": Workload("sweep", batch=16, hq=32, hkv=8, d=128, ctx=131072, seed=5),
+    # the llama layer with structured queries and calibrated transforms (next-step row f1)
+    "llama_cal": Workload("llama_cal", batch=8, hq=32, hkv=8, d=128, ctx=32768, seed=6,
+                          transform="calibrated", q_dist="lowrank", page_order="random"),
 }
 
 
@@ -158,6 +164,8 @@ def transforms(w: Workload):
     ``noise``: T_K = I + 0.1 N(0,1), redrawn with seed+1 until cond < 10,
     T_Q = inv(T_K)^T.
     """
+    if w.transform == "calibrated":
+        raise ValueError("calibrated transforms are built from calibration_rows by the calibrate module")
     t_k = np.empty((w.hkv, w.d, w.d))
     t_q = np.empty((w.hkv, w.d, w.d))
     for j in range(w.hkv):
@@ -290,11 +298,58 @@ def kv_rows_device(w: Workload, seqs, t0: int, t1: int, device):
     return k.to(dt).reshape(-1, w.hkv, w.d).contiguous(), v.to(dt).reshape(-1, w.hkv, w.d).contiguous()
 
 
+_QRANK = 8
+_QSCALES = np.array([4.0, 3.0, 2.5, 2.0, 1.6, 1.3, 1.0, 0.8])
+
+
+def _query_basis(w: Workload) -> np.ndarray:
+    """Per kv head, an orthonormal d x 8 basis the ``lowrank`` queries live near."""
+    rng = np.random.default_rng([w.seed, _S_QBASIS])
+    out = np.empty((w.hkv, w.d, _QRANK))
+    for j in range(w.hkv):
+        qm, _ = np.linalg.qr(rng.standard_normal((w.d, _QRANK)))
+        out[j] = qm
+    return out
+
+
+def _raw_queries(w: Workload, rng, rows: int) -> np.ndarray:
+    """[rows][hq][d] pre-RoPE queries of the workload's distribution."""
+    if w.q_dist == "lowrank":
+        basis = _query_basis(w)
+        z = rng.standard_normal((rows, w.hq, _QRANK)) * _QSCALES[None, None, :]
+        q = np.einsum("jdr,nhr->nhd", basis[np.arange(w.hq) // w.group], z)
+        q += 0.25 * rng.standard_normal((rows, w.hq, w.d))
+        return q.astype(np.float32)
+    return rng.standard_normal((rows, w.hq, w.d)).astype(np.float32)
+
+
+def calibration_rows(w: Workload, n_keys: int = 4096, n_queries: int = 1024):
+    """Calibration activations: keys [n_keys][hkv][d] and queries
+    [n_queries][hq][d] of the workload's distributions, RoPE'd at seeded random
+    positions within the context, in model dtype (fp32 arrays).  Drawn from
+    their own streams, disjoint from the decoded rows."""
+    rng = np.random.default_rng([w.seed, _S_CAL])
+    ctx = w.ctx if w.ctx is not None else w.ctx_hi
+    gain = _outlier_gain(w)
+    if w.k_dist == "t3":
+        k = rng.standard_t(3, size=(n_keys, w.hkv, w.d)).astype(np.float32)
+    else:
+        k = rng.standard_normal((n_keys, w.hkv, w.d)).astype(np.float32)
+    k *= gain[None]
+    q = _raw_queries(w, rng, n_queries)
+    if w.rope_theta is not None:
+        pk = rng.integers(0, ctx, size=n_keys)
+        pq = rng.integers(0, ctx, size=n_queries)
+        k = np.concatenate([_rope(k[i:i + 1], pk[i:i + 1], w.rope_theta) for i in range(n_keys)])
+        q = np.concatenate([_rope(q[i:i + 1], pq[i:i + 1], w.rope_theta) for i in range(n_queries)])
+    return _to_model_dtype(k, w.kv_dtype), _to_model_dtype(q, w.kv_dtype)
+
+
 def queries(w: Workload, lens: np.ndarray, step: int = 0) -> np.ndarray:
     """Decode queries [batch][hq][d] (fp32 holding model-dtype values), RoPE'd
     at position L_b - 1.  ``step`` selects an independent draw."""
     rng = np.random.default_rng([w.seed, _S_Q, step])
-    q = rng.standard_normal((w.batch, w.hq, w.d)).astype(np.float32)
+    q = _raw_queries(w, rng, w.batch)
     if w.rope_theta is not None:
         for b in range(w.batch):
             q[b] = _rope(q[b][None], np.array([int(lens[b]) - 1]), w.rope_theta)[0]
@@ -315,4 +370,4 @@ def ceil_div(a: int, b: int) -> int:
 
 
 __all__ = ["Workload", "CONFIGS", "PAGE", "lengths", "page_table", "transforms",
-           "kv_rows", "kv_rows_device", "queries", "describe", "ceil_div"]
+           "kv_rows", "kv_rows_device", "queries", "calibration_rows", "describe", "ceil_div"]

@@ -435,3 +435,142 @@ int oracle_decode_dense(int d, int hq, int hkv, int pct, int L, const double *t_
     free(kp); free(qp); free(a); free(s); free(sel); free(in_s);
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * (0) calibrated transform pair -- the step before the path ("Paired
+ * transforms instead of shared rotation": partial key whitening combined
+ * with a query-aligned basis, guided by calibrated query and key
+ * statistics).  Written out from its definition:
+ *
+ *   C_K = K^T K / n + eps I,  eps = 1e-6 * trace(K^T K / n) / d
+ *   P   = C_K^(alpha/2)                       (alpha = 1/2: partial whitening)
+ *   C_Q = P (Q^T Q / m) P                     (second moment of P q)
+ *   C_Q = U diag(mu) U^T, mu descending, each column of U signed so that its
+ *         entry of largest magnitude (lowest index on ties) is positive
+ *   T_K = U^T P^-1,  T_Q = U^T P              (so T_Q = T_K^-T, q'.k' = q.k)
+ *
+ * Matrix functions and eigenvectors come from a cyclic Jacobi
+ * eigen-solver (plain rotations until the off-diagonal mass vanishes).
+ * ---------------------------------------------------------------------- */
+
+/* Eigen-decomposition of the symmetric d x d matrix A (destroyed): eigenvalues
+ * in w[], eigenvectors as the columns of V (row-major V[i*d + k]). */
+static void jacobi_eigen(int d, double *A, double *w, double *V)
+{
+    for (int i = 0; i < d; ++i)
+        for (int k = 0; k < d; ++k) V[(size_t)i * d + k] = (i == k) ? 1.0 : 0.0;
+    for (int sweep = 0; sweep < 100; ++sweep) {
+        double off = 0.0, tot = 0.0;
+        for (int i = 0; i < d; ++i)
+            for (int k = 0; k < d; ++k) {
+                const double a = A[(size_t)i * d + k] * A[(size_t)i * d + k];
+                tot += a;
+                if (i != k) off += a;
+            }
+        if (off <= 1e-30 * tot) break;
+        for (int p = 0; p < d - 1; ++p)
+            for (int q = p + 1; q < d; ++q) {
+                const double apq = A[(size_t)p * d + q];
+                if (apq == 0.0) continue;
+                const double app = A[(size_t)p * d + p], aqq = A[(size_t)q * d + q];
+                const double theta = (aqq - app) / (2.0 * apq);
+                const double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
+                const double c = 1.0 / sqrt(t * t + 1.0), s = t * c;
+                for (int k = 0; k < d; ++k) {       /* A <- A J (columns p, q) */
+                    const double akp = A[(size_t)k * d + p], akq = A[(size_t)k * d + q];
+                    A[(size_t)k * d + p] = c * akp - s * akq;
+                    A[(size_t)k * d + q] = s * akp + c * akq;
+                }
+                for (int k = 0; k < d; ++k) {       /* A <- J^T A (rows p, q) */
+                    const double apk = A[(size_t)p * d + k], aqk = A[(size_t)q * d + k];
+                    A[(size_t)p * d + k] = c * apk - s * aqk;
+                    A[(size_t)q * d + k] = s * apk + c * aqk;
+                }
+                for (int k = 0; k < d; ++k) {       /* V <- V J */
+                    const double vkp = V[(size_t)k * d + p], vkq = V[(size_t)k * d + q];
+                    V[(size_t)k * d + p] = c * vkp - s * vkq;
+                    V[(size_t)k * d + q] = s * vkp + c * vkq;
+                }
+            }
+    }
+    for (int i = 0; i < d; ++i) w[i] = A[(size_t)i * d + i];
+}
+
+/* B = V diag(f(w)) V^T with f(x) = x^e. */
+static void sym_power(int d, const double *w, const double *V, double e, double *B)
+{
+    for (int i = 0; i < d; ++i)
+        for (int k = 0; k < d; ++k) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j) acc += V[(size_t)i * d + j] * pow(w[j], e) * V[(size_t)k * d + j];
+            B[(size_t)i * d + k] = acc;
+        }
+}
+
+int oracle_calibrate(int d, long long n, long long m, double alpha, const double *K, const double *Q,
+                     double *t_k, double *t_q)
+{
+    if (d <= 0 || n <= 0 || m <= 0) return 1;
+    const size_t dd = (size_t)d * d;
+    double *A = (double *)calloc(dd, sizeof(double));
+    double *V = (double *)malloc(dd * sizeof(double));
+    double *w = (double *)malloc((size_t)d * sizeof(double));
+    double *P = (double *)malloc(dd * sizeof(double));
+    double *Pi = (double *)malloc(dd * sizeof(double));
+    double *S = (double *)calloc(dd, sizeof(double));
+    double *U = (double *)malloc(dd * sizeof(double));
+    double *mu = (double *)malloc((size_t)d * sizeof(double));
+    int *ord = (int *)malloc((size_t)d * sizeof(int));
+    /* key second moment plus a small ridge */
+    for (long long r = 0; r < n; ++r)
+        for (int i = 0; i < d; ++i)
+            for (int k = 0; k < d; ++k) A[(size_t)i * d + k] += K[r * d + i] * K[r * d + k];
+    double tr = 0.0;
+    for (int i = 0; i < d; ++i) tr += A[(size_t)i * d + i] / (double)n;
+    for (size_t i = 0; i < dd; ++i) A[i] /= (double)n;
+    for (int i = 0; i < d; ++i) A[(size_t)i * d + i] += 1e-6 * tr / d;
+    jacobi_eigen(d, A, w, V);
+    sym_power(d, w, V, alpha / 2.0, P);
+    sym_power(d, w, V, -alpha / 2.0, Pi);
+    /* query second moment in the partially whitened frame: P (Q^T Q / m) P */
+    double *M = (double *)calloc(dd, sizeof(double));
+    for (long long r = 0; r < m; ++r)
+        for (int i = 0; i < d; ++i)
+            for (int k = 0; k < d; ++k) M[(size_t)i * d + k] += Q[r * d + i] * Q[r * d + k];
+    for (size_t i = 0; i < dd; ++i) M[i] /= (double)m;
+    for (int i = 0; i < d; ++i)
+        for (int k = 0; k < d; ++k) {
+            double acc = 0.0;
+            for (int a = 0; a < d; ++a)
+                for (int b = 0; b < d; ++b) acc += P[(size_t)i * d + a] * M[(size_t)a * d + b] * P[(size_t)b * d + k];
+            S[(size_t)i * d + k] = acc;
+        }
+    jacobi_eigen(d, S, mu, U);
+    /* order by descending energy (stable), fix signs */
+    for (int i = 0; i < d; ++i) ord[i] = i;
+    for (int i = 1; i < d; ++i) {
+        const int x = ord[i];
+        int j = i - 1;
+        while (j >= 0 && mu[ord[j]] < mu[x]) { ord[j + 1] = ord[j]; --j; }
+        ord[j + 1] = x;
+    }
+    for (int c = 0; c < d; ++c) {
+        const int src = ord[c];
+        int arg = 0;
+        for (int i = 1; i < d; ++i)
+            if (fabs(U[(size_t)i * d + src]) > fabs(U[(size_t)arg * d + src])) arg = i;
+        const double sgn = U[(size_t)arg * d + src] < 0.0 ? -1.0 : 1.0;
+        /* row c of T_K = (column src of U)^T P^-1, row c of T_Q = (column src)^T P */
+        for (int k = 0; k < d; ++k) {
+            double ak = 0.0, bk = 0.0;
+            for (int i = 0; i < d; ++i) {
+                ak += sgn * U[(size_t)i * d + src] * Pi[(size_t)i * d + k];
+                bk += sgn * U[(size_t)i * d + src] * P[(size_t)i * d + k];
+            }
+            t_k[(size_t)c * d + k] = ak;
+            t_q[(size_t)c * d + k] = bk;
+        }
+    }
+    free(A); free(V); free(w); free(P); free(Pi); free(S); free(U); free(mu); free(ord); free(M);
+    return 0;
+}

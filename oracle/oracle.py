@@ -58,6 +58,8 @@ def lib():
         _lib.oracle_decode_seq.argtypes = [C.c_int] * 6 + [P] * 10 + [P, P, P, C.c_int]
         _lib.oracle_decode_dense.restype = C.c_int
         _lib.oracle_decode_dense.argtypes = [C.c_int] * 5 + [P] * 7
+        _lib.oracle_calibrate.restype = C.c_int
+        _lib.oracle_calibrate.argtypes = [C.c_int, C.c_longlong, C.c_longlong, C.c_double, P, P, P, P]
     return _lib
 
 
@@ -212,3 +214,16 @@ def dequant(cache: Cache, v_ch0: bool = False):
             x[..., 0] = bf(cache[pre + "ch0"])
         out.append(x)
     return out[0], out[1]
+
+
+def calibrate(k: np.ndarray, q: np.ndarray, alpha: float = 0.5):
+    """Calibrated transform pair of one kv head from calibration keys k [n][d]
+    and queries q [m][d] (fp64 results T_K, T_Q; see oracle_calibrate)."""
+    k, q = _f64(k), _f64(q)
+    d = k.shape[1]
+    t_k = np.empty((d, d), np.float64)
+    t_q = np.empty((d, d), np.float64)
+    rc = lib().oracle_calibrate(d, k.shape[0], q.shape[0], float(alpha), _p(k), _p(q), _p(t_k), _p(t_q))
+    if rc:
+        raise ValueError(f"oracle_calibrate failed ({rc})")
+    return t_k, t_q

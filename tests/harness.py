@@ -21,6 +21,28 @@ ATOL = 2e-3          # max abs error on fp32 outputs
 RTOL_ROW = 1e-2      # relative error per output row (||o - o_ref|| / ||o_ref||)
 
 
+_TRANSFORMS = {}
+
+
+def workload_transforms(w: I.Workload):
+    """(t_k32, t_q32, t_k64, t_q64) of a workload, the same arrays for the device
+    and the oracle.  Calibrated pairs are built by the oracle's own calibration
+    from the workload's calibration rows."""
+    key = w
+    if key not in _TRANSFORMS:
+        if w.transform == "calibrated":
+            k, q = I.calibration_rows(w)
+            g = w.hq // w.hkv
+            tk = np.empty((w.hkv, w.d, w.d))
+            tq = np.empty((w.hkv, w.d, w.d))
+            for j in range(w.hkv):
+                tk[j], tq[j] = O.calibrate(k[:, j, :], q[:, j * g:(j + 1) * g, :].reshape(-1, w.d))
+            _TRANSFORMS[key] = (tk.astype(np.float32), tq.astype(np.float32), tk, tq)
+        else:
+            _TRANSFORMS[key] = I.transforms(w)
+    return _TRANSFORMS[key]
+
+
 def torch_dtype(w):
     return torch.bfloat16 if w.kv_dtype == "bf16" else torch.float32
 
@@ -36,7 +58,7 @@ class DeviceRun:
         self.lens = I.lengths(w) if lens is None else np.asarray(lens, dtype=np.int32)
         self.table, self.num_pages = I.page_table(w, np.maximum(self.lens, 1))
         self.max_pages = self.table.shape[1]
-        tk, tq, _, _ = I.transforms(w)
+        tk, tq, _, _ = workload_transforms(w)
         self.tk_host, self.tq_host = tk, tq
         self.t_k = torch.from_numpy(tk).to(self.dev)
         self.t_q = torch.from_numpy(tq).to(self.dev)
@@ -191,7 +213,7 @@ def decode_pool(pool: np.ndarray, table_row: np.ndarray, L: int, d: int, v_ch0: 
 # oracle side
 # ---------------------------------------------------------------------------
 def oracle_cache(w: I.Workload, b: int, L: int, heads=None) -> O.Cache:
-    tk, _, _, _ = I.transforms(w)
+    tk, _, _, _ = workload_transforms(w)
     k, v = I.kv_rows(w, b, 0, L)
     if heads is not None:
         k, v, tk = k[:, heads], v[:, heads], tk[heads]
@@ -201,7 +223,7 @@ def oracle_cache(w: I.Workload, b: int, L: int, heads=None) -> O.Cache:
 def oracle_reference(w: I.Workload, run: DeviceRun, pct: int | None = None, lens=None) -> dict:
     pct = w.pct if pct is None else pct
     lens = run.lens if lens is None else np.asarray(lens)
-    _, tq, _, _ = I.transforms(w)
+    _, tq, _, _ = workload_transforms(w)
     outs, sels, caches = [], [], []
     shared = w.page_order == "shared"
     base = oracle_cache(w, 0, int(lens.max())) if shared else None

@@ -37,6 +37,8 @@ CASES = {
     "g1-d128": small("llama", batch=2, hq=4, hkv=4, ctx=257),
     "g2-d64": small("llama", batch=2, hq=8, hkv=4, d=64, ctx=500),
     "g8": small("llama", batch=2, hq=16, hkv=2, ctx=600),
+    # calibrated transform pair and structured queries (next-step row f1)
+    "calibrated": small("llama_cal", batch=2, ctx=None, ctx_lo=300, ctx_hi=900),
 }
 
 
@@ -126,7 +128,7 @@ def test_invalid_arguments_are_rejected_before_launch():
 
 # ---------------------------------------------------------------- full sizes
 def _sampled_units(w, run, out, sel, units):
-    _, tq, _, _ = I.transforms(w)
+    _, tq, _, _ = H.workload_transforms(w)
     G = w.group
     for b, j in units:
         L = int(run.lens[b])
