@@ -159,10 +159,11 @@ class Layer:
         tk, tq, _, _ = Cb.layer_transforms(w)
         self.t_k = torch.from_numpy(tk).to(dev)
         self.t_q = torch.from_numpy(tq).to(dev)
-        probe = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, 0, 1)
+        probe = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, 0, 1, group_size=w.group_size)
         self.bb = Q.dqk_block_bytes(probe)
         self.pool = torch.empty(self.num_pages * w.hkv * self.bb, dtype=torch.uint8, device=dev)
-        self.desc = Q.layer_desc(w.d, w.hq, w.hkv, self.t_k, self.t_q, self.pool, self.num_pages)
+        self.desc = Q.layer_desc(w.d, w.hq, w.hkv, self.t_k, self.t_q, self.pool, self.num_pages,
+                                 group_size=w.group_size)
         self.table_d = torch.from_numpy(self.table).to(dev)
         self.lens_d = torch.from_numpy(self.lens).to(dev)
         self.ws_bytes = Q.dqk_decode_workspace_size(self.desc, w.batch, self.max_pages)
@@ -236,7 +237,7 @@ def algorithmic_bytes(w, sel: np.ndarray, lens: np.ndarray) -> tuple[float, floa
     """Bytes the attend kernel must touch per launch (retained-channel key
     codes for the union of the GQA group's kept channels, K scale/min of
     touched groups, K channel 0, V codes, V scale/min) and per token-kv-head."""
-    G, ng = w.group, w.d // 32
+    G, ns = w.group, w.d // w.group_size
     total = 0.0
     for b in range(len(lens)):
         for j in range(w.hkv):
@@ -244,8 +245,8 @@ def algorithmic_bytes(w, sel: np.ndarray, lens: np.ndarray) -> tuple[float, floa
             kept[sel[b, j * G:(j + 1) * G].ravel()] = True
             kept[0] = False
             u = int(kept.sum())
-            groups = int(kept.reshape(ng, 32).any(axis=1).sum())
-            per_tok = -(-u // 4) + 4 * groups + 2 + w.d // 4 + 4 * ng
+            groups = int(kept.reshape(ns, w.group_size).any(axis=1).sum())
+            per_tok = -(-u // 4) + 4 * groups + 2 + w.d // 4 + 4 * ns
             total += per_tok * int(lens[b])
     return total, total / (w.hkv * float(np.sum(lens)))
 

@@ -29,15 +29,18 @@ struct AppendSmem {
 // fp16(min), code = clamp(rne((x - min) / scale), 0, 3) (0 when scale is 0).
 // excluded: this lane's value (channel 0 of a protected key) takes no part
 // and gets code 0.
-__device__ __forceinline__ int quantize_group(float xv, bool excluded, uint16_t &sh, uint16_t &mh) {
-    const float x = xv + 0.0f;
-    float lo = excluded ? __int_as_float(0x7f800000) : x;
-    float hi = excluded ? __int_as_float(0xff800000) : x;
+__device__ __forceinline__ void warp_minmax(float x, bool excluded, float &lo, float &hi) {
+    lo = excluded ? __int_as_float(0x7f800000) : x;
+    hi = excluded ? __int_as_float(0xff800000) : x;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
+}
+
+// scale/min of a group from its range, and the code of x
+__device__ __forceinline__ int quant_code(float x, bool excluded, float lo, float hi, uint16_t &sh, uint16_t &mh) {
     sh = f64_to_f16_rne(((double)hi - (double)lo) / 3.0);
     mh = f64_to_f16_rne((double)lo);
     const double s = f16_to_f64(sh), mn = f16_to_f64(mh);
@@ -49,22 +52,51 @@ __device__ __forceinline__ int quantize_group(float xv, bool excluded, uint16_t 
     return code;
 }
 
+__device__ __forceinline__ int quantize_group(float xv, bool excluded, uint16_t &sh, uint16_t &mh) {
+    const float x = xv + 0.0f;
+    float lo, hi;
+    warp_minmax(x, excluded, lo, hi);
+    return quant_code(x, excluded, lo, hi, sh, mh);
+}
+
 // Quantize the D values a warp holds (lane owns channels lane + 32*m, i.e.
-// channel `lane` of group m) into codes / fp16 scale / fp16 min / BF16 ch0.
+// channel `lane` of block m) into codes / fp16 scale / fp16 min / BF16 ch0,
+// with NS scale groups (NG of 32 channels, or 1 over the whole row).
 // protect: channel 0 goes to BF16, is excluded from group 0's range and its
 // code is 0.
-template <int NG>
+template <int NG, int NS>
 __device__ __forceinline__ void quantize_warp(const float (&vals)[NG], bool protect, int lane,
                                               uint8_t *codes, uint16_t *scale, uint16_t *minv,
                                               uint16_t *ch0) {
+    if constexpr (NS == 1) {
+        float lo = __int_as_float(0x7f800000), hi = __int_as_float(0xff800000);
 #pragma unroll
-    for (int m = 0; m < NG; ++m) {
-        uint16_t sh, mh;
-        const int code = quantize_group(vals[m], protect && m == 0 && lane == 0, sh, mh);
-        codes[m * kGroup + lane] = (uint8_t)code;
-        if (lane == 0) {
-            scale[m] = sh;
-            minv[m] = mh;
+        for (int m = 0; m < NG; ++m) {
+            float l, h;
+            warp_minmax(vals[m] + 0.0f, protect && m == 0 && lane == 0, l, h);
+            lo = fminf(lo, l);
+            hi = fmaxf(hi, h);
+        }
+#pragma unroll
+        for (int m = 0; m < NG; ++m) {
+            uint16_t sh, mh;
+            const int code = quant_code(vals[m] + 0.0f, protect && m == 0 && lane == 0, lo, hi, sh, mh);
+            codes[m * kGroup + lane] = (uint8_t)code;
+            if (lane == 0 && m == 0) {
+                scale[0] = sh;
+                minv[0] = mh;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < NG; ++m) {
+            uint16_t sh, mh;
+            const int code = quantize_group(vals[m], protect && m == 0 && lane == 0, sh, mh);
+            codes[m * kGroup + lane] = (uint8_t)code;
+            if (lane == 0) {
+                scale[m] = sh;
+                minv[m] = mh;
+            }
         }
     }
     if (lane == 0) *ch0 = protect ? f32_to_bf16_rne(vals[0]) : (uint16_t)0;
@@ -101,12 +133,13 @@ __device__ void unpack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
         S.vcode[t][c] = (uint8_t)((*reinterpret_cast<const uint32_t *>(vb + off) >> bit) & 3u);
     }
     const uint16_t *h = reinterpret_cast<const uint16_t *>(S.blk);
-    for (int idx = threadIdx.x; idx < kPage * NG; idx += blockDim.x) {
-        const int t = idx / NG, g = idx % NG;
-        S.kscale[t][g] = h[(L.ks >> 1) + kscale_idx(NG, t, g)];
-        S.kmin[t][g] = h[(L.km >> 1) + kscale_idx(NG, t, g)];
-        S.vscale[t][g] = h[(L.vs >> 1) + vscale_idx(NG, t, g)];
-        S.vmin[t][g] = h[(L.vm >> 1) + vscale_idx(NG, t, g)];
+    const int ns = L.ns;
+    for (int idx = threadIdx.x; idx < kPage * ns; idx += blockDim.x) {
+        const int t = idx / ns, g = idx % ns;
+        S.kscale[t][g] = h[(L.ks >> 1) + kscale_idx(ns, t, g)];
+        S.kmin[t][g] = h[(L.km >> 1) + kscale_idx(ns, t, g)];
+        S.vscale[t][g] = h[(L.vs >> 1) + vscale_idx(ns, t, g)];
+        S.vmin[t][g] = h[(L.vm >> 1) + vscale_idx(ns, t, g)];
     }
     for (int t = threadIdx.x; t < kPage; t += blockDim.x) {
         S.kch0[t] = h[(L.k0 >> 1) + k0_idx(t)];
@@ -140,12 +173,13 @@ __device__ void pack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
         atomicOr(&w[(L.vc + off) >> 2], ((uint32_t)S.vcode[t][c] & 3u) << bit);
     }
     uint16_t *h = reinterpret_cast<uint16_t *>(S.blk);
-    for (int idx = threadIdx.x; idx < kPage * NG; idx += blockDim.x) {
-        const int t = idx / NG, g = idx % NG;
-        h[(L.ks >> 1) + kscale_idx(NG, t, g)] = S.kscale[t][g];
-        h[(L.km >> 1) + kscale_idx(NG, t, g)] = S.kmin[t][g];
-        h[(L.vs >> 1) + vscale_idx(NG, t, g)] = S.vscale[t][g];
-        h[(L.vm >> 1) + vscale_idx(NG, t, g)] = S.vmin[t][g];
+    const int ns = L.ns;
+    for (int idx = threadIdx.x; idx < kPage * ns; idx += blockDim.x) {
+        const int t = idx / ns, g = idx % ns;
+        h[(L.ks >> 1) + kscale_idx(ns, t, g)] = S.kscale[t][g];
+        h[(L.km >> 1) + kscale_idx(ns, t, g)] = S.kmin[t][g];
+        h[(L.vs >> 1) + vscale_idx(ns, t, g)] = S.vscale[t][g];
+        h[(L.vm >> 1) + vscale_idx(ns, t, g)] = S.vmin[t][g];
     }
     for (int t = threadIdx.x; t < kPage; t += blockDim.x) {
         h[(L.k0 >> 1) + k0_idx(t)] = S.kch0[t];
@@ -161,7 +195,7 @@ __device__ void pack_block(AppendSmem<D> &S, const Layout &L, int v_ch0) {
 // token slot w.  early_release lets a kernel launched after this one with
 // programmatic stream serialization start at once (it must not read the
 // cache before its own grid-dependency wait).
-template <int D>
+template <int D, int NS>
 __global__ void __launch_bounds__(512) k_quant_pack(
     const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin,
     int dtype, int batch, const int *__restrict__ new_lens, const int *__restrict__ seq_before,
@@ -173,7 +207,7 @@ __global__ void __launch_bounds__(512) k_quant_pack(
     AppendSmem<D> &S = *reinterpret_cast<AppendSmem<D> *>(smem_raw);
     const int j = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Layout L = make_layout(D, v_ch0);
+    const Layout L = make_layout(D, v_ch0, NS);
     if (early_release) grid_dependents_launch();
 
     stage_f64_padded<D>(S.tk, t_k + (size_t)j * D * D);
@@ -234,12 +268,13 @@ __global__ void __launch_bounds__(512) k_quant_pack(
             float kp[NG];
 #pragma unroll
             for (int m = 0; m < NG; ++m) kp[m] = S.kp[warp][lane + 32 * m];
-            quantize_warp<NG>(kp, true, lane, S.kcode[warp], S.kscale[warp], S.kmin[warp], &S.kch0[warp]);
+            quantize_warp<NG, NS>(kp, true, lane, S.kcode[warp], S.kscale[warp], S.kmin[warp], &S.kch0[warp]);
             const size_t base = ((size_t)(row_of_slot + warp) * hkv + j) * D;
             float vv[NG];
 #pragma unroll
             for (int m = 0; m < NG; ++m) vv[m] = load_elem(vin, dtype, base + lane + 32 * m);
-            quantize_warp<NG>(vv, v_ch0 != 0, lane, S.vcode[warp], S.vscale[warp], S.vmin[warp], &S.vch0[warp]);
+            quantize_warp<NG, NS>(vv, v_ch0 != 0, lane, S.vcode[warp], S.vscale[warp], S.vmin[warp],
+                                  &S.vch0[warp]);
         }
         __syncthreads();
         pack_block<D>(S, L, v_ch0);
@@ -264,7 +299,7 @@ __global__ void __launch_bounds__(512) k_quant_pack(
 constexpr int kDirectMaxNew = 64;   // dqk_append uses k_append_rows up to this many rows per sequence
 constexpr int kRowsPerCta = 4;
 
-template <int D>
+template <int D, int NS>
 __global__ void __launch_bounds__(D) k_append_rows(
     const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin, int dtype,
     const int *__restrict__ new_lens, const int *__restrict__ seq_before, const int *__restrict__ page_table,
@@ -319,11 +354,40 @@ __global__ void __launch_bounds__(D) k_append_rows(
 #pragma unroll
             for (int i = 0; i < RW; ++i) acc[i] = fma(t4[e], xs[i][4 * u + e], acc[i]);
     }
-    const Layout L = make_layout(D, v_ch0);
+    const Layout L = make_layout(D, v_ch0, NS);
+    // group ranges: per warp (32 channels); with one group per row, combined
+    // over the row's NG warps through shared memory
+    __shared__ float rng[NS == 1 ? RW : 1][4][NG];
+    float kp[RW], klo[RW], khi[RW], vlo[RW], vhi[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        kp[i] = __double2float_rn(acc[i]);    // channel 0 keeps its sign; ranges read -0 as +0
+        warp_minmax(kp[i] + 0.0f, c == 0, klo[i], khi[i]);
+        warp_minmax(xv[i] + 0.0f, v_ch0 != 0 && c == 0, vlo[i], vhi[i]);
+        if constexpr (NS == 1) {
+            if (lane == 0) {
+                rng[i][0][warp] = klo[i];
+                rng[i][1][warp] = khi[i];
+                rng[i][2][warp] = vlo[i];
+                rng[i][3][warp] = vhi[i];
+            }
+        }
+    }
+    if constexpr (NS == 1) {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < RW; ++i)
+#pragma unroll
+            for (int w = 0; w < NG; ++w) {
+                klo[i] = fminf(klo[i], rng[i][0][w]);
+                khi[i] = fmaxf(khi[i], rng[i][1][w]);
+                vlo[i] = fminf(vlo[i], rng[i][2][w]);
+                vhi[i] = fmaxf(vhi[i], rng[i][3][w]);
+            }
+    }
 #pragma unroll
     for (int i = 0; i < RW; ++i) {
         if (i >= nr) break;                   // uniform
-        const float kp = __double2float_rn(acc[i]);
         if (phys[i] < 0 || phys[i] >= num_pages) {   // uniform
             if (c == 0) dqk_flag_error(kErrBounds);
             continue;
@@ -331,16 +395,17 @@ __global__ void __launch_bounds__(D) k_append_rows(
         const int slot = (L0 + t0 + i) % kPage;
         uint16_t *h16 = reinterpret_cast<uint16_t *>(pool + ((size_t)phys[i] * hkv + j) * L.bytes);
         uint16_t ksh, kmh, vsh, vmh;
-        const int kc = quantize_group(kp, c == 0, ksh, kmh);
-        const int vc = quantize_group(xv[i], v_ch0 != 0 && c == 0, vsh, vmh);
-        if (lane == 0) {
-            h16[(L.ks >> 1) + kscale_idx(NG, slot, warp)] = ksh;
-            h16[(L.km >> 1) + kscale_idx(NG, slot, warp)] = kmh;
-            h16[(L.vs >> 1) + vscale_idx(NG, slot, warp)] = vsh;
-            h16[(L.vm >> 1) + vscale_idx(NG, slot, warp)] = vmh;
+        const int kc = quant_code(kp[i] + 0.0f, c == 0, klo[i], khi[i], ksh, kmh);
+        const int vc = quant_code(xv[i] + 0.0f, v_ch0 != 0 && c == 0, vlo[i], vhi[i], vsh, vmh);
+        if (NS == 1 ? c == 0 : lane == 0) {
+            const int g = NS == 1 ? 0 : warp;
+            h16[(L.ks >> 1) + kscale_idx(NS, slot, g)] = ksh;
+            h16[(L.km >> 1) + kscale_idx(NS, slot, g)] = kmh;
+            h16[(L.vs >> 1) + vscale_idx(NS, slot, g)] = vsh;
+            h16[(L.vm >> 1) + vscale_idx(NS, slot, g)] = vmh;
         }
         if (c == 0) {
-            h16[(L.k0 >> 1) + k0_idx(slot)] = f32_to_bf16_rne(kp);
+            h16[(L.k0 >> 1) + k0_idx(slot)] = f32_to_bf16_rne(kp[i]);
             if (v_ch0) h16[(L.v0 >> 1) + slot] = f32_to_bf16_rne(xv[i]);
         }
         int off, bit;

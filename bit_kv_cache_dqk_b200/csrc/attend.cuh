@@ -203,38 +203,52 @@ struct LaneOffsets {
 // (softmax weights and the value accumulation).  NB (page, kv head) blocks at
 // shared addresses sb[], same run; MASKED (NB == 1 only): only the first nv
 // tokens are valid.
-template <int D, int G, int NB, bool MASKED>
+template <int D, int G, int NS, int NB, bool MASKED>
 __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, const WarpState<D, G> &st, int lane,
                                           const LaneOffsets &o, float (&s0)[NB][AttendTile<D, G>::NT],
                                           float (&s1)[NB][AttendTile<D, G>::NT]) {
     using T = AttendTile<D, G>;
     constexpr int NG = T::NG, NT = T::NT;
-    constexpr Layout Ly = make_layout(D, 0);   // section offsets do not depend on v_ch0 (V0 is last)
+    constexpr Layout Ly = make_layout(D, 0, NS);   // section offsets do not depend on v_ch0 (V0 is last)
     static_assert(NB == 1 || !MASKED, "masked blocks are processed alone");
     const int gid = lane >> 2;
 
-    uint32_t kw[NB][NG], ks0[NB][NG / 2], ks1[NB][NG / 2], km0[NB], km1[NB];
+    constexpr int KS = NS == 1 ? 1 : NG / 2;   // words of key scales per token
+    uint32_t kw[NB][NG], ks0[NB][KS], ks1[NB][KS], km0[NB], km1[NB];
     float k0a[NB], k0b[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
         if constexpr (NG == 4) {
             const uint4 v = ld_s128(sb[b] + o.lane16 + Ly.kc);
             kw[b][0] = v.x; kw[b][1] = v.y; kw[b][2] = v.z; kw[b][3] = v.w;
-            const uint32_t a = sb[b] + o.gid8;
-            const uint2 x = ld_s64(a + Ly.ks), y = ld_s64(a + Ly.ks + 64);
-            ks0[b][0] = x.x; ks0[b][1] = x.y; ks1[b][0] = y.x; ks1[b][1] = y.y;
         } else {
             const uint2 v = ld_s64(sb[b] + (o.lane16 >> 1) + Ly.kc);
             kw[b][0] = v.x; kw[b][1] = v.y;
-            const uint32_t a = sb[b] + (o.gid8 >> 1);
-            ks0[b][0] = ld_s32(a + Ly.ks);
-            ks1[b][0] = ld_s32(a + Ly.ks + 32);
         }
-        const uint32_t akm = sb[b] + o.kmin;
-        // lanes past the groups read this token's other mins; the min-term B
-        // operand is zero in those rows
-        km0[b] = ld_s32(akm + Ly.km);
-        km1[b] = ld_s32(akm + Ly.km + 16 * NG);
+        if constexpr (NS == 1) {
+            // one scale and one min per token: tokens gid and gid + 8
+            const uint32_t a = sb[b] + (o.gid4 >> 1);
+            ks0[b][0] = ld_s16(a + Ly.ks);
+            ks1[b][0] = ld_s16(a + Ly.ks + 16);
+            const uint32_t m0 = ld_s16(a + Ly.km), m1 = ld_s16(a + Ly.km + 16);
+            km0[b] = m0 | (m0 << 16);          // the same min against every group's Qsum
+            km1[b] = m1 | (m1 << 16);
+        } else {
+            if constexpr (NG == 4) {
+                const uint32_t a = sb[b] + o.gid8;
+                const uint2 x = ld_s64(a + Ly.ks), y = ld_s64(a + Ly.ks + 64);
+                ks0[b][0] = x.x; ks0[b][1] = x.y; ks1[b][0] = y.x; ks1[b][1] = y.y;
+            } else {
+                const uint32_t a = sb[b] + (o.gid8 >> 1);
+                ks0[b][0] = ld_s32(a + Ly.ks);
+                ks1[b][0] = ld_s32(a + Ly.ks + 32);
+            }
+            const uint32_t akm = sb[b] + o.kmin;
+            // lanes past the groups read this token's other mins; the min-term B
+            // operand is zero in those rows
+            km0[b] = ld_s32(akm + Ly.km);
+            km1[b] = ld_s32(akm + Ly.km + 16 * NG);
+        }
         const uint32_t k0w = ld_s32(sb[b] + o.gid4 + Ly.k0);
         k0a[b] = __uint_as_float(k0w << 16);
         k0b[b] = __uint_as_float(k0w & 0xffff0000u);
@@ -275,8 +289,14 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
                 A2 = (kw[b][0] >> 4) & msk; A3 = (kw[b][1] >> 4) & msk;
             }
             // key scales of tokens gid and gid + 8
-            const float sa = (g & 1) ? f16hi_to_f32(ks0[b][g >> 1]) : f16lo_to_f32(ks0[b][g >> 1]);
-            const float sbv = (g & 1) ? f16hi_to_f32(ks1[b][g >> 1]) : f16lo_to_f32(ks1[b][g >> 1]);
+            float sa, sbv;
+            if constexpr (NS == 1) {
+                sa = f16lo_to_f32(ks0[b][0]);
+                sbv = f16lo_to_f32(ks1[b][0]);
+            } else {
+                sa = (g & 1) ? f16hi_to_f32(ks0[b][g >> 1]) : f16lo_to_f32(ks0[b][g >> 1]);
+                sbv = (g & 1) ? f16hi_to_f32(ks1[b][g >> 1]) : f16lo_to_f32(ks1[b][g >> 1]);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 int dg[4];
@@ -338,41 +358,49 @@ __device__ __forceinline__ void max_update(WarpState<D, G> &st, const float (&s0
     }
 }
 
-template <int D, int G, bool VCH0, int NB, bool MASKED>
+template <int D, int G, bool VCH0, int NS, int NB, bool MASKED>
 __device__ __forceinline__ void pv_accum(const uint32_t (&sb)[NB], int nv, WarpState<D, G> &st, int lane,
                                          const LaneOffsets &o, const float (&s0)[NB][AttendTile<D, G>::NT],
                                          const float (&s1)[NB][AttendTile<D, G>::NT]) {
     using T = AttendTile<D, G>;
     constexpr int NG = T::NG, NT = T::NT;
-    constexpr Layout Ly = make_layout(D, 0);
+    constexpr Layout Ly = make_layout(D, 0, NS);
     const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        uint32_t vw[NG], vsa[NG], vsb[NG];   // vsa/vsb: scale pairs of tokens (2tig, 2tig+1) and (+8, +9)
+        // vsa/vsb: scale pairs of tokens (2tig, 2tig+1) and (+8, +9), per scale group
+        uint32_t vw[NG], vsa[NS], vsb[NS];
         if constexpr (NG == 4) {
             const uint4 v = ld_s128(sb[b] + o.lane16 + Ly.vc);
             vw[0] = v.x; vw[1] = v.y; vw[2] = v.z; vw[3] = v.w;
+        } else {
+            const uint2 v = ld_s64(sb[b] + (o.lane16 >> 1) + Ly.vc);
+            vw[0] = v.x; vw[1] = v.y;
+        }
+        if constexpr (NS == 4) {
             const uint32_t a = sb[b] + o.tig16;
             const uint4 x = ld_s128(a + Ly.vs), y = ld_s128(a + Ly.vs + 64);
             vsa[0] = x.x; vsa[1] = x.y; vsa[2] = x.z; vsa[3] = x.w;
             vsb[0] = y.x; vsb[1] = y.y; vsb[2] = y.z; vsb[3] = y.w;
-        } else {
-            const uint2 v = ld_s64(sb[b] + (o.lane16 >> 1) + Ly.vc);
-            vw[0] = v.x; vw[1] = v.y;
+        } else if constexpr (NS == 2) {
             const uint32_t a = sb[b] + (o.tig16 >> 1);
             const uint2 x = ld_s64(a + Ly.vs), y = ld_s64(a + Ly.vs + 32);
             vsa[0] = x.x; vsa[1] = x.y;
             vsb[0] = y.x; vsb[1] = y.y;
+        } else {
+            const uint32_t a = sb[b] + (o.tig16 >> 2);
+            vsa[0] = ld_s32(a + Ly.vs);
+            vsb[0] = ld_s32(a + Ly.vs + 16);
         }
-        // A rows of the min / denominator / channel-0 product: row g < NG = v-min
-        // of group g, row NG = ones, row NG+1 = value channel 0 (when protected).
+        // A rows of the min / denominator / channel-0 product: row g < NS = v-min
+        // of scale group g, row NS = ones, row NS+1 = value channel 0 (when protected).
         const uint32_t avm = sb[b] + o.vmin;
         uint32_t vma = (ld_s32(avm + Ly.vm) & o.vmin_mask) | o.ones_lane;
-        uint32_t vmb = (ld_s32(avm + Ly.vm + 16 * NG) & o.vmin_mask) | o.ones_lane;
+        uint32_t vmb = (ld_s32(avm + Ly.vm + 16 * NS) & o.vmin_mask) | o.ones_lane;
         if constexpr (VCH0) {
-            const Layout L1 = make_layout(D, 1);
+            constexpr Layout L1 = make_layout(D, 1, NS);
             const uint32_t a = ld_s32(sb[b] + L1.v0 + tig * 4), c = ld_s32(sb[b] + L1.v0 + 16 + tig * 4);
-            if (gid == NG + 1) {
+            if (gid == NS + 1) {
                 vma = pack_f16x2(__uint_as_float(a << 16), __uint_as_float(a & 0xffff0000u));
                 vmb = pack_f16x2(__uint_as_float(c << 16), __uint_as_float(c & 0xffff0000u));
             }
@@ -382,7 +410,7 @@ __device__ __forceinline__ void pv_accum(const uint32_t (&sb)[NB], int nv, WarpS
             const uint32_t ma = (2 * tig < nv ? 0x0000ffffu : 0u) | (2 * tig + 1 < nv ? 0xffff0000u : 0u);
             const uint32_t mb = (2 * tig + 8 < nv ? 0x0000ffffu : 0u) | (2 * tig + 9 < nv ? 0xffff0000u : 0u);
 #pragma unroll
-            for (int g = 0; g < NG; ++g) {
+            for (int g = 0; g < NS; ++g) {
                 vsa[g] &= ma;
                 vsb[g] &= mb;
             }
@@ -413,7 +441,8 @@ __device__ __forceinline__ void pv_accum(const uint32_t (&sb)[NB], int nv, WarpS
             for (int g = 0; g < NG; ++g) {
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const uint32_t b0 = hmul2(pb0[nt], vsa[g]), b1 = hmul2(pb1[nt], vsb[g]);
+                    const int gs = NS == 1 ? 0 : g;
+                    const uint32_t b0 = hmul2(pb0[nt], vsa[gs]), b1 = hmul2(pb1[nt], vsb[gs]);
 #pragma unroll
                     for (int mm = 2 * g; mm < 2 * g + 2; ++mm) {
                         const int P = mm <= 4 ? mm : mm - 5;
@@ -433,7 +462,8 @@ __device__ __forceinline__ void pv_accum(const uint32_t (&sb)[NB], int nv, WarpS
                 const uint32_t f1 = code_field<5>(x, xh), f3 = code_field<7>(x, xh);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const uint32_t b0 = hmul2(pb0[nt], vsa[w2]), b1 = hmul2(pb1[nt], vsb[w2]);
+                    const int gs = NS == 1 ? 0 : w2;
+                    const uint32_t b0 = hmul2(pb0[nt], vsa[gs]), b1 = hmul2(pb1[nt], vsb[gs]);
                     mma_f16(st.oacc[nt][2 * w2], e0, e2, e1, e3, b0, b1);
                     mma_f16(st.oacc[nt][2 * w2 + 1], f0, f2, f1, f3, b0, b1);
                 }
@@ -442,14 +472,14 @@ __device__ __forceinline__ void pv_accum(const uint32_t (&sb)[NB], int nv, WarpS
     }
 }
 
-template <int D, int G, bool VCH0, int NB, bool MASKED>
+template <int D, int G, bool VCH0, int NS, int NB, bool MASKED>
 __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpState<D, G> &st, int lane,
                                         const LaneOffsets &o) {
     constexpr int NT = AttendTile<D, G>::NT;
     float s0[NB][NT], s1[NB][NT];
-    qk_scores<D, G, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
+    qk_scores<D, G, NS, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
     max_update<D, G, NB>(st, s0, s1);
-    pv_accum<D, G, VCH0, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
+    pv_accum<D, G, VCH0, NS, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
 }
 
 // Every (run, page slot, kv head) record a consumer warp could own starts
@@ -557,7 +587,7 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
             (void)mbar_wait_bounded(&full[k % S], (uint32_t)(k / S) & 1u, kWaitLimitNs);
 }
 
-template <int D, int G, bool VCH0>
+template <int D, int G, bool VCH0, int NS>
 __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendParams p) {
     using T = AttendTile<D, G>;
     constexpr int kConsumerWarps = attend_warps(G), kStageBlocks = attend_stage_blocks(G);
@@ -624,15 +654,15 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     lo.kmin = gid * 2 * NG + (tig & (NG / 2 - 1)) * 4;   // in range for every lane (B rows past NG are 0)
     lo.gid4 = gid * 4;
     lo.tig16 = tig * 16;
-    lo.vmin = (tig * NG + (gid < NG ? gid : 0)) * 4;
+    lo.vmin = (tig * NS + (gid < NS ? gid : 0)) * 4;
     lo.srcA = (2 * tig) * 4 + (gid >> 1);
     {
         unsigned char *mine = frag_mem + (size_t)warp * NT * NG * (32 * 8 + 4 * 16);
         lo.sq = smem_addr(mine) + lane * 8;
         lo.sk = smem_addr(mine + NT * NG * 32 * 8) + tig * 16;
     }
-    lo.ones_lane = gid == NG ? 0x3C003C00u : 0u;
-    lo.vmin_mask = gid < NG ? 0xffffffffu : 0u;
+    lo.ones_lane = gid == NS ? 0x3C003C00u : 0u;
+    lo.vmin_mask = gid < NS ? 0xffffffffu : 0u;
 
     auto start_run = [&](int rr) {
         const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
@@ -674,11 +704,11 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     auto finish_run = [&](int rr) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float minterm[NG];
+            float minterm[NS];
 #pragma unroll
-            for (int g = 0; g < NG; ++g) minterm[g] = __shfl_sync(0xffffffffu, st.macc[nt][0], g * 4 + tig);
-            const float l = __shfl_sync(0xffffffffu, st.macc[nt][0], NG * 4 + tig);
-            const float v0t = __shfl_sync(0xffffffffu, st.macc[nt][0], (NG + 1) * 4 + tig);
+            for (int g = 0; g < NS; ++g) minterm[g] = __shfl_sync(0xffffffffu, st.macc[nt][0], g * 4 + tig);
+            const float l = __shfl_sync(0xffffffffu, st.macc[nt][0], NS * 4 + tig);
+            const float v0t = __shfl_sync(0xffffffffu, st.macc[nt][0], (NS + 1) * 4 + tig);
             const int hh = 4 * nt + tig;
             if (hh < G) {
                 float *rec = p.part + record_index(slot_base + rr, pi, jl, hh, p.pw, p.hc, G) * (2 + D);
@@ -689,7 +719,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
                     const int c0 = 16 * m + gid, c1 = c0 + 8;
-                    const float mt = minterm[m >> 1];
+                    const float mt = minterm[NS == 1 ? 0 : (m >> 1)];
                     const float f = vfield_scale<NG>(m);
                     rec[2 + c0] = (VCH0 && c0 == 0) ? v0t : fmaf(st.oacc[nt][m][0], f, mt);
                     rec[2 + c1] = fmaf(st.oacc[nt][m][2], f, mt);
@@ -754,7 +784,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
                 uint32_t sbb[BPW];
 #pragma unroll
                 for (int q = 0; q < BPW; ++q) sbb[q] = sa + q * page_gap;
-                consume<D, G, VCH0, BPW, false>(sbb, kPage, st, lane, lo);
+                consume<D, G, VCH0, NS, BPW, false>(sbb, kPage, st, lane, lo);
             } else {
 #pragma unroll
                 for (int q = 0; q < BPW; ++q) {
@@ -763,8 +793,8 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
                     if (uq >= run_end) switch_run(uq);
                     if ((vv >> q) & 1u) {
                         const uint32_t s1[1] = {sa + q * page_gap};
-                        if (uq == partial_u) consume<D, G, VCH0, 1, true>(s1, nv_last, st, lane, lo);
-                        else consume<D, G, VCH0, 1, false>(s1, kPage, st, lane, lo);
+                        if (uq == partial_u) consume<D, G, VCH0, NS, 1, true>(s1, nv_last, st, lane, lo);
+                        else consume<D, G, VCH0, NS, 1, false>(s1, kPage, st, lane, lo);
                     }
                 }
             }

@@ -18,22 +18,23 @@ constexpr unsigned kErrBounds = 1u;
 constexpr unsigned kErrTimeout = 2u;
 
 // Byte offsets of the sections of one (page, kv head) block; see dualqk.h.
+// ns = scale groups per token: d / 32, or 1 (one group over the whole head).
 struct Layout {
-    int d, ng, kc, ks, km, k0, vc, vs, vm, v0, bytes;
+    int d, ns, kc, ks, km, k0, vc, vs, vm, v0, bytes;
 };
 
-__host__ __device__ constexpr Layout make_layout(int d, int v_ch0) {
+__host__ __device__ constexpr Layout make_layout(int d, int v_ch0, int ns) {
     Layout L{};
     L.d = d;
-    L.ng = d / kGroup;
+    L.ns = ns;
     L.kc = 0;
     L.ks = 4 * d;
-    L.km = L.ks + 32 * L.ng;
-    L.k0 = L.km + 32 * L.ng;
+    L.km = L.ks + 32 * ns;
+    L.k0 = L.km + 32 * ns;
     L.vc = L.k0 + 32;
     L.vs = L.vc + 4 * d;
-    L.vm = L.vs + 32 * L.ng;
-    L.v0 = L.vm + 32 * L.ng;
+    L.vm = L.vs + 32 * ns;
+    L.v0 = L.vm + 32 * ns;
     L.bytes = L.v0 + (v_ch0 ? 32 : 0);
     return L;
 }

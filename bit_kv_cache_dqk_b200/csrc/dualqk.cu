@@ -29,7 +29,9 @@ dqk_status check_layer(const dqk_layer_desc *L) {
         return DQK_ERR_INVALID_ARG;
     const int G = L->num_q_heads / L->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return DQK_ERR_UNSUPPORTED;
-    if (L->page_size != kPage || L->group_size != kGroup) return DQK_ERR_UNSUPPORTED;
+    if (L->page_size != kPage) return DQK_ERR_UNSUPPORTED;
+    // scale groups of 32 channels, or one group over the whole head
+    if (L->group_size != kGroup && L->group_size != L->head_dim) return DQK_ERR_UNSUPPORTED;
     if (L->v_ch0_protect != 0 && L->v_ch0_protect != 1) return DQK_ERR_INVALID_ARG;
     if (!L->pool || !aligned(L->pool, 16) || L->num_pages <= 0) return DQK_ERR_INVALID_ARG;
     return DQK_OK;
@@ -72,7 +74,7 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     // Records are sized for kMaxAttendCtas so the workspace size does not depend
     // on the device; the launch (check_decode) uses one CTA per SM up to that bound.
     P.num_ctas = kMaxAttendCtas;
-    P.bb = make_layout(P.d, L->v_ch0_protect).bytes;
+    P.bb = make_layout(P.d, L->v_ch0_protect, P.d / L->group_size).bytes;
     // shared memory: ring stages | mbarriers | valid flags | abort flag | per-warp query fragments
     const size_t stage_bytes = (size_t)stage_blocks * P.bb;
     // (score fragments live in shared memory only for two query-head tiles)
@@ -173,10 +175,10 @@ dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
                       a.sel_out);
 }
 
-template <int D, int G, bool VCH0>
+template <int D, int G, bool VCH0, int NS>
 dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
-    prefer_max_shared(k_attend<D, G, VCH0>);
-    if (cudaFuncSetAttribute(k_attend<D, G, VCH0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
+    prefer_max_shared(k_attend<D, G, VCH0, NS>);
+    if (cudaFuncSetAttribute(k_attend<D, G, VCH0, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
         cudaSuccess)
         return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
@@ -202,17 +204,22 @@ dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
     prm.v_ch0 = a.L->v_ch0_protect;
     prm.stages = P.stages;
     prm.num_ctas = P.num_ctas;
-    return launch_pdl(k_attend<D, G, VCH0>, dim3(P.num_ctas), dim3(attend_threads(G)), P.smem, a.stream, prm);
+    return launch_pdl(k_attend<D, G, VCH0, NS>, dim3(P.num_ctas), dim3(attend_threads(G)), P.smem, a.stream, prm);
+}
+
+template <int D, bool VCH0, int NS>
+dqk_status run_attend_s(const DecodeArgs &a, const DecodePlan &P) {
+    switch (P.G) {
+        case 1: return run_attend_g<D, 1, VCH0, NS>(a, P);
+        case 2: return run_attend_g<D, 2, VCH0, NS>(a, P);
+        case 4: return run_attend_g<D, 4, VCH0, NS>(a, P);
+        default: return run_attend_g<D, 8, VCH0, NS>(a, P);
+    }
 }
 
 template <int D, bool VCH0>
 dqk_status run_attend_v(const DecodeArgs &a, const DecodePlan &P) {
-    switch (P.G) {
-        case 1: return run_attend_g<D, 1, VCH0>(a, P);
-        case 2: return run_attend_g<D, 2, VCH0>(a, P);
-        case 4: return run_attend_g<D, 4, VCH0>(a, P);
-        default: return run_attend_g<D, 8, VCH0>(a, P);
-    }
+    return a.L->group_size == D ? run_attend_s<D, VCH0, 1>(a, P) : run_attend_s<D, VCH0, D / kGroup>(a, P);
 }
 
 template <int D>
@@ -252,22 +259,23 @@ dqk_status decode_stages(const DecodeArgs &a, int stages) {
     return DQK_OK;
 }
 
-template <int D>
+template <int D, int NS>
 dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk_dtype dtype, int batch,
                       const int *new_lens, const int *seq_before, int max_new, const int *page_table,
                       int max_pages, int early_release, cudaStream_t stream) {
     if (max_new <= kDirectMaxNew) {
-        prefer_max_shared(k_append_rows<D>);
+        prefer_max_shared(k_append_rows<D, NS>);
         const int groups = (max_new + kRowsPerCta - 1) / kRowsPerCta;
         const long long gx = (long long)batch * groups;
         if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
-        k_append_rows<D><<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
+        k_append_rows<D, NS><<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
             L->t_k, k, v, dtype, new_lens, seq_before, page_table, max_pages, groups,
             static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
         return launch_status();
     }
     const size_t smem = sizeof(AppendSmem<D>);
-    if (cudaFuncSetAttribute(k_quant_pack<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_quant_pack<D, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
         return DQK_ERR_CUDA;
     const int slots = (max_new + kPage - 1) / kPage + 1;
     const long long items = (long long)batch * slots;
@@ -277,7 +285,7 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
     long long gx = ((long long)sms + L->num_kv_heads - 1) / L->num_kv_heads;   // ~1 CTA per SM (fp64 T_K in smem)
     if (gx > items) gx = items;
     if (gx < 1) gx = 1;
-    k_quant_pack<D><<<dim3((unsigned)gx, L->num_kv_heads), 512, smem, stream>>>(
+    k_quant_pack<D, NS><<<dim3((unsigned)gx, L->num_kv_heads), 512, smem, stream>>>(
         L->t_k, k, v, dtype, batch, new_lens, seq_before, page_table, max_pages, slots,
         static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
     return launch_status();
@@ -290,7 +298,8 @@ extern "C" {
 size_t dqk_block_bytes(const dqk_layer_desc *layer) {
     if (!layer || (layer->head_dim != 64 && layer->head_dim != 128)) return 0;
     if (layer->v_ch0_protect != 0 && layer->v_ch0_protect != 1) return 0;
-    return (size_t)make_layout(layer->head_dim, layer->v_ch0_protect).bytes;
+    if (layer->group_size != kGroup && layer->group_size != layer->head_dim) return 0;
+    return (size_t)make_layout(layer->head_dim, layer->v_ch0_protect, layer->head_dim / layer->group_size).bytes;
 }
 
 }  // extern "C"
@@ -311,10 +320,16 @@ dqk_status check_append(const dqk_layer_desc *layer, const void *k, const void *
 dqk_status launch_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
                          const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
                          int max_pages, int early_release, cudaStream_t s) {
-    return layer->head_dim == 128 ? run_append<128>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new,
-                                                    page_table, max_pages, early_release, s)
-                                  : run_append<64>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new,
-                                                   page_table, max_pages, early_release, s);
+    const bool one = layer->group_size == layer->head_dim;   // one scale group per token
+    if (layer->head_dim == 128)
+        return one ? run_append<128, 1>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
+                                        max_pages, early_release, s)
+                   : run_append<128, 4>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
+                                        max_pages, early_release, s);
+    return one ? run_append<64, 1>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
+                                   max_pages, early_release, s)
+               : run_append<64, 2>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
+                                   max_pages, early_release, s);
 }
 }  // namespace
 

@@ -67,6 +67,7 @@ class Workload:
     ctx_lo: int = 4096
     ctx_hi: int = 65536
     v_ch0_protect: int = 0
+    group_size: int = 32         # channels per (scale, min) group: 32, or head_dim (one group per token)
 
     @property
     def group(self) -> int:
@@ -86,6 +87,8 @@ CONFIGS = {
     "qwen": Workload("qwen", batch=16, hq=32, hkv=8, d=128, ctx=None, seed=4,
                      k_dist="t3", outliers="none", rope_theta=1e6, append_new=64),
     "sweep": Workload("sweep", batch=16, hq=32, hkv=8, d=128, ctx=131072, seed=5),
+    # the 128K layer with one (scale, min) group per token (74 B per token and kv head)
+    "long128": Workload("long128", batch=4, hq=32, hkv=8, d=128, ctx=131072, seed=3, group_size=128),
     # the llama layer with structured queries and calibrated transforms (next-step row f1)
     "llama_cal": Workload("llama_cal", batch=8, hq=32, hkv=8, d=128, ctx=32768, seed=6,
                           transform="calibrated", q_dist="lowrank", page_order="random"),

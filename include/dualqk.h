@@ -64,7 +64,9 @@ typedef enum { DQK_F32 = 0, DQK_BF16 = 1 } dqk_dtype;
  *  num_q_heads    Hq; num_kv_heads Hkv; Hq % Hkv == 0 and G = Hq/Hkv in
  *                 {1, 2, 4, 8}.  Query head h reads kv head h / G.
  *  page_size      must be 16 tokens.
- *  group_size     must be 32 channels.
+ *  group_size     channels per (scale, min) group: 32, or head_dim for one
+ *                 group per token (74 B per token and kv head at d = 128,
+ *                 the compression "Results at 128K context" reports).
  *  v_ch0_protect  0: value channel 0 quantized like the others (default);
  *                 1: value channel 0 kept in BF16 as well.
  *  t_k, t_q       (device) fp32 [Hkv][d][d] row-major: k' = T_K k,
@@ -87,28 +89,30 @@ typedef struct {
 } dqk_layer_desc;
 
 /* Bytes of one (page, kv head) block: 16 tokens of INT2 codes, fp16
- * scale/min per 32-channel group for K and V, and the BF16 channel 0.
- * d = 128: 1568 (98 B per token and kv head), d = 64: 800 (50 B); +32 with
- * v_ch0_protect.  Returns 0 for an unsupported descriptor.
+ * scale/min per group for K and V, and the BF16 channel 0.  Groups of 32:
+ * d = 128: 1568 (98 B per token and kv head), d = 64: 800 (50 B); one group
+ * per token: 1184 (74 B) and 672 (42 B); +32 with v_ch0_protect.  Returns 0
+ * for an unsupported descriptor.
  *
- * Block layout (byte offsets, NG = d/32 groups, P = 16 tokens; the code
- * sections are in the operand order of the decode kernel's tensor-core
- * tiles, each lane of a warp reading 4*NG contiguous bytes):
+ * Block layout (byte offsets, NG = d/32 code blocks, NS = d/group_size scale
+ * groups, P = 16 tokens; the code sections are in the operand order of the
+ * decode kernel's tensor-core tiles, each lane of a warp reading 4*NG
+ * contiguous bytes):
  *   KC = 0            K codes, 4*d bytes: code of (token t, channel c) is in the
  *                     32-bit word at KC + 4*(lane*NG + W), bit 8*j + 2*f, with
  *                     g=c/32, cc=c%32, r=2*(cc/16)+t/8, lane=4*(t%8)+(cc%16)/4,
  *                     j=cc%4, W=r%NG, f=g+NG*(r/NG).
- *   KS = 4d           K scale fp16 [t][g]
- *   KM = KS + 32*NG   K min   fp16 [t][g]
- *   K0 = KM + 32*NG   K channel 0 BF16, token t at index 2*(t%8) + t/8
+ *   KS = 4d           K scale fp16 [t][g], g < NS
+ *   KM = KS + 32*NS   K min   fp16 [t][g]
+ *   K0 = KM + 32*NS   K channel 0 BF16, token t at index 2*(t%8) + t/8
  *   VC = K0 + 32      V codes, 4*d bytes: (t, c) is in the word at
  *                     VC + 4*(lane*NG + W), bit 16*e + 2*i, with m=c/16,
  *                     cr=(c%16)/8, tb=t/8, tig=(t%8)/2, e=t%2,
  *                     lane=4*(c%8)+tig; NG=4: W=cr+2*tb, i=m;
  *                     NG=2: q=(2m+cr)*2+tb, W=q/8, i=q%8.
- *   VS = VC + 4d      V scale fp16, (t, g) at index 2*(NG*(t/2) + g) + t%2
- *   VM = VS + 32*NG   V min fp16, same indexing
- *   V0 = VM + 32*NG   V channel 0 BF16 [t] (only with v_ch0_protect)
+ *   VS = VC + 4d      V scale fp16, (t, g) at index 2*(NS*(t/2) + g) + t%2
+ *   VM = VS + 32*NS   V min fp16, same indexing
+ *   V0 = VM + 32*NS   V channel 0 BF16 [t] (only with v_ch0_protect)
  * The code slot of a protected channel 0 holds 0.
  */
 size_t dqk_block_bytes(const dqk_layer_desc *layer);
@@ -128,7 +132,8 @@ size_t dqk_block_bytes(const dqk_layer_desc *layer);
  *                   be valid and not shared with another sequence being
  *                   appended in the same call.
  * Per token and kv head: k' = fp32(fp64 sum over i ascending of
- * T_K[c][i]*k[i]); per group g: scale = fp16((max-min)/3), min = fp16(min)
+ * T_K[c][i]*k[i]); per group g (group_size channels): scale =
+ * fp16((max-min)/3), min = fp16(min)
  * (fp64 arithmetic, RNE, saturating), code = clamp(rne((x-min)/scale), 0, 3)
  * or 0 when scale == 0; key channel 0 -> BF16, left out of group 0's range.
  * Values: same quantizer, no transform.  Positions of the touched pages that

@@ -148,19 +148,20 @@ void oracle_transform_f64(int d, const double *T, const double *x, double *y)
 
 /* x: d fp32 values (already transformed for keys).  protect_ch0: channel 0
  * is stored in BF16, left out of group 0's min/max, and its code slot is 0.
- * Per group g (channels 32g..32g+31):
+ * Per group g (channels gs*g .. gs*g + gs-1; gs = 32, or d for one group per
+ * token):
  *   mn, mx      = min / max over the group (fp32 values; a zero is +0)
  *   scale_h     = fp16( (mx - mn) / 3 )          (fp64 arithmetic)
  *   min_h       = fp16( mn )
  *   code_c      = 0 if scale_h == 0, else clamp(rne((x_c - min_h)/scale_h), 0, 3)
- * READING: fixed 32-channel groups aligned at channel 0; fp16 for scale and
- * min; round half to even; a zero scale gives code 0 (dequantizes to min). */
-void oracle_quantize_vec(int d, const float *x, int protect_ch0,
-                         uint8_t *codes, uint16_t *scale, uint16_t *minv, uint16_t *ch0)
+ * READING: fixed groups aligned at channel 0; fp16 for scale and min; round
+ * half to even; a zero scale gives code 0 (dequantizes to min). */
+void oracle_quantize_vec_g(int d, int gs, const float *x, int protect_ch0,
+                           uint8_t *codes, uint16_t *scale, uint16_t *minv, uint16_t *ch0)
 {
-    int ng = d / OR_GROUP;
+    int ng = d / gs;
     for (int g = 0; g < ng; ++g) {
-        int lo = g * OR_GROUP, hi = lo + OR_GROUP;
+        int lo = g * gs, hi = lo + gs;
         int first = (g == 0 && protect_ch0) ? 1 : 0;
         double mn = INFINITY, mx = -INFINITY;
         for (int c = lo + first; c < hi; ++c) {
@@ -185,12 +186,18 @@ void oracle_quantize_vec(int d, const float *x, int protect_ch0,
     if (ch0) *ch0 = protect_ch0 ? oracle_f32_to_bf16(x[0]) : 0;
 }
 
+void oracle_quantize_vec(int d, const float *x, int protect_ch0,
+                         uint8_t *codes, uint16_t *scale, uint16_t *minv, uint16_t *ch0)
+{
+    oracle_quantize_vec_g(d, OR_GROUP, x, protect_ch0, codes, scale, minv, ch0);
+}
+
 /* Dequantized channel value (fp64, exact from the stored fields). */
-static double dequant(int c, int protect_ch0, const uint8_t *codes, const uint16_t *scale,
+static double dequant(int c, int gs, int protect_ch0, const uint8_t *codes, const uint16_t *scale,
                       const uint16_t *minv, uint16_t ch0)
 {
     if (c == 0 && protect_ch0) return oracle_bf16_to_f64(ch0);
-    int g = c / OR_GROUP;
+    int g = c / gs;
     return oracle_f16_to_f64(minv[g]) + (double)codes[c] * oracle_f16_to_f64(scale[g]);
 }
 
@@ -205,27 +212,36 @@ static double dequant(int c, int protect_ch0, const uint8_t *codes, const uint16
  * Keys: channel 0 always protected.  Values: no transform; channel 0
  * protected only when v_ch0 != 0 (READING: the pages name channel-0
  * protection beside the key-side RoPE, so keys by default). */
-int oracle_append(int d, int hkv, int v_ch0, const float *t_k,
-                  const float *k, const float *v, long long n,
-                  uint8_t *kcodes, uint16_t *kscale, uint16_t *kmin, uint16_t *kch0,
-                  uint8_t *vcodes, uint16_t *vscale, uint16_t *vmin, uint16_t *vch0)
+int oracle_append_g(int d, int gs, int hkv, int v_ch0, const float *t_k,
+                    const float *k, const float *v, long long n,
+                    uint8_t *kcodes, uint16_t *kscale, uint16_t *kmin, uint16_t *kch0,
+                    uint8_t *vcodes, uint16_t *vscale, uint16_t *vmin, uint16_t *vch0)
 {
-    if (d % OR_GROUP || d <= 0 || hkv <= 0 || n < 0) return 1;
-    int ng = d / OR_GROUP;
+    if (gs <= 0 || d % gs || d <= 0 || hkv <= 0 || n < 0) return 1;
+    int ng = d / gs;
     float *kp = (float *)malloc(sizeof(float) * (size_t)d);
     if (!kp) return 2;
     for (long long t = 0; t < n; ++t) {
         for (int j = 0; j < hkv; ++j) {
             size_t row = (size_t)(t * hkv + j);
             oracle_transform_f32(d, t_k + (size_t)j * d * d, k + row * d, kp);
-            oracle_quantize_vec(d, kp, 1, kcodes + row * d, kscale + row * ng, kmin + row * ng,
-                                kch0 + row);
-            oracle_quantize_vec(d, v + row * d, v_ch0, vcodes + row * d, vscale + row * ng,
-                                vmin + row * ng, vch0 + row);
+            oracle_quantize_vec_g(d, gs, kp, 1, kcodes + row * d, kscale + row * ng, kmin + row * ng,
+                                  kch0 + row);
+            oracle_quantize_vec_g(d, gs, v + row * d, v_ch0, vcodes + row * d, vscale + row * ng,
+                                  vmin + row * ng, vch0 + row);
         }
     }
     free(kp);
     return 0;
+}
+
+int oracle_append(int d, int hkv, int v_ch0, const float *t_k,
+                  const float *k, const float *v, long long n,
+                  uint8_t *kcodes, uint16_t *kscale, uint16_t *kmin, uint16_t *kch0,
+                  uint8_t *vcodes, uint16_t *vscale, uint16_t *vmin, uint16_t *vch0)
+{
+    return oracle_append_g(d, OR_GROUP, hkv, v_ch0, t_k, k, v, n, kcodes, kscale, kmin, kch0, vcodes, vscale,
+                           vmin, vch0);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -283,7 +299,7 @@ void oracle_qprep(int d, const float *t_q_head, const float *q, int pct, float *
 /* ------------------------------------------------------------------------- */
 
 typedef struct {
-    int d, hq, hkv, v_ch0, pct, L;
+    int d, gs, hq, hkv, v_ch0, pct, L;
     const uint8_t *kcodes; const uint16_t *kscale, *kmin, *kch0;
     const uint8_t *vcodes; const uint16_t *vscale, *vmin, *vch0;
     const float *q, *t_q;
@@ -297,7 +313,7 @@ typedef struct {
  * o = sum_t p_t v^_t. */
 static void decode_head(seq_job *J, int h, double *s, double *qd, char *in_s, int16_t *sel)
 {
-    int d = J->d, ng = d / OR_GROUP, G = J->hq / J->hkv, j = h / G, L = J->L;
+    int d = J->d, gs = J->gs, ng = d / gs, G = J->hq / J->hkv, j = h / G, L = J->L;
     int nk = oracle_n_keep(d, J->pct);
     float *qp = (float *)malloc(sizeof(float) * (size_t)d);
     oracle_qprep(d, J->t_q + (size_t)j * d * d, J->q + (size_t)h * d, J->pct, qp, sel);
@@ -310,7 +326,7 @@ static void decode_head(seq_job *J, int h, double *s, double *qd, char *in_s, in
         double acc = 0.0;
         for (int c = 0; c < d; ++c) {
             if (!in_s[c]) continue;
-            acc += qd[c] * dequant(c, 1, J->kcodes + row * d, J->kscale + row * ng,
+            acc += qd[c] * dequant(c, gs, 1, J->kcodes + row * d, J->kscale + row * ng,
                                    J->kmin + row * ng, J->kch0[row]);
         }
         s[t] = acc * inv_sqrt_d;
@@ -324,7 +340,7 @@ static void decode_head(seq_job *J, int h, double *s, double *qd, char *in_s, in
         size_t row = (size_t)t * J->hkv + j;
         double p = s[t] / den;
         for (int c = 0; c < d; ++c)
-            o[c] += p * dequant(c, J->v_ch0, J->vcodes + row * d, J->vscale + row * ng,
+            o[c] += p * dequant(c, gs, J->v_ch0, J->vcodes + row * d, J->vscale + row * ng,
                                 J->vmin + row * ng, J->vch0[row]);
     }
     if (L == 0)
@@ -359,15 +375,15 @@ static void *seq_worker(void *arg)
  * hq query heads; query head h reads kv head h / (hq/hkv).
  * out [hq][d] fp64; sel [hq][n_keep] (nullable); qprime [hq][d] (nullable).
  * Work is spread over up to `threads` POSIX threads, one kv head at a time. */
-int oracle_decode_seq(int d, int hq, int hkv, int v_ch0, int pct, int L,
-                      const uint8_t *kcodes, const uint16_t *kscale, const uint16_t *kmin,
-                      const uint16_t *kch0, const uint8_t *vcodes, const uint16_t *vscale,
-                      const uint16_t *vmin, const uint16_t *vch0,
-                      const float *q, const float *t_q, double *out, int16_t *sel,
-                      float *qprime, int threads)
+int oracle_decode_seq_g(int d, int gs, int hq, int hkv, int v_ch0, int pct, int L,
+                        const uint8_t *kcodes, const uint16_t *kscale, const uint16_t *kmin,
+                        const uint16_t *kch0, const uint8_t *vcodes, const uint16_t *vscale,
+                        const uint16_t *vmin, const uint16_t *vch0,
+                        const float *q, const float *t_q, double *out, int16_t *sel,
+                        float *qprime, int threads)
 {
-    if (d % OR_GROUP || hkv <= 0 || hq % hkv || pct < 0 || pct > 99 || L < 0) return 1;
-    seq_job J = {d, hq, hkv, v_ch0, pct, L, kcodes, kscale, kmin, kch0, vcodes, vscale, vmin,
+    if (gs <= 0 || d % gs || hkv <= 0 || hq % hkv || pct < 0 || pct > 99 || L < 0) return 1;
+    seq_job J = {d, gs, hq, hkv, v_ch0, pct, L, kcodes, kscale, kmin, kch0, vcodes, vscale, vmin,
                  vch0, q, t_q, out, sel, qprime, 0, PTHREAD_MUTEX_INITIALIZER};
     if (threads < 1) threads = 1;
     if (threads > hkv) threads = hkv;
@@ -380,6 +396,17 @@ int oracle_decode_seq(int d, int hq, int hkv, int v_ch0, int pct, int L,
     free(tid);
     pthread_mutex_destroy(&J.mu);
     return 0;
+}
+
+int oracle_decode_seq(int d, int hq, int hkv, int v_ch0, int pct, int L,
+                      const uint8_t *kcodes, const uint16_t *kscale, const uint16_t *kmin,
+                      const uint16_t *kch0, const uint8_t *vcodes, const uint16_t *vscale,
+                      const uint16_t *vmin, const uint16_t *vch0,
+                      const float *q, const float *t_q, double *out, int16_t *sel,
+                      float *qprime, int threads)
+{
+    return oracle_decode_seq_g(d, OR_GROUP, hq, hkv, v_ch0, pct, L, kcodes, kscale, kmin, kch0, vcodes, vscale,
+                               vmin, vch0, q, t_q, out, sel, qprime, threads);
 }
 
 /* ------------------------------------------------------------------------- */

@@ -58,6 +58,12 @@ def lib():
         _lib.oracle_decode_seq.argtypes = [C.c_int] * 6 + [P] * 10 + [P, P, P, C.c_int]
         _lib.oracle_decode_dense.restype = C.c_int
         _lib.oracle_decode_dense.argtypes = [C.c_int] * 5 + [P] * 7
+        _lib.oracle_quantize_vec_g.argtypes = [C.c_int, C.c_int, P, C.c_int, P, P, P, P]
+        _lib.oracle_append_g.restype = C.c_int
+        _lib.oracle_append_g.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, C.c_longlong,
+                                         P, P, P, P, P, P, P, P]
+        _lib.oracle_decode_seq_g.restype = C.c_int
+        _lib.oracle_decode_seq_g.argtypes = [C.c_int] * 7 + [P] * 10 + [P, P, P, C.c_int]
         _lib.oracle_calibrate.restype = C.c_int
         _lib.oracle_calibrate.argtypes = [C.c_int, C.c_longlong, C.c_longlong, C.c_double, P, P, P, P]
     return _lib
@@ -104,14 +110,15 @@ def transform_f32(t: np.ndarray, x: np.ndarray) -> np.ndarray:
     return y
 
 
-def quantize_vec(x: np.ndarray, protect_ch0: bool):
+def quantize_vec(x: np.ndarray, protect_ch0: bool, gs: int = GROUP):
+    """One token vector: codes, fp16 scale/min per group of gs channels, BF16 ch0."""
     x = _f32(x)
     d = x.shape[0]
     codes = np.empty(d, dtype=np.uint8)
-    scale = np.empty(d // GROUP, dtype=np.uint16)
-    mn = np.empty(d // GROUP, dtype=np.uint16)
+    scale = np.empty(d // gs, dtype=np.uint16)
+    mn = np.empty(d // gs, dtype=np.uint16)
     ch0 = np.zeros(1, dtype=np.uint16)
-    lib().oracle_quantize_vec(d, _p(x), int(protect_ch0), _p(codes), _p(scale), _p(mn), _p(ch0))
+    lib().oracle_quantize_vec_g(d, gs, _p(x), int(protect_ch0), _p(codes), _p(scale), _p(mn), _p(ch0))
     return codes, scale, mn, int(ch0[0])
 
 
@@ -141,19 +148,20 @@ class Cache(dict):
     kscale/kmin/vscale/vmin [n][hkv][d/32] fp16 bits, kch0/vch0 [n][hkv]."""
 
 
-def append(t_k: np.ndarray, k: np.ndarray, v: np.ndarray, v_ch0: bool = False) -> Cache:
-    """Transform and quantize rows k, v [n][hkv][d] (fp32 values)."""
+def append(t_k: np.ndarray, k: np.ndarray, v: np.ndarray, v_ch0: bool = False, gs: int = GROUP) -> Cache:
+    """Transform and quantize rows k, v [n][hkv][d] (fp32 values); scale groups
+    of gs channels (32, or d for one group per token)."""
     t_k, k, v = _f32(t_k), _f32(k), _f32(v)
     n, hkv, d = k.shape
-    ng = d // GROUP
+    ng = d // gs
     c = Cache(
         kcodes=np.empty((n, hkv, d), np.uint8), kscale=np.empty((n, hkv, ng), np.uint16),
         kmin=np.empty((n, hkv, ng), np.uint16), kch0=np.empty((n, hkv), np.uint16),
         vcodes=np.empty((n, hkv, d), np.uint8), vscale=np.empty((n, hkv, ng), np.uint16),
         vmin=np.empty((n, hkv, ng), np.uint16), vch0=np.empty((n, hkv), np.uint16))
-    rc = lib().oracle_append(d, hkv, int(v_ch0), _p(t_k), _p(k), _p(v), n,
-                             _p(c["kcodes"]), _p(c["kscale"]), _p(c["kmin"]), _p(c["kch0"]),
-                             _p(c["vcodes"]), _p(c["vscale"]), _p(c["vmin"]), _p(c["vch0"]))
+    rc = lib().oracle_append_g(d, gs, hkv, int(v_ch0), _p(t_k), _p(k), _p(v), n,
+                               _p(c["kcodes"]), _p(c["kscale"]), _p(c["kmin"]), _p(c["kch0"]),
+                               _p(c["vcodes"]), _p(c["vscale"]), _p(c["vmin"]), _p(c["vch0"]))
     if rc:
         raise ValueError(f"oracle_append failed ({rc})")
     return c
@@ -176,7 +184,8 @@ def decode_seq(cache: Cache, q: np.ndarray, t_q: np.ndarray, hq: int, pct: int,
     sel = np.empty((hq, keep), np.int16)
     qp = np.empty((hq, d), np.float32)
     cc = {k: np.ascontiguousarray(a) for k, a in cache.items()}
-    rc = lib().oracle_decode_seq(d, hq, hkv, int(v_ch0), pct, L,
+    gs = d // cache["kscale"].shape[2]          # scale-group size the cache was built with
+    rc = lib().oracle_decode_seq_g(d, gs, hq, hkv, int(v_ch0), pct, L,
                                  _p(cc["kcodes"]), _p(cc["kscale"]), _p(cc["kmin"]), _p(cc["kch0"]),
                                  _p(cc["vcodes"]), _p(cc["vscale"]), _p(cc["vmin"]), _p(cc["vch0"]),
                                  _p(q), _p(t_q), _p(out), _p(sel), _p(qp), threads)
@@ -204,7 +213,7 @@ def dequant(cache: Cache, v_ch0: bool = False):
     n, hkv, d = cache["kcodes"].shape
     f16 = np.vectorize(f16_bits_to_f64, otypes=[np.float64])
     bf = np.vectorize(bf16_bits_to_f64, otypes=[np.float64])
-    grp = np.arange(d) // GROUP
+    grp = np.arange(d) // (d // cache["kscale"].shape[2])
     out = []
     for pre, prot in (("k", True), ("v", v_ch0)):
         s = f16(cache[pre + "scale"])[..., grp]

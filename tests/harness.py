@@ -62,12 +62,13 @@ class DeviceRun:
         self.tk_host, self.tq_host = tk, tq
         self.t_k = torch.from_numpy(tk).to(self.dev)
         self.t_q = torch.from_numpy(tq).to(self.dev)
-        probe = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, 0, 1, v_ch0_protect=w.v_ch0_protect)
+        probe = Q.layer_desc(w.d, w.hq, w.hkv, 0, 0, 0, 1, v_ch0_protect=w.v_ch0_protect,
+                             group_size=w.group_size)
         self.block_bytes = Q.dqk_block_bytes(probe)
         self.pool = torch.full((self.num_pages * w.hkv * self.block_bytes,), fill, dtype=torch.uint8,
                                device=self.dev)
         self.desc = Q.layer_desc(w.d, w.hq, w.hkv, self.t_k, self.t_q, self.pool, self.num_pages,
-                                 v_ch0_protect=w.v_ch0_protect)
+                                 v_ch0_protect=w.v_ch0_protect, group_size=w.group_size)
         self.table_dev = torch.from_numpy(self.table).to(self.dev)
         self.cached = np.zeros(w.batch, dtype=np.int32)      # tokens appended so far
         self.ws_bytes = Q.dqk_decode_workspace_size(self.desc, w.batch, self.max_pages)
@@ -136,8 +137,8 @@ class DeviceRun:
 # ---------------------------------------------------------------------------
 # layout decoder, written from the block layout documented in dualqk.h
 # ---------------------------------------------------------------------------
-def _layout(d, v_ch0):
-    ng = d // 32
+def _layout(d, v_ch0, gs=32):
+    ng = d // gs                     # scale groups per token
     kc = 0
     ks = 4 * d
     km = ks + 32 * ng
@@ -177,9 +178,9 @@ def _code_tables(d):
     return kw, kb, vw, vb
 
 
-def decode_pool(pool: np.ndarray, table_row: np.ndarray, L: int, d: int, v_ch0: int) -> O.Cache:
+def decode_pool(pool: np.ndarray, table_row: np.ndarray, L: int, d: int, v_ch0: int, gs: int = 32) -> O.Cache:
     """Plain arrays (same form as oracle.append) of tokens 0..L-1 of one sequence."""
-    lay = _layout(d, v_ch0)
+    lay = _layout(d, v_ch0, gs)
     ng = lay["ng"]
     hkv = pool.shape[1]
     t = np.arange(L)
@@ -217,7 +218,8 @@ def oracle_cache(w: I.Workload, b: int, L: int, heads=None) -> O.Cache:
     k, v = I.kv_rows(w, b, 0, L)
     if heads is not None:
         k, v, tk = k[:, heads], v[:, heads], tk[heads]
-    return O.append(tk, np.ascontiguousarray(k), np.ascontiguousarray(v), v_ch0=bool(w.v_ch0_protect))
+    return O.append(tk, np.ascontiguousarray(k), np.ascontiguousarray(v), v_ch0=bool(w.v_ch0_protect),
+                    gs=w.group_size)
 
 
 def oracle_reference(w: I.Workload, run: DeviceRun, pct: int | None = None, lens=None) -> dict:
@@ -244,7 +246,7 @@ def assert_cache_matches_oracle(run: DeviceRun, ref: dict):
         L = int(ref["lens"][b])
         if L == 0:
             continue
-        got = decode_pool(pool, run.table[b], L, w.d, w.v_ch0_protect)
+        got = decode_pool(pool, run.table[b], L, w.d, w.v_ch0_protect, w.group_size)
         exp = ref["caches"][b]
         for key in ("kcodes", "kscale", "kmin", "kch0", "vcodes", "vscale", "vmin", "vch0"):
             e = exp[key][:L]

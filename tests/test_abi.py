@@ -51,7 +51,27 @@ def test_compression_ratio_vs_bf16(Q):
     assert abs(2 * 2 * 128 / per_token - 5.224) < 1e-3       # K+V BF16 = 512 B
 
 
+@pytest.mark.parametrize("d,vch0,bytes_", [(128, 0, 1184), (64, 0, 672), (128, 1, 1216)])
+def test_one_group_per_token_bytes(Q, d, vch0, bytes_):
+    """group_size = head_dim: one fp16 (scale, min) per token for K and for V."""
+    per_token = d // 4 + d // 4 + 2 * 4 + 2 + 2 * vch0
+    desc = Q.layer_desc(d, 8, 2, 0, 0, 0, 1, v_ch0_protect=vch0, group_size=d)
+    assert Q.dqk_block_bytes(desc) == 16 * per_token == bytes_
+
+
+def test_one_group_compression_matches_the_pages(Q):
+    """74 B per token and kv head at d = 128: 512/74 = 6.92x against BF16 K+V
+    (the 6.8x of "Results at 128K context"); dropping 40 % of the key codes
+    from reads leaves 74 - 0.4 * 31.75 = 61.3 B, 8.35x (the estimated 8.3x)."""
+    desc = Q.layer_desc(128, 32, 8, 0, 0, 0, 1, group_size=128)
+    per_token = Q.dqk_block_bytes(desc) / 16
+    assert per_token == 74
+    assert abs(512 / per_token - 6.92) < 0.01
+    assert abs(512 / (per_token - 0.4 * 127 / 4) - 8.35) < 0.01
+
+
 def test_unsupported_layers(Q):
+    assert Q.dqk_block_bytes(Q.layer_desc(128, 8, 2, 0, 0, 0, 1, group_size=64)) == 0
     assert Q.dqk_block_bytes(Q.layer_desc(96, 8, 2, 0, 0, 0, 1)) == 0
     assert Q.dqk_decode_workspace_size(Q.layer_desc(128, 24, 8, 0, 0, 1, 1), 1, 4) == 0   # G = 3
     assert Q.dqk_decode_workspace_size(Q.layer_desc(128, 32, 8, 0, 0, 0, 1), 1, 4) == 0   # no pool

@@ -37,6 +37,10 @@ CASES = {
     "g1-d128": small("llama", batch=2, hq=4, hkv=4, ctx=257),
     "g2-d64": small("llama", batch=2, hq=8, hkv=4, d=64, ctx=500),
     "g8": small("llama", batch=2, hq=16, hkv=2, ctx=600),
+    # one (scale, min) group per token (74 B per token and kv head), ragged, random pages
+    "g128": small("llama", batch=4, ctx=None, ctx_lo=1, ctx_hi=700, page_order="random", group_size=128),
+    "g128-vch0": small("llama", batch=2, ctx=333, v_ch0_protect=1, group_size=128),
+    "g64-d64": small("llama", batch=2, hq=8, hkv=4, d=64, ctx=500, group_size=64),
     # calibrated transform pair and structured queries (next-step row f1)
     "calibrated": small("llama_cal", batch=2, ctx=None, ctx_lo=300, ctx_hi=900),
 }
@@ -133,7 +137,7 @@ def _sampled_units(w, run, out, sel, units):
     for b, j in units:
         L = int(run.lens[b])
         cache = H.oracle_cache(w, b, L, heads=[j])
-        got = H.decode_pool(run.pool_host()[:, j:j + 1], run.table[b], L, w.d, w.v_ch0_protect)
+        got = H.decode_pool(run.pool_host()[:, j:j + 1], run.table[b], L, w.d, w.v_ch0_protect, w.group_size)
         for key in ("kcodes", "kscale", "kmin", "kch0", "vcodes", "vscale", "vmin"):
             assert np.array_equal(got[key], cache[key]), (b, j, key)
         o, s, _ = O.decode_seq(cache, run.q_host[b, j * G:(j + 1) * G], tq[j:j + 1], G, w.pct, L=L)
@@ -144,6 +148,7 @@ def _sampled_units(w, run, out, sel, units):
 @pytest.mark.slow
 @pytest.mark.parametrize("name,units", [("llama", [(0, 0), (7, 5)]),
                                         ("long", [(1, 3), (3, 7)]),
+                                        ("long128", [(0, 2), (2, 5)]),
                                         ("qwen", [(2, 1), (15, 6)])])
 def test_full_size_configs_sampled(name, units):
     w = I.CONFIGS[name]

@@ -322,3 +322,58 @@ def test_append_is_per_row_transform_then_quantize(oracle_mod):
             assert np.array_equal(c["kcodes"][t, j], codes) and c["kch0"][t, j] == ch0
             codes, s, m, _ = oracle_mod.quantize_vec(v[t, j], False)
             assert np.array_equal(c["vcodes"][t, j], codes) and np.array_equal(c["vscale"][t, j], s)
+
+
+# ------------------------------------------------- one (scale, min) group per token
+def test_one_group_grid_round_trip(oracle_mod):
+    """group_size = d: values on one INT2 grid over the whole row (channel 0
+    protected or not) come back with the same codes, scale and min."""
+    rng = np.random.default_rng(21)
+    for trial in range(200):
+        d = 128 if trial % 2 else 64
+        scale = 2.0 ** int(rng.integers(-6, 4))
+        mn = float(_f16(rng.standard_normal() * 4))
+        codes = rng.integers(0, 4, size=d).astype(np.uint8)
+        protect = bool(trial % 3 == 0)
+        codes[1], codes[2] = 0, 3
+        x = (mn + codes * scale).astype(np.float32)
+        if protect:
+            x[0] = np.float32(rng.standard_normal() * 50)
+            codes[0] = 0
+        c2, s2, m2, ch0 = oracle_mod.quantize_vec(x, protect, gs=d)
+        assert s2.shape == (1,) and m2.shape == (1,)
+        assert np.array_equal(c2, codes)
+        assert s2[0] == np.float16(scale).view(np.uint16) and m2[0] == np.float16(mn).view(np.uint16)
+
+
+def test_one_group_equals_per_group_when_ranges_agree(oracle_mod):
+    """When every 32-channel group spans the same [min, max], the per-group and
+    the per-token quantizers must give the same codes, scales and mins."""
+    rng = np.random.default_rng(22)
+    for trial in range(100):
+        d = 128
+        x = rng.uniform(-1.0, 1.0, size=d).astype(np.float32)
+        lo, hi = np.float32(-1.5), np.float32(2.25)
+        for g in range(4):
+            x[32 * g + 3], x[32 * g + 17] = lo, hi
+        protect = bool(trial % 2)
+        c32, s32, m32, ch32 = oracle_mod.quantize_vec(x, protect)
+        c1, s1, m1, ch1 = oracle_mod.quantize_vec(x, protect, gs=d)
+        assert np.array_equal(c32, c1) and ch32 == ch1
+        assert np.all(s32 == s1[0]) and np.all(m32 == m1[0])
+
+
+def test_one_group_decode_is_attention_over_dequantized_cache(oracle_mod):
+    rng = np.random.default_rng(23)
+    L, hkv, d = 40, 2, 128
+    k = rng.standard_normal((L, hkv, d)).astype(np.float32)
+    v = rng.standard_normal((L, hkv, d)).astype(np.float32)
+    eye = np.broadcast_to(np.eye(d, dtype=np.float32), (hkv, d, d)).copy()
+    cache = oracle_mod.append(eye, k, v, gs=d)
+    assert cache["kscale"].shape == (L, hkv, 1)
+    q = rng.standard_normal((4, d)).astype(np.float32)
+    out, sel, qp = oracle_mod.decode_seq(cache, q, eye, hq=4, pct=0)
+    kh, vh = oracle_mod.dequant(cache)
+    for h in range(4):
+        ref = textbook_attention(qp[h:h + 1].astype(np.float64), kh[:, h // 2], vh[:, h // 2], 1 / math.sqrt(d))[0]
+        assert np.max(np.abs(out[h] - ref)) <= 1e-12
