@@ -60,15 +60,16 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.NG = P.d / kGroup;
     const int hkv = L->num_kv_heads;
     const int warps = attend_warps(P.G), stage_blocks = attend_stage_blocks(P.G);
-    if (hkv <= warps) {
-        if (warps % hkv) return false;
-        P.hc = hkv;
-    } else {
-        if (hkv % warps) return false;
-        P.hc = warps;
-    }
+    // kv heads per chunk: the largest divisor of Hkv that divides the warp count
+    P.hc = 0;
+    for (int c = std::min(hkv, warps); c >= 1; --c)
+        if (hkv % c == 0 && warps % c == 0) {
+            P.hc = c;
+            break;
+        }
+    if (P.hc == 0) return false;
     P.pps = stage_blocks / P.hc;    // pages per stage
-    P.pw = warps / P.hc;            // warps per kv head (each takes 2 pages of a stage)
+    P.pw = warps / P.hc;            // warps per kv head (each takes attend_pages_per_warp pages of a stage)
     P.nchunks = hkv / P.hc;
     if ((long long)batch * P.nchunks * (L->num_pages + 1) >= (1LL << 31)) return false;
     // Records are sized for kMaxAttendCtas so the workspace size does not depend
