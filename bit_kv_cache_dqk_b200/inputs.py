@@ -320,7 +320,7 @@ def _raw_queries(w: Workload, rng, rows: int) -> np.ndarray:
     if w.q_dist == "lowrank":
         basis = _query_basis(w)
         z = rng.standard_normal((rows, w.hq, _QRANK)) * _QSCALES[None, None, :]
-        q = np.einsum("jdr,nhr->nhd", basis[np.arange(w.hq) // w.group], z)
+        q = np.einsum("hdr,nhr->nhd", basis[np.arange(w.hq) // w.group], z)   # head h near its kv head's subspace
         q += 0.25 * rng.standard_normal((rows, w.hq, w.d))
         return q.astype(np.float32)
     return rng.standard_normal((rows, w.hq, w.d)).astype(np.float32)
