@@ -824,10 +824,15 @@ constexpr int kCombineThreads = 256;
 // running max moves from chunk to chunk with an exact rescale.  Maxima and
 // denominators are reduced in a fixed order, so the result does not depend on
 // scheduling.
+//
+// partial_out: instead of the normalized output, the merged record itself --
+// (m, l, o[D]) per (sequence, query head), m in log2 units -- for a later merge
+// with the records of other context ranges (dqk_merge_partials).
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restrict__ seq_lens, int batch, int hq,
                                                              int hkv, int hc, int pw, int nchunks, int num_ctas,
-                                                             const float *__restrict__ part, float *__restrict__ out) {
+                                                             const float *__restrict__ part, float *__restrict__ out,
+                                                             int partial_out) {
     constexpr int kSlices = kCombineThreads / D;
     constexpr int kPer = kCombineChunk / kSlices;   // records of a chunk per thread
     constexpr int kWarps = kCombineThreads / 32;
@@ -882,8 +887,19 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restri
     index_chunk(0);
     __syncthreads();
     grid_dependency_wait();     // partial records come from k_attend
+    float *pr = out + ((size_t)b * hq + h) * (D + 2);   // partial record of (b, h)
     if (np == 0) {
-        if (slice == 0) o[ch] = 0.0f;
+        if (slice == 0) {
+            if (partial_out) {
+                pr[2 + ch] = 0.0f;
+                if (ch == 0) {
+                    pr[0] = -INFINITY;
+                    pr[1] = 0.0f;
+                }
+            } else {
+                o[ch] = 0.0f;
+            }
+        }
         return;
     }
     float mrun = -INFINITY, acc = 0.0f, dsum = 0.0f;
@@ -947,8 +963,41 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restri
         float num = 0.0f;
 #pragma unroll
         for (int k = 0; k < kSlices; ++k) num += sh_acc[k][ch];
-        o[ch] = dsum > 0.0f ? num / dsum : 0.0f;
+        if (partial_out) {
+            pr[2 + ch] = num;
+            if (ch == 0) {
+                pr[0] = mrun;
+                pr[1] = dsum;
+            }
+        } else {
+            o[ch] = dsum > 0.0f ? num / dsum : 0.0f;
+        }
     }
+}
+
+// ---------------------------------------------------------------------------
+// merge of partial records from n context ranges (one CTA per (sequence,
+// query head), one thread per channel): out = sum_r 2^(m_r - M) o_r /
+// sum_r 2^(m_r - M) l_r with M = max_r m_r, ranges taken in index order.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(D) k_merge(const float *__restrict__ parts, int n, long long rows,
+                                            float *__restrict__ out) {
+    const long long row = blockIdx.x;
+    const int c = threadIdx.x;
+    float M = -INFINITY;
+    for (int r = 0; r < n; ++r) M = fmaxf(M, parts[((size_t)r * rows + row) * (D + 2)]);
+    float num = 0.0f, den = 0.0f;
+    if (M != -INFINITY) {
+        for (int r = 0; r < n; ++r) {
+            const float *pr = parts + ((size_t)r * rows + row) * (D + 2);
+            if (pr[0] == -INFINITY) continue;
+            const float w = exp2f(pr[0] - M);
+            den = fmaf(w, pr[1], den);
+            num = fmaf(w, pr[2 + c], num);
+        }
+    }
+    out[row * D + c] = den > 0.0f ? num / den : 0.0f;
 }
 
 }  // namespace dqk

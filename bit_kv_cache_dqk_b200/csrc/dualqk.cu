@@ -113,6 +113,7 @@ struct DecodeArgs {
     void *ws;
     size_t ws_bytes;
     cudaStream_t stream;
+    bool partial = false;      // the combine writes (m, l, o) records instead of outputs
 };
 
 dqk_status check_decode(const DecodeArgs &a, DecodePlan &P) {
@@ -235,7 +236,7 @@ dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
     return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(kCombineThreads), 0, a.stream, a.seq_lens,
                       a.batch,
                       a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pw, P.nchunks, P.num_ctas,
-                      reinterpret_cast<const float *>(ws + P.off_part), a.out);
+                      reinterpret_cast<const float *>(ws + P.off_part), a.out, (int)a.partial);
 }
 
 enum Stage { kPrepare = 1, kAttend = 2, kCombine = 4 };
@@ -387,6 +388,27 @@ dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const voi
     }
     return decode_stages(a, kPrepare | kAttend | kCombine);
 }
+dqk_status dqk_decode_partial(DQK_DECODE_ARGS) {
+    DQK_DECODE_PACK;
+    a.partial = true;
+    return decode_stages(a, kPrepare | kAttend | kCombine);
+}
+
+dqk_status dqk_merge_partials(const float *parts, int n_parts, int batch, int num_q_heads, int head_dim,
+                              float *out, dqk_stream_t stream) {
+    if (!parts || !out || n_parts <= 0 || batch <= 0 || num_q_heads <= 0) return DQK_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return DQK_ERR_UNSUPPORTED;
+    if (!aligned(parts, 4) || !aligned(out, 4)) return DQK_ERR_INVALID_ARG;
+    const long long rows = (long long)batch * num_q_heads;
+    if (rows > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (head_dim == 128)
+        k_merge<128><<<(unsigned)rows, 128, 0, s>>>(parts, n_parts, rows, out);
+    else
+        k_merge<64><<<(unsigned)rows, 64, 0, s>>>(parts, n_parts, rows, out);
+    return launch_status();
+}
+
 dqk_status dqk_decode_prepare(DQK_DECODE_ARGS) {
     DQK_DECODE_PACK;
     return decode_stages(a, kPrepare);

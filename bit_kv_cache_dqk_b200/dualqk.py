@@ -24,7 +24,7 @@ DQK_ERR_CUDA, DQK_ERR_DEVICE_BOUNDS, DQK_ERR_TIMEOUT = 4, 5, 6
 DQK_F32, DQK_BF16 = 0, 1
 
 EXPORTED = ["dqk_block_bytes", "dqk_append", "dqk_decode_workspace_size", "dqk_decode",
-            "dqk_decode_step", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine",
+            "dqk_decode_step", "dqk_decode_partial", "dqk_merge_partials", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine",
             "dqk_decode_noalloc", "dqk_bf16_block_bytes", "dqk_bf16_append",
             "dqk_bf16_decode_workspace_size", "dqk_bf16_decode", "dqk_last_device_error", "dqk_status_string"]
 
@@ -46,10 +46,12 @@ _lib.dqk_append.restype = C.c_int
 _lib.dqk_append.argtypes = [_D, _P, _P, C.c_int, C.c_int, _P, _P, C.c_int, _P, C.c_int, _P]
 _lib.dqk_decode_workspace_size.restype = C.c_size_t
 _lib.dqk_decode_workspace_size.argtypes = [_D, C.c_int, C.c_int]
-for _n in ("dqk_decode", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine"):
+for _n in ("dqk_decode", "dqk_decode_partial", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine"):
     getattr(_lib, _n).restype = C.c_int
     getattr(_lib, _n).argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P,
                                   C.c_size_t, _P]
+_lib.dqk_merge_partials.restype = C.c_int
+_lib.dqk_merge_partials.argtypes = [_P, C.c_int, C.c_int, C.c_int, C.c_int, _P, _P]
 _lib.dqk_decode_step.restype = C.c_int
 _lib.dqk_decode_step.argtypes = [_D, _P, _P, C.c_int, _P, _P, C.c_int, _P, C.c_int, C.c_int, _P, _P, C.c_int,
                                  C.c_int, _P, _P, _P, C.c_size_t, _P]
@@ -140,6 +142,17 @@ def dqk_decode_step(layer, k, v, kv_dtype, new_lens, seq_lens_before, max_new, q
                               _addr(page_table), max_pages, sparsity_pct, _addr(out), _addr(sel_out),
                               _addr(workspace), workspace_bytes, _stream(stream))
     return _check(st, "dqk_decode_step", raise_on_error)
+
+
+def dqk_decode_partial(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, part, sel_out,
+                       workspace, workspace_bytes, stream=None, raise_on_error=True) -> int:
+    return _decode(_lib.dqk_decode_partial, "dqk_decode_partial", layer, q, q_dtype, batch, seq_lens, page_table,
+                   max_pages, sparsity_pct, part, sel_out, workspace, workspace_bytes, stream, raise_on_error)
+
+
+def dqk_merge_partials(parts, n_parts, batch, num_q_heads, head_dim, out, stream=None, raise_on_error=True) -> int:
+    st = _lib.dqk_merge_partials(_addr(parts), n_parts, batch, num_q_heads, head_dim, _addr(out), _stream(stream))
+    return _check(st, "dqk_merge_partials", raise_on_error)
 
 
 def dqk_decode_prepare(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out,

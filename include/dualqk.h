@@ -194,6 +194,31 @@ dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const voi
                            int sparsity_pct, float *out, int16_t *sel_out, void *workspace,
                            size_t workspace_bytes, dqk_stream_t stream);
 
+/* Context-parallel decode (one sequence's pages spread over several GPUs):
+ * each rank decodes the pages it holds with dqk_decode_partial, the ranks
+ * exchange their records (an all-gather over NCCL), and dqk_merge_partials
+ * forms the output.  Passage: the split-K combine of the decode path, taken
+ * across ranks; the pages' attention is over the whole context.
+ *
+ * dqk_decode_partial -- dqk_decode over the cached tokens this caller holds
+ * (its own pool, page table and token counts seq_lens), writing instead of
+ * `out` one record per (sequence, query head): part [batch][Hq][2 + d] fp32 =
+ * (m, l, o[d]) with m the running max of the scores in log2 units (scores
+ * scaled by log2(e)/sqrt(d)), l = sum of 2^(s - m), o = sum of 2^(s - m) v^.
+ * A sequence with no tokens here gives (-inf, 0, 0...).  Same arguments as
+ * dqk_decode otherwise; all ranks must use the same q and sparsity_pct. */
+dqk_status dqk_decode_partial(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
+                              int batch, const int *seq_lens, const int *page_table,
+                              int max_pages, int sparsity_pct, float *part, int16_t *sel_out,
+                              void *workspace, size_t workspace_bytes, dqk_stream_t stream);
+
+/* out[b][h] = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r over the n_parts
+ * records parts [n_parts][batch][Hq][2 + d] (device, fp32), M = max_r m_r,
+ * records taken in index order (the same result on every rank); 0 where no
+ * range held tokens.  out (device) fp32 [batch][Hq][d]. */
+dqk_status dqk_merge_partials(const float *parts, int n_parts, int batch, int num_q_heads,
+                              int head_dim, float *out, dqk_stream_t stream);
+
 /* The three stages of dqk_decode, exported so callers can place or time them
  * separately.  Same arguments; each uses the ones its stage needs. */
 dqk_status dqk_decode_prepare(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,

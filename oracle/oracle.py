@@ -194,6 +194,53 @@ def decode_seq(cache: Cache, q: np.ndarray, t_q: np.ndarray, hq: int, pct: int,
     return out, sel, qp
 
 
+LOG2E = 1.4426950408889634
+
+
+def decode_partial(cache: Cache, q: np.ndarray, t_q: np.ndarray, hq: int, pct: int,
+                   v_ch0: bool = False, t0: int = 0, t1: int | None = None) -> np.ndarray:
+    """Unnormalized attention record of the rows [t0, t1) of one sequence (the
+    split-K combine of the decode path, taken over a row range): for each
+    query head, with s_t the pruned score of row t (q'_sel . k^'_sel / sqrt(d))
+    written in log2 units u_t = s_t log2(e),
+        m = max_t u_t,   l = sum_t 2^(u_t - m),   o = sum_t 2^(u_t - m) v^_t.
+    Returns rec [hq][2 + d] fp64 = (m, l, o); (-inf, 0, 0) for an empty range.
+    Softmax over the union of ranges is then the merge below."""
+    n, hkv, d = cache["kcodes"].shape
+    t1 = n if t1 is None else t1
+    g = hq // hkv
+    rec = np.zeros((hq, 2 + d))
+    rec[:, 0] = -np.inf
+    if t1 <= t0:
+        return rec
+    part = Cache({k: a[t0:t1] for k, a in cache.items()})
+    kd, vd = dequant(part, v_ch0)
+    for h in range(hq):
+        j = h // g
+        qp, sel = qprep(np.asarray(t_q)[j], np.asarray(q)[h], pct)
+        sel = sel.astype(np.int64)
+        u = (kd[:, j, sel] @ qp[sel].astype(np.float64)) / np.sqrt(d) * LOG2E
+        m = u.max()
+        p = np.exp2(u - m)
+        rec[h, 0], rec[h, 1] = m, p.sum()
+        rec[h, 2:] = p @ vd[:, j, :]
+    return rec
+
+
+def merge_partials(recs: np.ndarray) -> np.ndarray:
+    """Output of attention over the union of the ranges of the records recs
+    [n][..][2 + d]: sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r, M = max_r m_r;
+    0 where no range held a row."""
+    recs = np.asarray(recs, np.float64)
+    m = recs[..., 0]
+    top = m.max(axis=0)
+    safe = np.where(np.isfinite(top), top, 0.0)
+    wgt = np.where(np.isfinite(m), np.exp2(m - safe[None]), 0.0)
+    den = (wgt * recs[..., 1]).sum(axis=0)
+    num = (wgt[..., None] * recs[..., 2:]).sum(axis=0)
+    return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
+
+
 def decode_dense(t_k64, t_q64, k, v, q, pct: int, want_scores: bool = False):
     """Quantization-off attention, fp64 throughout.  k, v [L][hkv][d]; q [hq][d]."""
     t_k64, t_q64, k, v, q = map(_f64, (t_k64, t_q64, k, v, q))
