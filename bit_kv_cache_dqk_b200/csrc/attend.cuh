@@ -42,7 +42,7 @@ namespace dqk {
 // independent instruction streams), plus one producer warp.  Four pages per
 // warp where the per-warp state allows (G <= 4), two for G = 8, whose two
 // query-head tiles double that state.
-__host__ __device__ constexpr int attend_warps(int G) { return 8; }
+__host__ __device__ constexpr int attend_warps(int G) { return G > 4 ? 8 : 12; }
 __host__ __device__ constexpr int attend_pages_per_warp(int G) { return G > 4 ? 2 : 4; }
 __host__ __device__ constexpr int attend_stage_blocks(int G) { return attend_pages_per_warp(G) * attend_warps(G); }
 __host__ __device__ constexpr int attend_threads(int G) { return 32 * (attend_warps(G) + 1); }
@@ -506,7 +506,17 @@ __device__ __forceinline__ void init_records(const AttendParams &p, const CtaUni
 // The producer warp of the attend kernels: brings the CTA's units [u0, u1)
 // into the ring, pps pages (each hc blocks, one bulk copy) per stage, marks
 // which page slots of a stage hold a page, and never leaves with copies in
-// flight.  Waits are bounded; a stuck pipeline sets the abort flag.
+// flight.  Lane l fills page slots l and l + 32 of a stage (pps <= 64).  The
+// page-table entries of the next stage are loaded before the wait for a free
+// stage, and checked when their copies are issued.  Waits are bounded; a
+// stuck pipeline sets the abort flag.
+constexpr int kMaxPagesPerStage = 64;
+
+struct ProducerSlots {
+    int phys[2], chunk[2];   // raw page-table entry and kv-head chunk of slot lane + 32k
+    bool in[2];              // the slot holds a unit of the CTA that maps to a page-table entry
+};
+
 __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned char *stage_mem, uint64_t *full,
                                                 uint64_t *empty, unsigned char *valid, volatile int *abort_flag,
                                                 int S, uint32_t stage_bytes, int kStageBlocks, const CtaUnits &cu,
@@ -516,69 +526,88 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
     const int u0 = cu.u0, u1 = cu.u1;
     grid_dependents_launch();   // the combine kernel may start its prologue
     if (iters == 0) return;
+    if (pps < 1 || pps > kMaxPagesPerStage || pps > kStageBlocks) {   // host plans never do this
+        if (lane == 0) {
+            *abort_flag = 1;
+            dqk_flag_error(kErrBounds);
+        }
+        return;
+    }
+    // cursor: run r starts at unit ur and has npr pages; never past the next stage's first unit
     int r = cu.r, ur = cu.ur;
     int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     const uint32_t copy_bytes = (uint32_t)(p.hc * p.bb);
-    // pool byte offset of unit ubase + lane (or -1); moves the cursor to unit ubase + 32
-    auto fetch = [&](int ubase) -> long long {
-        const int u = ubase + lane;
+    auto fetch = [&](int it) -> ProducerSlots {
+        ProducerSlots f;
+        const int base = u0 + it * pps;
         int rr = r, st = ur, np = npr;
-        while (rr < R && u >= st + np) {
-            st += np;
-            ++rr;
-            np = rr < R ? run_pages(p.seq_lens, p.nchunks, rr) : 0;
-        }
-        long long off = -1;
-        if (u < u1 && rr < R) {
-            const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
-            const int page = u - st;
-            if (page < p.max_pages) {
-                const int phys = p.page_table[(size_t)b * p.max_pages + page];
-                if (phys >= 0 && phys < p.num_pages)
-                    off = ((long long)phys * p.hkv + (long long)chunk * p.hc) * p.bb;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int slot = 32 * k + lane, u = base + slot;
+            f.in[k] = false;
+            f.phys[k] = -1;
+            f.chunk[k] = 0;
+            if (slot < pps && u < u1) {
+                while (rr < R && u >= st + np) {
+                    st += np;
+                    ++rr;
+                    np = rr < R ? run_pages(p.seq_lens, p.nchunks, rr) : 0;
+                }
+                if (rr < R) {
+                    const int b = rr / p.nchunks, page = u - st;
+                    f.chunk[k] = rr - b * p.nchunks;
+                    f.in[k] = true;
+                    if (page < p.max_pages) f.phys[k] = p.page_table[(size_t)b * p.max_pages + page];
+                }
             }
-            if (off < 0) dqk_flag_error(kErrBounds);
         }
-        r = __shfl_sync(0xffffffffu, rr, 31);
-        ur = __shfl_sync(0xffffffffu, st, 31);
-        npr = __shfl_sync(0xffffffffu, np, 31);
-        return off;
+        // the run of the stage's last unit becomes the cursor
+        const int last = min(pps, u1 - base) - 1;   // >= 0: stage `it` < iters
+        r = __shfl_sync(0xffffffffu, rr, last & 31);
+        ur = __shfl_sync(0xffffffffu, st, last & 31);
+        npr = __shfl_sync(0xffffffffu, np, last & 31);
+        return f;
     };
-    long long off_next = fetch(u0);
+    ProducerSlots cur = fetch(0);
     int it = 0, stage = 0;
     uint32_t phase = 0;
-    bool ok = true;
-    for (int ubase = u0; ubase < u1 && ok; ubase += 32) {
-        const long long off_cur = off_next;
-        if (ubase + 32 < u1) off_next = fetch(ubase + 32);
-        for (; it < iters && u0 + it * pps < ubase + 32; ++it) {
-            int good = 1;
-            if (lane == 0)
-                good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs, 2000u) && !*abort_flag;
-            if (!__shfl_sync(0xffffffffu, good, 0)) {
-                if (lane == 0) {
-                    *abort_flag = 1;
-                    dqk_flag_error(kErrTimeout);
-                }
-                ok = false;
-                break;
+    for (; it < iters; ++it) {
+        ProducerSlots nxt = cur;
+        if (it + 1 < iters) nxt = fetch(it + 1);
+        int good = 1;
+        if (lane == 0) good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs, 2000u) && !*abort_flag;
+        if (!__shfl_sync(0xffffffffu, good, 0)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                dqk_flag_error(kErrTimeout);
             }
-            // lane k < pps fills page slot k of this stage
-            const int uk = u0 + it * pps + lane;
-            const long long off = __shfl_sync(0xffffffffu, off_cur, (uk - ubase) & 31);
-            const bool have = lane < pps && uk < u1 && off >= 0;
-            const unsigned ballot = __ballot_sync(0xffffffffu, have);
-            if (lane < pps) valid[stage * kStageBlocks + lane] = have ? 1 : 0;
-            __syncwarp();
-            if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(ballot) * copy_bytes);
-            __syncwarp();
-            if (have)
-                bulk_copy_g2s(stage_mem + (size_t)stage * stage_bytes + (size_t)lane * copy_bytes, p.pool + off,
-                              copy_bytes, &full[stage]);
-            if (++stage == S) {
-                stage = 0;
-                phase ^= 1u;
-            }
+            break;
+        }
+        long long off[2];
+        bool have[2];
+        unsigned n = 0;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const bool ok = cur.in[k] && cur.phys[k] >= 0 && cur.phys[k] < p.num_pages;
+            if (cur.in[k] && !ok) dqk_flag_error(kErrBounds);
+            off[k] = ((long long)cur.phys[k] * p.hkv + (long long)cur.chunk[k] * p.hc) * p.bb;
+            have[k] = ok;
+            n += __popc(__ballot_sync(0xffffffffu, ok));
+            const int slot = 32 * k + lane;
+            if (slot < pps) valid[stage * kStageBlocks + slot] = ok ? 1 : 0;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&full[stage], n * copy_bytes);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            if (have[k])
+                bulk_copy_g2s(stage_mem + (size_t)stage * stage_bytes + (size_t)(32 * k + lane) * copy_bytes,
+                              p.pool + off[k], copy_bytes, &full[stage]);
+        cur = nxt;
+        if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
         }
     }
     // never leave with copies in flight (exit path: wait, bounded, for the last round of each stage)

@@ -69,6 +69,7 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
         }
     if (P.hc == 0) return false;
     P.pps = stage_blocks / P.hc;    // pages per stage
+    if (P.pps > kMaxPagesPerStage) return false;   // the producer warp fills two page slots per lane
     P.pw = warps / P.hc;            // warps per kv head (each takes attend_pages_per_warp pages of a stage)
     P.nchunks = hkv / P.hc;
     if ((long long)batch * P.nchunks * (L->num_pages + 1) >= (1LL << 31)) return false;

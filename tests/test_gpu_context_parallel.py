@@ -80,7 +80,9 @@ def test_context_parallel_matches_oracle(case, world):
     torch.cuda.synchronize(run.dev)
     merged = out.cpu().numpy().astype(np.float64)
     H.assert_outputs_close(merged, ref["out"])
-    np.testing.assert_allclose(merged, full, rtol=0, atol=1e-4)
+    # each split rounds its softmax weights to fp16 against its own running
+    # max, so two partitions of the same pages agree to ~2^-11 of |v|, not bitwise
+    np.testing.assert_allclose(merged, full, rtol=0, atol=1e-3)
 
 
 def test_single_range_partial_then_merge_is_decode():
