@@ -477,7 +477,24 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
                                         const LaneOffsets &o) {
     constexpr int NT = AttendTile<D, G>::NT;
     float s0[NB][NT], s1[NB][NT];
-    qk_scores<D, G, NS, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
+    if constexpr (NB > 2 && NB % 2 == 0) {
+        // scores two pages at a time: fewer registers live than with all NB at once
+#pragma unroll
+        for (int h = 0; h < NB; h += 2) {
+            const uint32_t hb[2] = {sb[h], sb[h + 1]};
+            float t0[2][NT], t1[2][NT];
+            qk_scores<D, G, NS, 2, MASKED>(hb, nv, st, lane, o, t0, t1);
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    s0[h + b][nt] = t0[b][nt];
+                    s1[h + b][nt] = t1[b][nt];
+                }
+        }
+    } else {
+        qk_scores<D, G, NS, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
+    }
     max_update<D, G, NB>(st, s0, s1);
     pv_accum<D, G, VCH0, NS, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
 }
