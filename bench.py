@@ -440,7 +440,10 @@ def _event_time_us(torch, fn, reps, flush):
         e1.record()
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1) * 1e3)
-    return statistics.median(ts)
+    # trimmed mean: event timestamps come in steps of about 2 us, which a median would keep
+    ts.sort()
+    cut = len(ts) // 10
+    return statistics.mean(ts[cut:len(ts) - cut])
 
 
 def run_sweep(args):
@@ -497,14 +500,46 @@ def run_sweep(args):
                                "dqk_algorithmic_gbs": algo / (t_dqk * 1e-6) / 1e9,
                                "dqk_bytes_per_token_kv_head": per_tok,
                                "bf16_gbs": b16_bytes / (t_b16 * 1e-6) / 1e9})
+    # whole decode steps (append one row per sequence, then decode) at 128K context, 40 %
+    steps = []
+    k1, v1 = I.kv_rows_device(w, range(Bmax), Lmax - 1, Lmax, dev)
+    for B in (4, 16):
+        L = Lmax
+        ws_bytes = max(Q.dqk_decode_workspace_size(desc, B, max_pages),
+                       Q.dqk_bf16_decode_workspace_size(desc_b, B, max_pages))
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        out = torch.empty((B, w.hq, w.d), dtype=torch.float32, device=dev)
+        lens_d = torch.full((B,), L, dtype=torch.int32, device=dev)
+        ones = torch.ones(B, dtype=torch.int32, device=dev)
+        before = torch.full((B,), L - 1, dtype=torch.int32, device=dev)
+        kb, vb = k1[:B].contiguous(), v1[:B].contiguous()
+        sel = torch.empty((B, w.hq, w.d - (40 * w.d) // 100), dtype=torch.int16, device=dev)
+
+        def dqk_step():
+            Q.dqk_decode_step(desc, kb, vb, Q.DQK_BF16, ones, before, 1, q, Q.DQK_BF16, B, lens_d, table_d,
+                              max_pages, 40, out, sel, ws, ws_bytes)
+
+        def bf16_step():
+            Q.dqk_bf16_append(desc_b, kb, vb, Q.DQK_BF16, B, ones, before, 1, table_d, max_pages)
+            Q.dqk_bf16_decode(desc_b, q, Q.DQK_BF16, B, lens_d, table_d, max_pages, out, ws, ws_bytes)
+
+        t_dqk = _event_time_us(torch, dqk_step, args.reps, flush)
+        t_b16 = _event_time_us(torch, bf16_step, args.reps, flush)
+        steps.append({"batch": B, "context": L, "sparsity_pct": 40, "dqk_step_us": t_dqk, "bf16_step_us": t_b16,
+                      "speedup": t_b16 / t_dqk, "dqk_kv_tokens_per_s": B * L / (t_dqk * 1e-6)})
     print(json.dumps({"metric": "decode time vs BF16 decode over sparsity x batch x context", "unit": "us",
                       "peak_hbm_gbs": peak, "peak_kind": peak_kind, "reps": args.reps,
-                      "timing": "median of CUDA-event times of one dqk_decode / dqk_bf16_decode call each, "
+                      "timing": "10 %-trimmed mean of CUDA-event times of one dqk_decode / dqk_bf16_decode call each, "
                                 "256 MB L2 flush before every call",
                       "data": "synthetic, drawn on the device (torch Philox), random page order",
                       "config": {"workload": "sweep: 32/8 heads, head_dim 128, BF16 K/V, batch {1,4,16} x "
                                              "context {8K,32K,128K} x sparsity {0,20,40,60}%"},
-                      "points": points}), flush=True)
+                      "points": points,
+                      "steps": steps,
+                      "step_timing": "one decode step each: dqk_decode_step (append 1 row per sequence + "
+                                     "decode, overlapped) vs dqk_bf16_append of the same row + "
+                                     "dqk_bf16_decode; 10 %-trimmed mean of CUDA-event times, 256 MB L2 flush before each"}),
+          flush=True)
 
 
 def run_append64(args):
@@ -544,7 +579,7 @@ def run_append64(args):
                       "rows_per_s": rows / (t * 1e-6),
                       "bytes_in": rows * w.d * 2 * 2, "bytes_out": pages_touched * w.hkv * bb,
                       "achieved_gbs": (rows * w.d * 4 + 2 * pages_touched * w.hkv * bb) / (t * 1e-6) / 1e9,
-                      "reps": args.reps, "timing": "median of CUDA-event times, 256 MB L2 flush before each call",
+                      "reps": args.reps, "timing": "10 %-trimmed mean of CUDA-event times, 256 MB L2 flush before each call",
                       "config": {"workload": f"qwen: batch {w.batch}, 32/8 heads, head_dim 128, lengths "
                                              f"{int(lens.min())}..{int(lens.max())}, {n} rows appended per "
                                              f"sequence"}}), flush=True)
