@@ -525,8 +525,9 @@ __device__ __forceinline__ void init_records(const AttendParams &p, const CtaUni
 // which page slots of a stage hold a page, and never leaves with copies in
 // flight.  Lane l fills page slots l and l + 32 of a stage (pps <= 64).  The
 // page-table entries of the next stage are loaded before the wait for a free
-// stage, and checked when their copies are issued.  Waits are bounded; a
-// stuck pipeline sets the abort flag.
+// stage, and checked when their copies are issued.  The pages are read once
+// per launch, so their copies carry an L2 evict-first policy.  Waits are
+// bounded; a stuck pipeline sets the abort flag.
 constexpr int kMaxPagesPerStage = 64;
 
 struct ProducerSlots {
@@ -554,6 +555,7 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
     int r = cu.r, ur = cu.ur;
     int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     const uint32_t copy_bytes = (uint32_t)(p.hc * p.bb);
+    const uint64_t stream_policy = l2_policy_evict_first();
     auto fetch = [&](int it) -> ProducerSlots {
         ProducerSlots f;
         const int base = u0 + it * pps;
@@ -619,8 +621,8 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
 #pragma unroll
         for (int k = 0; k < 2; ++k)
             if (have[k])
-                bulk_copy_g2s(stage_mem + (size_t)stage * stage_bytes + (size_t)(32 * k + lane) * copy_bytes,
-                              p.pool + off[k], copy_bytes, &full[stage]);
+                bulk_copy_g2s_hint(stage_mem + (size_t)stage * stage_bytes + (size_t)(32 * k + lane) * copy_bytes,
+                                   p.pool + off[k], copy_bytes, &full[stage], stream_policy);
         cur = nxt;
         if (++stage == S) {
             stage = 0;
