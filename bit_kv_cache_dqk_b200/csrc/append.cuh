@@ -286,8 +286,9 @@ __global__ void __launch_bounds__(512) k_quant_pack(
 
 // ---------------------------------------------------------------------------
 // k_append_rows: appends of up to a few dozen rows per sequence (decode steps,
-// speculative or chunked appends).  One CTA of D threads per (group of kRows
-// consecutive new rows of a sequence, kv head); thread c holds T_K's row c in
+// speculative or chunked appends).  One CTA of D threads per (group of RW
+// consecutive new rows of a sequence, kv head) -- RW = 1 when every sequence
+// appends one row (a decode step), else kRowsPerCta; thread c holds T_K's row c in
 // registers (read straight from global memory, all loads in flight at once)
 // and computes k'_c of every row of the group as interleaved independent
 // sums; warp g quantizes group g of each row.  Only the rows' own fields of
@@ -299,31 +300,32 @@ __global__ void __launch_bounds__(512) k_quant_pack(
 constexpr int kDirectMaxNew = 64;   // dqk_append uses k_append_rows up to this many rows per sequence
 constexpr int kRowsPerCta = 4;
 
-template <int D, int NS>
+template <int D, int NS, int RW>
 __global__ void __launch_bounds__(D) k_append_rows(
     const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin, int dtype,
     const int *__restrict__ new_lens, const int *__restrict__ seq_before, const int *__restrict__ page_table,
     int max_pages, int groups_per_seq, uint8_t *__restrict__ pool, long long num_pages, int hkv, int v_ch0,
     int early_release) {
     constexpr int NG = D / kGroup;
-    constexpr int RW = kRowsPerCta;
     __shared__ double xs[RW][D];
     __shared__ uint32_t kimg[RW][D], kmask[RW][D], vimg[RW][D], vmask[RW][D];   // code regions: D words each
     const int j = blockIdx.y;
     const int b = blockIdx.x / groups_per_seq, t0 = (blockIdx.x - b * groups_per_seq) * RW;
     const int c = threadIdx.x, warp = c >> 5, lane = c & 31;
     if (early_release) grid_dependents_launch();
+    // every load that depends only on (sequence, kv head, channel) is in
+    // flight before the first one is used: the lengths, the row offset of the
+    // sequence and T_K's row c
     const int n = new_lens[b];
-    if (t0 >= n) return;                      // the whole CTA
-    const int nr = min(RW, n - t0);           // rows of this CTA
     const int L0 = seq_before[b];
-    // T_K row c, all loads in flight
+    int row0 = 0;                             // rows of sequences 0..b-1 come first
+    for (int bb = lane; bb < b; bb += 32) row0 += new_lens[bb];
     const float4 *tr = reinterpret_cast<const float4 *>(t_k + ((size_t)j * D + c) * D);
     float4 tv[D / 4];
 #pragma unroll
-    for (int u = 0; u < D / 4; ++u) tv[u] = tr[u];
-    int row0 = 0;                             // rows of sequences 0..b-1 come first
-    for (int bb = lane; bb < b; bb += 32) row0 += new_lens[bb];
+    for (int u = 0; u < D / 4; ++u) tv[u] = ld_nc_f4(tr + u);
+    if (t0 >= n) return;                      // the whole CTA
+    const int nr = min(RW, n - t0);           // rows of this CTA
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) row0 += __shfl_xor_sync(0xffffffffu, row0, o);
     float xv[RW];

@@ -477,10 +477,11 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
                                         const LaneOffsets &o) {
     constexpr int NT = AttendTile<D, G>::NT;
     float s0[NB][NT], s1[NB][NT];
-    if constexpr (NB > 2 && NB % 2 == 0) {
-        // scores two pages at a time: fewer registers live than with all NB at once
+    if constexpr (NB > 2) {
+        // scores two pages at a time (an odd last page alone): fewer registers
+        // live than with all NB at once
 #pragma unroll
-        for (int h = 0; h < NB; h += 2) {
+        for (int h = 0; h + 1 < NB; h += 2) {
             const uint32_t hb[2] = {sb[h], sb[h + 1]};
             float t0[2][NT], t1[2][NT];
             qk_scores<D, G, NS, 2, MASKED>(hb, nv, st, lane, o, t0, t1);
@@ -491,6 +492,16 @@ __device__ __forceinline__ void consume(const uint32_t (&sb)[NB], int nv, WarpSt
                     s0[h + b][nt] = t0[b][nt];
                     s1[h + b][nt] = t1[b][nt];
                 }
+        }
+        if constexpr (NB % 2 == 1) {
+            const uint32_t hb[1] = {sb[NB - 1]};
+            float t0[1][NT], t1[1][NT];
+            qk_scores<D, G, NS, 1, MASKED>(hb, nv, st, lane, o, t0, t1);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                s0[NB - 1][nt] = t0[0][nt];
+                s1[NB - 1][nt] = t1[0][nt];
+            }
         }
     } else {
         qk_scores<D, G, NS, NB, MASKED>(sb, nv, st, lane, o, s0, s1);
@@ -657,21 +668,25 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
 
-    __shared__ CtaUnits sh_cu;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+    // The producer initialises the ring's barriers and announces them on named
+    // barrier 1 without waiting; every warp works out the CTA's unit range on
+    // its own, so the producer's first copies wait on nothing but the lengths
+    // and the page table.  Consumers wait on barrier 1 before their first use
+    // of the ring.
+    constexpr int kRingReady = 1;
+    if (warp == kConsumerWarps) {
+        if (lane == 0) {
+            for (int s = 0; s < S; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], kConsumerWarps);
+            }
+            *abort_flag = 0;
+            fence_mbar_init();
         }
-        *abort_flag = 0;
-        fence_mbar_init();
+        __syncwarp();
+        named_bar_arrive(kRingReady, attend_threads(G));
     }
-    if (warp == 0) {
-        const CtaUnits c = cta_units(p.seq_lens, p.nchunks, R, blockIdx.x, p.num_ctas, lane);
-        if (lane == 0) sh_cu = c;
-    }
-    __syncthreads();
-    const CtaUnits cu = sh_cu;
+    const CtaUnits cu = cta_units(p.seq_lens, p.nchunks, R, blockIdx.x, p.num_ctas, lane);
     const int u0 = cu.u0, u1 = cu.u1;
     const int nunits = u1 - u0;
     const int iters = (nunits + pps - 1) / pps;
@@ -688,6 +703,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const int slot_base = (int)blockIdx.x;
 
     if (nunits > 0) init_records(p, cu, slot_base, pi, jl, G, D, lane);
+    named_bar_sync(kRingReady, attend_threads(G));
     if (iters == 0) return;
     grid_dependency_wait();     // query fragments come from k_qprep
 
@@ -799,6 +815,24 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     uint32_t phase = 0;
     const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((BPW * pi * p.hc + jl) * p.bb);
     const uint32_t page_gap = (uint32_t)(p.hc * p.bb);
+    // n (1 .. BPW-1) full pages of one run at shared addresses base + q * page_gap
+    auto consume_batch = [&](int n, uint32_t base) {
+        if constexpr (BPW == 4) {
+            if (n == 3) {
+                const uint32_t sb3[3] = {base, base + page_gap, base + 2 * page_gap};
+                consume<D, G, VCH0, NS, 3, false>(sb3, kPage, st, lane, lo);
+                return;
+            }
+            if (n == 2) {
+                const uint32_t sb2[2] = {base, base + page_gap};
+                consume<D, G, VCH0, NS, 2, false>(sb2, kPage, st, lane, lo);
+                return;
+            }
+        }
+        const uint32_t sb1[1] = {base};
+        consume<D, G, VCH0, NS, 1, false>(sb1, kPage, st, lane, lo);
+    };
+
     const uint32_t valid_addr = smem_addr(valid) + BPW * pi;
     constexpr uint32_t kAllValid = (1u << BPW) - 1u;
     for (int it = 0; it < iters; ++it) {
@@ -833,6 +867,25 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
 #pragma unroll
                 for (int q = 0; q < BPW; ++q) sbb[q] = sa + q * page_gap;
                 consume<D, G, VCH0, NS, BPW, false>(sbb, kPage, st, lane, lo);
+            } else if (vv == kAllValid && ul < u1 && run_end <= ul && partial_u < 0) {
+                // the pages cross one run boundary, the run's last page is full:
+                // the pages of each run as one batch
+                const int k = run_end - ua;   // 1 .. BPW-1 pages of the current run
+                consume_batch(k, sa);
+                switch_run(run_end);
+                if (ul < run_end && !(partial_u >= ua + k && partial_u <= ul)) {
+                    consume_batch(BPW - k, sa + (uint32_t)k * page_gap);
+                } else {
+#pragma unroll
+                    for (int q = 1; q < BPW; ++q) {
+                        if (q < k) continue;
+                        const int uq = ua + q;
+                        if (uq >= run_end) switch_run(uq);
+                        const uint32_t s1[1] = {sa + q * page_gap};
+                        if (uq == partial_u) consume<D, G, VCH0, NS, 1, true>(s1, nv_last, st, lane, lo);
+                        else consume<D, G, VCH0, NS, 1, false>(s1, kPage, st, lane, lo);
+                    }
+                }
             } else {
 #pragma unroll
                 for (int q = 0; q < BPW; ++q) {
@@ -934,6 +987,16 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restri
     };
     index_chunk(0);
     __syncthreads();
+    {   // the first chunk's record lines (and their address translations)
+        // are requested while k_attend finishes; values are read after the wait
+        const int n0 = min(kCombineChunk, nrec);
+        if (threadIdx.x < n0 && sh_rec[threadIdx.x] >= 0) prefetch_l2(part + (size_t)sh_rec[threadIdx.x] * (2 + D));
+        if (lane == 0 || lane == 31)
+            for (int k = 0; k < kPer; ++k) {
+                const int i = slice + kSlices * k;
+                if (i < n0 && sh_rec[i] >= 0) prefetch_l2(part + (size_t)sh_rec[i] * (2 + D) + 2 + ch);
+            }
+    }
     grid_dependency_wait();     // partial records come from k_attend
     float *pr = out + ((size_t)b * hq + h) * (D + 2);   // partial record of (b, h)
     if (np == 0) {

@@ -115,6 +115,7 @@ struct DecodeArgs {
     size_t ws_bytes;
     cudaStream_t stream;
     bool partial = false;      // the combine writes (m, l, o) records instead of outputs
+    bool after_append = false; // the query kernel directly follows a step's append (writes first, waits last)
 };
 
 dqk_status check_decode(const DecodeArgs &a, DecodePlan &P) {
@@ -133,12 +134,13 @@ dqk_status check_decode(const DecodeArgs &a, DecodePlan &P) {
 
 // Every kernel of the path prefers the largest shared-memory carveout, so that
 // consecutive kernels do not make the SMs switch their L1 / shared split.
-// Attributes are per function; setting one twice is harmless.
-template <typename Kern>
-void prefer_max_shared(Kern kernel) {
+// Attributes are per function (one flag per kernel instance); setting one
+// twice is harmless.
+template <auto Kernel>
+void prefer_max_shared() {
     static bool done = false;
     if (!done) {
-        (void)cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+        (void)cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                    (int)cudaSharedmemCarveoutMaxShared);
         done = true;
     }
@@ -166,7 +168,7 @@ dqk_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 template <int D>
 dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
     const size_t smem = qprep_smem_bytes(D, P.G);
-    prefer_max_shared(k_qprep<D>);
+    prefer_max_shared<k_qprep<D>>();
     if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return DQK_ERR_CUDA;
     char *ws = static_cast<char *>(a.ws);
@@ -175,12 +177,12 @@ dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
                       a.q, (int)a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qscale,
                       reinterpret_cast<uint2 *>(ws + P.off_qf), reinterpret_cast<float *>(ws + P.off_qk),
                       reinterpret_cast<uint32_t *>(ws + P.off_qm), reinterpret_cast<float *>(ws + P.off_q0),
-                      a.sel_out);
+                      a.sel_out, a.after_append ? 1 : 0);
 }
 
 template <int D, int G, bool VCH0, int NS>
 dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
-    prefer_max_shared(k_attend<D, G, VCH0, NS>);
+    prefer_max_shared<k_attend<D, G, VCH0, NS>>();
     if (cudaFuncSetAttribute(k_attend<D, G, VCH0, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
         cudaSuccess)
         return DQK_ERR_CUDA;
@@ -233,7 +235,7 @@ dqk_status run_attend(const DecodeArgs &a, const DecodePlan &P) {
 template <int D>
 dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
     char *ws = static_cast<char *>(a.ws);
-    prefer_max_shared(k_combine<D>);
+    prefer_max_shared<k_combine<D>>();
     return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(kCombineThreads), 0, a.stream, a.seq_lens,
                       a.batch,
                       a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pw, P.nchunks, P.num_ctas,
@@ -267,11 +269,15 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
                       const int *new_lens, const int *seq_before, int max_new, const int *page_table,
                       int max_pages, int early_release, cudaStream_t stream) {
     if (max_new <= kDirectMaxNew) {
-        prefer_max_shared(k_append_rows<D, NS>);
-        const int groups = (max_new + kRowsPerCta - 1) / kRowsPerCta;
+        // one row per sequence (a decode step): one row per CTA, no idle row slots
+        if (max_new == 1) prefer_max_shared<k_append_rows<D, NS, 1>>();
+        else prefer_max_shared<k_append_rows<D, NS, kRowsPerCta>>();
+        auto kernel = max_new == 1 ? k_append_rows<D, NS, 1> : k_append_rows<D, NS, kRowsPerCta>;
+        const int rw = max_new == 1 ? 1 : kRowsPerCta;
+        const int groups = (max_new + rw - 1) / rw;
         const long long gx = (long long)batch * groups;
         if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
-        k_append_rows<D, NS><<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
+        kernel<<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
             L->t_k, k, v, dtype, new_lens, seq_before, page_table, max_pages, groups,
             static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
         return launch_status();
@@ -386,6 +392,7 @@ dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const voi
         st = launch_append(layer, k, v, kv_dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages,
                            1, a.stream);
         if (st != DQK_OK) return st;
+        a.after_append = true;
     }
     return decode_stages(a, kPrepare | kAttend | kCombine);
 }

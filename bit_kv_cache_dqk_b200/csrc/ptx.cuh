@@ -69,6 +69,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+// 16-byte load of read-only global data as a volatile asm statement: the
+// compiler keeps it where it stands (it may not sink it into a later loop),
+// so a batch of such loads is in flight at once.
+__device__ __forceinline__ float4 ld_nc_f4(const float4 *ptr) {
+    float4 v;
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(ptr));
+    return v;
+}
+
+// Non-binding prefetch of one global line into L2 (address translation
+// included); no data is returned.
+__device__ __forceinline__ void prefetch_l2(const void *ptr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
+// Named barrier `id` over `n` threads: arrive without waiting, or arrive and
+// wait.  (Barrier 0 is __syncthreads.)
+__device__ __forceinline__ void named_bar_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // L2 policy for data read once per launch: evicted first, so the small
 // tensors a decode step re-reads (page table, lengths, transforms, query
 // fragments, split records) stay resident across steps.

@@ -72,7 +72,8 @@ constexpr int kQprepThreads = 512;
 
 // Shared memory of k_qprep: T_Q[j] in fp32 with rows padded to D+4 floats
 // (conflict-free 16-byte row reads), the query rows in fp64, per-head sort
-// buffers and the outputs before they are laid out.
+// buffers and the outputs before they are laid out.  (T_Q held in fp64 would
+// double this; the larger CTAs then slow a co-running append.)
 __host__ __device__ constexpr size_t qprep_smem_bytes(int D, int G) {
     return (size_t)D * (D + 4) * 4 + (size_t)G * D * 8 + (size_t)kQprepThreads * 8 + (size_t)G * (D / 32) * 8 +
            (size_t)G * D * 3 + 64;
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
                                                         int dtype, int hq, int hkv, int pct, float qscale,
                                                         uint2 *__restrict__ qf, float *__restrict__ qk,
                                                         uint32_t *__restrict__ qm, float *__restrict__ q0,
-                                                        int16_t *__restrict__ sel_out) {
+                                                        int16_t *__restrict__ sel_out, int write_first) {
     constexpr int NG = D / 32;
     constexpr int kRow = D + 4;                       // padded fp32 row of T_Q
     constexpr int kHeadsPerPass = kQprepThreads / D;
@@ -133,7 +134,13 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
     }
     __syncthreads();
 
-    bool waited = false;
+    // write_first: the kernel before this one on the stream (a cache append
+    // launched without programmatic serialization) writes nothing this kernel
+    // reads or writes, and everything before it has finished, so the outputs
+    // are written at once and the wait for it comes last (this kernel's
+    // completion then implies the append's).  Otherwise the outputs wait for
+    // every earlier kernel of the stream.
+    bool waited = write_first != 0;
     for (int h0 = 0; h0 < G; h0 += kHeadsPerPass) {
         const int hl = h0 + hp;                 // local query head of this thread
         const bool active = hl < G;
@@ -261,6 +268,10 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
             w = lo | (hi << 16);
         }
         qm[(bj * NT + nt) * 32 + L] = w;
+    }
+    if (write_first) {
+        grid_dependency_wait();     // the append is complete
+        grid_dependents_launch();   // the attend kernel may start streaming pages now
     }
 }
 
