@@ -536,9 +536,11 @@ __device__ __forceinline__ void init_records(const AttendParams &p, const CtaUni
 // which page slots of a stage hold a page, and never leaves with copies in
 // flight.  Lane l fills page slots l and l + 32 of a stage (pps <= 64).  The
 // page-table entries of the next stage are loaded before the wait for a free
-// stage, and checked when their copies are issued.  The pages are read once
-// per launch, so their copies carry an L2 evict-first policy.  Waits are
-// bounded; a stuck pipeline sets the abort flag.
+// stage, and checked when their copies are issued.  kEvictFirst: the pages
+// are read once per launch, so their copies carry an L2 evict-first policy
+// (the packed cache; the BF16 comparison streams without a policy, which
+// measured faster for it).  Waits are bounded; a stuck pipeline sets the
+// abort flag.
 constexpr int kMaxPagesPerStage = 64;
 
 struct ProducerSlots {
@@ -546,6 +548,7 @@ struct ProducerSlots {
     bool in[2];              // the slot holds a unit of the CTA that maps to a page-table entry
 };
 
+template <bool kEvictFirst>
 __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned char *stage_mem, uint64_t *full,
                                                 uint64_t *empty, unsigned char *valid, volatile int *abort_flag,
                                                 int S, uint32_t stage_bytes, int kStageBlocks, const CtaUnits &cu,
@@ -566,7 +569,7 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
     int r = cu.r, ur = cu.ur;
     int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     const uint32_t copy_bytes = (uint32_t)(p.hc * p.bb);
-    const uint64_t stream_policy = l2_policy_evict_first();
+    const uint64_t stream_policy = kEvictFirst ? l2_policy_evict_first() : 0ull;
     auto fetch = [&](int it) -> ProducerSlots {
         ProducerSlots f;
         const int base = u0 + it * pps;
@@ -631,9 +634,11 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
         __syncwarp();
 #pragma unroll
         for (int k = 0; k < 2; ++k)
-            if (have[k])
-                bulk_copy_g2s_hint(stage_mem + (size_t)stage * stage_bytes + (size_t)(32 * k + lane) * copy_bytes,
-                                   p.pool + off[k], copy_bytes, &full[stage], stream_policy);
+            if (have[k]) {
+                void *dst = stage_mem + (size_t)stage * stage_bytes + (size_t)(32 * k + lane) * copy_bytes;
+                if constexpr (kEvictFirst) bulk_copy_g2s_hint(dst, p.pool + off[k], copy_bytes, &full[stage], stream_policy);
+                else bulk_copy_g2s(dst, p.pool + off[k], copy_bytes, &full[stage]);
+            }
         cur = nxt;
         if (++stage == S) {
             stage = 0;
@@ -692,7 +697,8 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     const int iters = (nunits + pps - 1) / pps;
 
     if (warp == kConsumerWarps) {
-        attend_producer(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kStageBlocks, cu, iters, lane);
+        attend_producer<true>(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kStageBlocks, cu, iters,
+                              lane);
         return;
     }
 

@@ -242,8 +242,8 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     const int u0 = cu.u0, u1 = cu.u1;
     const int iters = (u1 - u0 + pps - 1) / pps;
     if (warp == kB16Warps) {
-        attend_producer(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kB16StageBlocks, cu, iters,
-                        lane);
+        attend_producer<false>(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kB16StageBlocks, cu, iters,
+                               lane);
         return;
     }
     // consumer warp: kv head jl of the chunk, page slot pi of each stage

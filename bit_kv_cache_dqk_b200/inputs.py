@@ -68,6 +68,7 @@ class Workload:
     ctx_hi: int = 65536
     v_ch0_protect: int = 0
     group_size: int = 32         # channels per (scale, min) group: 32, or head_dim (one group per token)
+    len_multiple: int = 1        # ragged lengths rounded up to a multiple of this (16: only full pages)
 
     @property
     def group(self) -> int:
@@ -103,7 +104,9 @@ def lengths(w: Workload) -> np.ndarray:
     if w.ctx is not None:
         return np.full(w.batch, w.ctx, dtype=np.int32)
     rng = np.random.default_rng([w.seed, _S_LEN])
-    return rng.integers(w.ctx_lo, w.ctx_hi + 1, size=w.batch).astype(np.int32)
+    lens = rng.integers(w.ctx_lo, w.ctx_hi + 1, size=w.batch)
+    m = w.len_multiple
+    return (((lens + m - 1) // m) * m).astype(np.int32)
 
 
 def page_table(w: Workload, lens: np.ndarray):

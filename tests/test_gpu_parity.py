@@ -43,6 +43,10 @@ CASES = {
     "g64-d64": small("llama", batch=2, hq=8, hkv=4, d=64, ctx=500, group_size=64),
     # calibrated transform pair and structured queries (next-step row f1)
     "calibrated": small("llama_cal", batch=2, ctx=None, ctx_lo=300, ctx_hi=900),
+    # lengths that are whole pages: run boundaries fall at every offset within a
+    # warp's four pages of a stage with the run's last page full, so the pages on
+    # each side of a boundary are consumed as separate batches
+    "full-pages": small("llama", batch=12, ctx=None, ctx_lo=16, ctx_hi=900, len_multiple=16, page_order="random"),
     # five kv heads: one head per chunk, the most pages per stage; long enough
     # that every CTA's ring wraps several times
     "hkv5-wrap": small("llama", batch=2, hq=20, hkv=5, ctx=34000, page_order="random"),
