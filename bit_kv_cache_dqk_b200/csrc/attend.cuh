@@ -19,7 +19,8 @@
 //        in the columns a GQA group of 4 leaves free (16 bits relative to the
 //        group's largest |qs|); one AND per 4 codes forms the u8 operand;
 //        s[t, h] = sum_g scale[t, g] * kappa_g * (D_g[t,(h,1)] + D_g[t,(h,2)]/256)
-//                + sum_g min[t, g] * Qsum[g, h]   (one extra m16n8k16)
+//                + sum_g min[t, g] * Qsum[g, h]   (one extra m16n8k16; the high and
+//                                                  low fp16 parts of Qsum in separate rows)
 //                + qs_0[h] * k0[t]                (BF16 channel 0, fp32)
 //   online softmax in base 2 (running max per head, exact rescale on growth)
 //   PV   O^T[c, h] += sum_t code_v[t, c] * (p~[t, h] * vscale[t, g(c)])
@@ -244,8 +245,9 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
                 ks1[b][0] = ld_s32(a + Ly.ks + 32);
             }
             const uint32_t akm = sb[b] + o.kmin;
-            // lanes past the groups read this token's other mins; the min-term B
-            // operand is zero in those rows
+            // A columns k and NG + k both hold group k's min (lanes tig >= NG/2
+            // repeat the pairs of the lanes below); the B operand holds the high
+            // and the low fp16 part of Qsum there, so one tile sums both
             km0[b] = ld_s32(akm + Ly.km);
             km1[b] = ld_s32(akm + Ly.km + 16 * NG);
         }
@@ -314,8 +316,8 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
     for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            s0[b][nt] = a0[b][nt] + fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0] + cmin[b][nt][1]);
-            s1[b][nt] = a1[b][nt] + fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2] + cmin[b][nt][3]);
+            s0[b][nt] = a0[b][nt] + fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0]);
+            s1[b][nt] = a1[b][nt] + fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2]);
             if constexpr (MASKED) {
                 if (gid >= nv) s0[b][nt] = -INFINITY;
                 if (gid + 8 >= nv) s1[b][nt] = -INFINITY;
@@ -721,7 +723,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
     LaneOffsets lo;
     lo.lane16 = lane * 16;
     lo.gid8 = gid * 8;
-    lo.kmin = gid * 2 * NG + (tig & (NG / 2 - 1)) * 4;   // in range for every lane (B rows past NG are 0)
+    lo.kmin = gid * 2 * NG + (tig & (NG / 2 - 1)) * 4;   // in range for every lane (B rows past 2 NG are 0)
     lo.gid4 = gid * 4;
     lo.tig16 = tig * 16;
     lo.vmin = (tig * NS + (gid < NS ? gid : 0)) * 4;

@@ -59,8 +59,10 @@ __device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[E], in
 //   qk  [B*Hkv][NT][NG][4] float       kappa = sigma / 4^g per head (the key
 //       operand of group g carries code * 4^g).
 //   qm  [B*Hkv][NT][32] uint32         per lane: rows 2*tig, 2*tig+1 of the
-//       fp16 min-term B operand: Qsum_{g,h} = sum of qs over the group's kept
-//       channels (high part for even gid, low part for odd gid).
+//       fp16 min-term B operand, Qsum_{g,h} = sum of qs over the group's kept
+//       channels: row k < NG holds the high fp16 part of group k, row NG + k
+//       the low part (the key mins repeat in those A columns), so one tile
+//       sums both; column 2h holds query head 4*nt + h, odd columns are zero.
 //   q0  [B][Hq] float                  qs of channel 0 (always kept).
 __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
     const __half hi = __float2half_rn(x);
@@ -259,13 +261,14 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
     }
     for (int idx = threadIdx.x; idx < NT * 32; idx += blockDim.x) {
         const int L = idx & 31, nt = idx >> 5;
-        const int gid = L >> 2, tig = L & 3, hl = 4 * nt + (gid >> 1), piece = gid & 1;
+        const int gid = L >> 2, tig = L & 3, hl = 4 * nt + (gid >> 1);
         uint32_t w = 0;
-        if (hl < G) {
-            const int g0 = 2 * tig, g1 = 2 * tig + 1;
-            const uint32_t lo = g0 < NG ? f16_piece(qsum[hl * NG + g0], piece) : 0u;
-            const uint32_t hi = g1 < NG ? f16_piece(qsum[hl * NG + g1], piece) : 0u;
-            w = lo | (hi << 16);
+        if (hl < G && (gid & 1) == 0) {
+            // rows k = 2*tig, 2*tig + 1: piece k / NG (0 high, 1 low) of group k % NG
+            const int k0 = 2 * tig, k1 = 2 * tig + 1;
+            const uint32_t r0 = k0 < 2 * NG ? f16_piece(qsum[hl * NG + k0 % NG], k0 / NG) : 0u;
+            const uint32_t r1 = k1 < 2 * NG ? f16_piece(qsum[hl * NG + k1 % NG], k1 / NG) : 0u;
+            w = r0 | (r1 << 16);
         }
         qm[(bj * NT + nt) * 32 + L] = w;
     }

@@ -185,8 +185,9 @@ dqk_status dqk_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dt
  *  Result: the same bytes as dqk_append followed by dqk_decode on `stream`.
  *  The difference is on the GPU: the query transform and selection run while
  *  the append is still writing the cache (the query kernel reads only q and
- *  T_Q before waiting for the append), and the attention kernel starts
- *  streaming pages as soon as the append has finished. */
+ *  T_Q and writes only the workspace, so it writes its results at once and
+ *  waits for the append as its last step), and the attention kernel starts
+ *  streaming pages as soon as both have finished. */
 dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const void *v,
                            dqk_dtype kv_dtype, const int *new_lens, const int *seq_lens_before,
                            int max_new, const void *q, dqk_dtype q_dtype, int batch,
