@@ -16,12 +16,18 @@
 // qs = q' * log2(e)/sqrt(d) on the kept channels:
 //   QK   D_g[t, n] = sum_{c in g} code[t, c] * Q[c, n]    (m16n8k32 u8 x s8, per group)
 //        n = (head, piece): qs ~= sigma_g (Q1 + Q2/256) in two int8 pieces placed
-//        in the columns a GQA group of 4 leaves free (16 bits relative to the
-//        group's largest |qs|); one AND per 4 codes forms the u8 operand;
-//        s[t, h] = sum_g scale[t, g] * kappa_g * (D_g[t,(h,1)] + D_g[t,(h,2)]/256)
+//        in the columns a GQA group of 4 leaves free, sigma_g = sigma_h 2^-e_g
+//        (15-16 bits relative to the group's largest |qs|); one AND per 4 codes
+//        forms the u8 operand (code * 4^g);
+//        s[t, h] = sigma_h * sum_g scale[t, g] * p_g * (D_g[t,(h,1)] + D_g[t,(h,2)]/256)
 //                + sum_g min[t, g] * Qsum[g, h]   (one extra m16n8k16; the high and
 //                                                  low fp16 parts of Qsum in separate rows)
 //                + qs_0[h] * k0[t]                (BF16 channel 0, fp32)
+//        with p_g = 2^-e_g / 4^g.  The piece-1 accumulators start at 1.5 * 2^23
+//        and the piece-2 ones at 1.5 * 2^15, so as floats they read
+//        M1 + D1 and M2 + D2/256 exactly, and two FFMAs give
+//        p_g (D1 + D2/256) with one rounding: (M1 + D1) p - (M1 + M2) p is exact,
+//        then (M2 + D2/256) p is added.
 //   online softmax in base 2 (running max per head, exact rescale on growth)
 //   PV   O^T[c, h] += sum_t code_v[t, c] * (p~[t, h] * vscale[t, g(c)])
 //        with p~ = fp16(p); one extra m16n8k16 gives sum_t p~ * vmin[t, g] and
@@ -177,7 +183,8 @@ struct WarpState {
     using T = AttendTile<D, G>;
     static constexpr bool kRegFrags = T::NT == 1;   // score fragments in registers (else per-warp shared memory)
     uint2 qb[kRegFrags ? T::NG : 1];                // score B fragments of group g
-    float4 kp[kRegFrags ? T::NG : 1];               // kappa, kappa/256, -M kappa, -M kappa/256 of group g
+    float2 kp[kRegFrags ? T::NG : 1];               // p_g and -(M1 + M2) p_g of group g
+    float sgh[T::NT];              // sigma_h of this thread's head
     uint32_t qmin[T::NT];          // min-term B fragment
     float q0v[T::NT];              // scaled q'_0 of this thread's head
     float m_run[T::NT];            // running max (log2 units) of this thread's head
@@ -195,7 +202,7 @@ struct LaneOffsets {
     uint32_t vmin;     // V min pair of row min(gid, NG-1), tokens 2tig, 2tig+1
     int srcA;          // lane holding p of (token 2tig, head gid/2); +4: token 2tig+1
     uint32_t sq;       // shared address of this lane's QK B fragments: [NT][NG][32 lanes] uint2
-    uint32_t sk;       // shared address of this thread's head constants: [NT][NG][4 heads] float4
+    uint32_t sk;       // shared address of this thread's head constants: [NT][NG][4 heads] 16-byte slots (p_g pair)
     uint32_t ones_lane, vmin_mask;
 };
 
@@ -268,7 +275,7 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
     for (int g = 0; g < NG; ++g) {
         const uint32_t msk = 0x03030303u << (2 * g);   // group g's field in every byte: code * 4^g
         uint2 qb[NT];
-        float4 kp[NT];
+        float2 kp[NT];
         if constexpr (WarpState<D, G>::kRegFrags) {
             qb[0] = st.qb[g];
             kp[0] = st.kp[g];
@@ -276,9 +283,8 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 qb[nt] = ld_s64(o.sq + (nt * NG + g) * 256);
-                const uint4 kpu = ld_s128(o.sk + (nt * NG + g) * 64);
-                kp[nt] = make_float4(__uint_as_float(kpu.x), __uint_as_float(kpu.y), __uint_as_float(kpu.z),
-                                     __uint_as_float(kpu.w));
+                const uint2 kpu = ld_s64(o.sk + (nt * NG + g) * 64);
+                kp[nt] = make_float2(__uint_as_float(kpu.x), __uint_as_float(kpu.y));
             }
         }
 #pragma unroll
@@ -302,13 +308,13 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 int dg[4];
-                mma_u8s8(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y, kMagicI);
-                // (M + I) * kappa - M * kappa = I * kappa, one rounding
-                const float4 k4 = kp[nt];
-                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[0]), k4.x, k4.z), a0[b][nt]);
-                a0[b][nt] = fmaf(sa, fmaf(__int_as_float(dg[1]), k4.y, k4.w), a0[b][nt]);
-                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[2]), k4.x, k4.z), a1[b][nt]);
-                a1[b][nt] = fmaf(sbv, fmaf(__int_as_float(dg[3]), k4.y, k4.w), a1[b][nt]);
+                mma_u8s8_c2(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y, kMagicI, kMagicLoI);
+                // p (D1 + D2/256): (M1 + D1) p - (M1 + M2) p exact, + (M2 + D2/256) p, one rounding
+                const float2 k2 = kp[nt];
+                const float x0 = fmaf(__int_as_float(dg[1]), k2.x, fmaf(__int_as_float(dg[0]), k2.x, k2.y));
+                const float x1 = fmaf(__int_as_float(dg[3]), k2.x, fmaf(__int_as_float(dg[2]), k2.x, k2.y));
+                a0[b][nt] = fmaf(sa, x0, a0[b][nt]);
+                a1[b][nt] = fmaf(sbv, x1, a1[b][nt]);
             }
         }
     }
@@ -316,8 +322,8 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
     for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            s0[b][nt] = a0[b][nt] + fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0]);
-            s1[b][nt] = a1[b][nt] + fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2]);
+            s0[b][nt] = fmaf(st.sgh[nt], a0[b][nt], fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0]));
+            s1[b][nt] = fmaf(st.sgh[nt], a1[b][nt], fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2]));
             if constexpr (MASKED) {
                 if (gid >= nv) s0[b][nt] = -INFINITY;
                 if (gid + 8 >= nv) s1[b][nt] = -INFINITY;
@@ -745,19 +751,18 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendPar
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
                 const uint2 qb = p.qf[((bj * NT + nt) * NG + g) * 32 + lane];
-                const float kappa = p.qk[((bj * NT + nt) * NG + g) * 4 + tig];
-                const float4 kp = make_float4(kappa, kappa * (1.0f / 256.0f), -kMagicF * kappa,
-                                              -kMagicF * kappa * (1.0f / 256.0f));
+                const float pg = p.qk[((bj * NT + nt) * (NG + 1) + g) * 4 + tig];
+                const float2 kp = make_float2(pg, -(kMagicF + kMagicLoF) * pg);   // exact: power-of-two p_g
                 if constexpr (WarpState<D, G>::kRegFrags) {
                     st.qb[g] = qb;
                     st.kp[g] = kp;
                 } else {
                     st_s64(lo.sq + (nt * NG + g) * 256, qb);
                     if (gid == 0)
-                        st_s128(lo.sk + (nt * NG + g) * 64, make_uint4(__float_as_uint(kp.x), __float_as_uint(kp.y),
-                                                                       __float_as_uint(kp.z), __float_as_uint(kp.w)));
+                        st_s64(lo.sk + (nt * NG + g) * 64, make_uint2(__float_as_uint(kp.x), __float_as_uint(kp.y)));
                 }
             }
+            st.sgh[nt] = p.qk[((bj * NT + nt) * (NG + 1) + NG) * 4 + tig];
             __syncwarp();
             st.qmin[nt] = p.qm[(bj * NT + nt) * 32 + lane];
             const int hh = 4 * nt + tig;

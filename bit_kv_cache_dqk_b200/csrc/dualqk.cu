@@ -90,7 +90,7 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     const size_t bj = (size_t)batch * hkv;
     P.off_qf = 256;
     P.off_qk = round_up(P.off_qf + bj * P.NT * P.NG * 32 * sizeof(uint2), 256);
-    P.off_qm = round_up(P.off_qk + bj * P.NT * P.NG * 4 * sizeof(float), 256);
+    P.off_qm = round_up(P.off_qk + bj * P.NT * (P.NG + 1) * 4 * sizeof(float), 256);
     P.off_q0 = round_up(P.off_qm + bj * P.NT * 32 * sizeof(uint32_t), 256);
     P.off_part = round_up(P.off_q0 + (size_t)batch * L->num_q_heads * sizeof(float), 256);
     const size_t records = ((size_t)kMaxAttendCtas + R - 1) * P.pw * P.hc * P.G;

@@ -183,6 +183,16 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c));
 }
 
+// The same with the accumulator of even columns started at c_even and of odd
+// columns at c_odd.
+__device__ __forceinline__ void mma_u8s8_c2(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1, int c_even, int c_odd) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%10,%11};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c_even), "r"(c_odd));
+}
+
 // D = A * B (zero accumulator), m16n8k16 fp16, fp32 result.
 __device__ __forceinline__ void mma_f16_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                              uint32_t b0, uint32_t b1) {
@@ -197,6 +207,9 @@ __device__ __forceinline__ void mma_f16_zero(float (&d)[4], uint32_t a0, uint32_
 // reads as the float kMagicF + sum, exactly, while |sum| < 2^22.
 constexpr int kMagicI = 0x4B400000;
 constexpr float kMagicF = 12582912.0f;
+// 1.5 * 2^15 (0x47400000): reads as kMagicLoF + sum / 256, exactly, while |sum| < 2^22.
+constexpr int kMagicLoI = 0x47400000;
+constexpr float kMagicLoF = 49152.0f;
 
 // Two 2-bit codes at bit 2P of each 16-bit half of x -> an f16x2 holding the
 // exact values 0..3.  OR-ing the field into the mantissa of 2^(10-2P) gives

@@ -53,11 +53,13 @@ __device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[E], in
 //   qf  [B*Hkv][NT][NG][32] uint2      per lane: the two s8x4 registers of the
 //       m16n8k32 B operand of group g: rows (channels of the group) 4*tig..+3
 //       and 16+4*tig..+3, column n = gid -> query head 4*nt + gid/2; gid even:
-//       Q1 = rne(qs/sigma), odd: Q2 = clamp(rne((qs/sigma - Q1)*256)), with
-//       sigma = max_g |qs| / 127 rounded up to 22 significant bits, so
-//       qs ~= sigma * (Q1 + Q2/256).
-//   qk  [B*Hkv][NT][NG][4] float       kappa = sigma / 4^g per head (the key
-//       operand of group g carries code * 4^g).
+//       Q1 = rne(qs/sigma_g), odd: Q2 = clamp(rne((qs/sigma_g - Q1)*256)), so
+//       qs ~= sigma_g * (Q1 + Q2/256); sigma_h = (largest |qs| of the head) / 127
+//       and sigma_g = sigma_h * 2^-e_g, the smallest such value not below the
+//       group's largest |qs| / 127 (the pieces keep 15-16 bits relative to it).
+//   qk  [B*Hkv][NT][NG+1][4] float     per head: entry g < NG holds
+//       p_g = 2^-e_g / 4^g (the key operand of group g carries code * 4^g), so
+//       sigma_g / 4^g = sigma_h * p_g; entry NG holds sigma_h.
 //   qm  [B*Hkv][NT][32] uint32         per lane: rows 2*tig, 2*tig+1 of the
 //       fp16 min-term B operand, Qsum_{g,h} = sum of qs over the group's kept
 //       channels: row k < NG holds the high fp16 part of group k, row NG + k
@@ -78,7 +80,7 @@ constexpr int kQprepThreads = 512;
 // double this; the larger CTAs then slow a co-running append.)
 __host__ __device__ constexpr size_t qprep_smem_bytes(int D, int G) {
     return (size_t)D * (D + 4) * 4 + (size_t)G * D * 8 + (size_t)kQprepThreads * 8 + (size_t)G * (D / 32) * 8 +
-           (size_t)G * D * 3 + 64;
+           (size_t)G * (D / 32 + 1) * 4 + (size_t)G * D * 3 + 64;
 }
 
 // One thread per (query head, channel), kQprepThreads / D heads per pass.
@@ -103,8 +105,10 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
     double *qin = reinterpret_cast<double *>(tq + D * kRow);                         // [G][D]
     unsigned long long *xbuf = reinterpret_cast<unsigned long long *>(qin + G * D);  // [threads] sort exchange
     float *qsum = reinterpret_cast<float *>(xbuf + kQprepThreads);                   // [G][NG]
-    float *sig = qsum + G * NG;                                                       // [G][NG]  sigma
-    signed char *q8 = reinterpret_cast<signed char *>(sig + G * NG);                 // [G][2][D] pieces
+    float *sig = qsum + G * NG;                                                       // [G][NG]  p_g
+    float *gmax = sig + G * NG;                                                       // [G][NG]  largest |qs|
+    float *shd = gmax + G * NG;                                                       // [G]      sigma_h
+    signed char *q8 = reinterpret_cast<signed char *>(shd + G);                      // [G][2][D] pieces
     unsigned char *mask = reinterpret_cast<unsigned char *>(q8 + G * 2 * D);         // [G][D]
     int *wcount = reinterpret_cast<int *>(mask + G * D + ((16 - (G * D) % 16) % 16)); // [threads/32] kept per warp
     const int j = blockIdx.x, b = blockIdx.y;
@@ -196,9 +200,9 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
         const unsigned bal = __ballot_sync(0xffffffffu, keep);
         if (lane == 0) wcount[warp] = __popc(bal);
         // scaled q' on kept channels >= 1; group sums and two int8 pieces
-        // relative to the group's largest |qs| (warp = one group of one head),
-        // sigma rounded up to 22 significant bits (so 1.5 * 2^23 * sigma / 4^g
-        // is exact)
+        // (warp = one group of one head) relative to sigma_g = sigma_h * 2^-e,
+        // the smallest such value not below the group's largest |qs| / 127, so
+        // that sigma_g / sigma_h is a power of two
         const float qs = qp * qscale;
         const float v = (keep && c != 0) ? qs : 0.0f;
         float gs = v, gm = fabsf(v);
@@ -207,22 +211,33 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
             gs += __shfl_xor_sync(0xffffffffu, gs, o);
             gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
         }
-        float sgm = gm / 127.0f;
-        sgm = __uint_as_float((__float_as_uint(sgm) + 3u) & ~3u);
+        const int g = c >> 5;
+        if (active && lane == 0) gmax[hl * NG + g] = gm;
+        __syncthreads();
+        float hm = 0.0f;
+        if (active)
+            for (int gg = 0; gg < NG; ++gg) hm = fmaxf(hm, gmax[hl * NG + gg]);
+        const float sh = hm / 127.0f, tg = gm / 127.0f;
+        int e = 0;
+        if (tg > 0.0f) {
+            e = ilogbf(sh) - ilogbf(tg);   // >= 0: sh >= tg
+            if (ldexpf(sh, -e) < tg) --e;
+        }
+        const float sgm = ldexpf(sh, -e);   // in [tg, 2 tg)
         int q1 = 0, q2 = 0;
         if (sgm > 0.0f) {
             const float x = v / sgm;
             q1 = max(-127, min(127, __float2int_rn(x)));
             q2 = max(-128, min(127, __float2int_rn((x - (float)q1) * 256.0f)));
         }
-        const int g = c >> 5;
         if (active) {
             q8[(hl * 2 + 0) * D + c] = (signed char)q1;
             q8[(hl * 2 + 1) * D + c] = (signed char)q2;
             if (lane == 0) {
                 qsum[hl * NG + g] = gs;
-                sig[hl * NG + g] = sgm;
+                sig[hl * NG + g] = ldexpf(1.0f, -e - 2 * g);
             }
+            if (c == 0) shd[hl] = sh;
         }
         __syncthreads();
         if (!waited) {
@@ -255,9 +270,9 @@ __global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict
         }
         qf[((bj * NT + nt) * NG + g) * 32 + L] = make_uint2(w0, w1);
     }
-    for (int idx = threadIdx.x; idx < NT * NG * 4; idx += blockDim.x) {
-        const int hh = idx & 3, g = (idx >> 2) % NG, nt = (idx >> 2) / NG, hl = 4 * nt + hh;
-        qk[((bj * NT + nt) * NG + g) * 4 + hh] = hl < G ? sig[hl * NG + g] * (1.0f / (float)(1 << (2 * g))) : 0.0f;
+    for (int idx = threadIdx.x; idx < NT * (NG + 1) * 4; idx += blockDim.x) {
+        const int hh = idx & 3, g = (idx >> 2) % (NG + 1), nt = (idx >> 2) / (NG + 1), hl = 4 * nt + hh;
+        qk[((bj * NT + nt) * (NG + 1) + g) * 4 + hh] = hl < G ? (g < NG ? sig[hl * NG + g] : shd[hl]) : 0.0f;
     }
     for (int idx = threadIdx.x; idx < NT * 32; idx += blockDim.x) {
         const int L = idx & 31, nt = idx >> 5;
