@@ -288,10 +288,9 @@ __global__ void __launch_bounds__(512) k_quant_pack(
 // k_append_rows: appends of up to a few dozen rows per sequence (decode steps,
 // speculative or chunked appends).  One CTA of D threads per (group of RW
 // consecutive new rows of a sequence, kv head) -- RW = 1 when every sequence
-// appends one row (a decode step), else kRowsPerCta; thread c holds T_K's row c in
-// registers (read straight from global memory, all loads in flight at once)
-// and computes k'_c of every row of the group as interleaved independent
-// sums; warp g quantizes group g of each row.  Only the rows' own fields of
+// appends one row (a decode step), else kRowsPerCta; thread c reads T_K's row c
+// straight from global memory (the loads issued before any is used) and
+// computes k'_c of every row of the group as interleaved independent sums; warp g quantizes group g of each row.  Only the rows' own fields of
 // their (page, kv head) blocks are written: key code words (each holds codes
 // of one token) with plain stores, value code fields (words shared with
 // neighbouring tokens) with atomic and/or, scale/min/channel-0 entries with
@@ -313,8 +312,8 @@ __global__ void __launch_bounds__(D) k_append_rows(
     const int b = blockIdx.x / groups_per_seq, t0 = (blockIdx.x - b * groups_per_seq) * RW;
     const int c = threadIdx.x, warp = c >> 5, lane = c & 31;
     if (early_release) grid_dependents_launch();
-    // every load that depends only on (sequence, kv head, channel) is in
-    // flight before the first one is used: the lengths, the row offset of the
+    // every load that depends only on (sequence, kv head, channel) is issued
+    // before the first one is used: the lengths, the row offset of the
     // sequence and T_K's row c
     const int n = new_lens[b];
     const int L0 = seq_before[b];

@@ -69,9 +69,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
-// 16-byte load of read-only global data as a volatile asm statement: the
-// compiler keeps it where it stands (it may not sink it into a later loop),
-// so a batch of such loads is in flight at once.
+// 16-byte load of read-only global data through the non-coherent path, as an
+// asm statement: the front end issues it where it stands; how many such loads
+// the code generator keeps in flight depends on the registers it allots.
 __device__ __forceinline__ float4 ld_nc_f4(const float4 *ptr) {
     float4 v;
     asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
