@@ -10,7 +10,8 @@ Default workload: batch 4, 32 q / 8 kv heads, head_dim 128, 128K context,
 (411 MB) is larger than L2, so no flush is needed between steps.
 
 Prints ONE JSON line (rank 0).  --impl reference times the CPU oracle on a
-bounded sample of the same workload instead.
+bounded sample of the same workload instead.  --gpus N without an outer
+launcher re-runs this script under torch.distributed.run with N ranks.
 """
 from __future__ import annotations
 
@@ -18,7 +19,9 @@ import argparse
 import hashlib
 import json
 import os
+import socket
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -206,20 +209,23 @@ class Layer:
                           self.q_step, Q.DQK_BF16, w.batch, self.lens_d, self.table_d, self.max_pages, w.pct,
                           self.out, self.sel, self.ws, self.ws_bytes)
 
-    def step_staged(self, ev_attend):
-        """The same step as separate calls, with events around the attend
-        kernel (events between launches stop the overlap, so this pass only
-        times the kernel)."""
+    def decode(self):
+        """dqk_decode alone (the query and the cache as they are)."""
         Q, w = self.Q, self.w
-        Q.dqk_append(self.desc, self.k_step, self.v_step, Q.DQK_BF16, w.batch, self.ones, self.before, 1,
-                     self.table_d, self.max_pages)
-        args = (self.desc, self.q_step, Q.DQK_BF16, w.batch, self.lens_d, self.table_d, self.max_pages, w.pct,
-                self.out, self.sel, self.ws, self.ws_bytes)
-        Q.dqk_decode_prepare(*args)
-        ev_attend[0].record()
-        Q.dqk_decode_attend(*args)
-        ev_attend[1].record()
-        Q.dqk_decode_combine(*args)
+        Q.dqk_decode(self.desc, self.q_step, Q.DQK_BF16, w.batch, self.lens_d, self.table_d, self.max_pages, w.pct,
+                     self.out, self.sel, self.ws, self.ws_bytes)
+
+    def per_launch_ms(self, fn, n):
+        """Mean device time of one call of fn (one kernel launch), each call
+        bracketed by its own CUDA events on the current stream."""
+        torch = self.torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(self.dev)
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
 
     def step_e2e(self):
         """The same step from pinned host buffers: H2D inputs, D2H result."""
@@ -257,7 +263,7 @@ def run_dqk(args):
     rank, nranks, local = world()
     if nranks > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     from bit_kv_cache_dqk_b200 import inputs as I
@@ -270,51 +276,51 @@ def run_dqk(args):
         layer.step()
     torch.cuda.synchronize(dev)
     algo_bytes, per_tok = layer.algorithmic_bytes()
-
-    # device-timed steps (the fused step, as a serving loop runs it)
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if nranks > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     try:
         nvml_index = torch.cuda._get_nvml_device_index(dev)
     except Exception:
         nvml_index = local
+
     with ClockSampler(nvml_index) as clk:
+        # device-timed steps (one launch each, back to back, as a serving loop runs them)
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if nranks > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
         start.record()
         for _ in range(args.steps):
             layer.step()
         stop.record()
         torch.cuda.synchronize(dev)
-    if nranks > 1:
-        dist.barrier()
-    elapsed = start.elapsed_time(stop) / 1e3
-    agg = aggregate(tokens, elapsed, args.steps, nranks, dev)
+        if nranks > 1:
+            dist.barrier()
+        elapsed = start.elapsed_time(stop) / 1e3
+        agg = aggregate(tokens, elapsed, args.steps, nranks, dev)
 
-    # the attend kernel's own duration: the same steps as staged calls
-    ev_att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        layer.step_staged(ev_att[i])
-    torch.cuda.synchronize(dev)
-    attend_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev_att), dev)
+        # the kernel's own duration: each launch between its own events
+        step_ms = reduce_max(layer.per_launch_ms(layer.step, args.steps), dev)
+        for _ in range(3):
+            layer.decode()
+        decode_ms = reduce_max(layer.per_launch_ms(layer.decode, args.steps), dev)
 
-    # end to end from host buffers
-    for _ in range(2):
-        layer.step_e2e()
-    torch.cuda.synchronize(dev)
-    if nranks > 1:
-        dist.barrier()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record()
-    for _ in range(args.steps):
-        layer.step_e2e()
-    e2.record()
-    torch.cuda.synchronize(dev)
-    e2e = aggregate(tokens, s2.elapsed_time(e2) / 1e3, args.steps, nranks, dev)
+        # end to end from host buffers
+        for _ in range(2):
+            layer.step_e2e()
+        torch.cuda.synchronize(dev)
+        if nranks > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(args.steps):
+            layer.step_e2e()
+        e2.record()
+        torch.cuda.synchronize(dev)
+        e2e = aggregate(tokens, s2.elapsed_time(e2) / 1e3, args.steps, nranks, dev)
 
     peak, peak_kind = measured_peaks()
-    achieved = algo_bytes / (attend_ms / 1e3) / 1e9
-    traffic = recorded_traffic("k_attend", w.name)
+    achieved = algo_bytes / (step_ms / 1e3) / 1e9
+    decode_achieved = algo_bytes / (decode_ms / 1e3) / 1e9
+    traffic = recorded_traffic("k_decode", w.name)
     cpu = None
     if rank == 0 and nranks == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, layer.q_host.float().numpy(), args.cpu_seconds)
@@ -335,15 +341,18 @@ def run_dqk(args):
                              (layer.pool.numel() / 1e6)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": "k_attend", "kernel_ms": attend_ms,
+                         "kernel": "k_decode (the whole decode step: append + query prep + attend + merge)",
+                         "kernel_ms": step_ms,
                          "algorithmic_bytes_per_launch": algo_bytes,
                          "bytes_per_token_kv_head": per_tok},
+            "decode_call": {"kernel": "k_decode (dqk_decode: query prep + attend + merge)", "ms": decode_ms,
+                            "achieved_gbs": decode_achieved, "frac": decode_achieved / peak},
             "e2e": {"value": e2e["value"], "unit": "KV-tokens/s",
                     "h2d_bytes_per_step": int(layer.k_host.numel() * 2 + layer.v_host.numel() * 2 + layer.q_host.numel() * 2),
                     "d2h_bytes_per_step": int(layer.out_host.numel() * 4)},
-            "gpu_launches": 4 * args.steps,
-            "kernel_timing": "k_attend timed with CUDA events in a second pass of the same steps issued as "
-                             "separate calls (events between launches stop the append/query overlap)",
+            "gpu_launches": args.steps,
+            "kernel_timing": "one launch per step; kernel_ms = mean of CUDA-event times around each launch "
+                             "in a second pass of the same steps (decode_call: dqk_decode alone, same way)",
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }
@@ -351,6 +360,46 @@ def run_dqk(args):
     if nranks > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_cpu_selftest(args):
+    """The multi-rank path without a GPU (gloo): every rank times K steps of a
+    CPU stand-in step ((rank+1) ms of sleep), rank 0 prints the aggregate."""
+    import torch.distributed as dist
+    rank, nranks, _ = world()
+    if nranks > 1:
+        from datetime import timedelta
+        dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    for _ in range(args.warmup):
+        time.sleep(0.001 * (rank + 1))
+    if nranks > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(0.001 * (rank + 1))
+    agg = aggregate(1000, time.perf_counter() - t0, args.steps, nranks)
+    if nranks > 1:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps({"metric": "launcher self-test", "value": agg["value"], "unit": "tokens/s",
+                          "n_gpus": nranks, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": agg["ms_per_step"], "scaling": "weak"}), flush=True)
+    if nranks > 1:
+        dist.destroy_process_group()
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_under_torchrun(n: int, argv) -> int:
+    """--gpus N > 1 with no outer launcher: run this script as N ranks (one
+    per GPU of this node) under torch.distributed.run and return its status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={_free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 # ----------------------------------------------------------------------------
@@ -586,6 +635,7 @@ def run_append64(args):
 
 
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -598,10 +648,15 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true", help="sparsity x batch x context sweep vs the BF16 decode")
     ap.add_argument("--append64", action="store_true", help="time the 64-row append of the qwen workload")
     ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--cpu-selftest", action="store_true", help="the multi-rank launcher path on CPU (gloo)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_under_torchrun(args.gpus, argv))
+    if args.cpu_selftest:
+        run_cpu_selftest(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.sweep:
         run_sweep(args)

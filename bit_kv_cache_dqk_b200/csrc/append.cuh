@@ -285,32 +285,141 @@ __global__ void __launch_bounds__(512) k_quant_pack(
 }
 
 // ---------------------------------------------------------------------------
-// k_append_rows: appends of up to a few dozen rows per sequence (decode steps,
-// speculative or chunked appends).  One CTA of D threads per (group of RW
-// consecutive new rows of a sequence, kv head) -- RW = 1 when every sequence
-// appends one row (a decode step), else kRowsPerCta; thread c reads T_K's row c
-// straight from global memory (the loads issued before any is used) and
-// computes k'_c of every row of the group as interleaved independent sums; warp g quantizes group g of each row.  Only the rows' own fields of
-// their (page, kv head) blocks are written: key code words (each holds codes
-// of one token) with plain stores, value code fields (words shared with
-// neighbouring tokens) with atomic and/or, scale/min/channel-0 entries with
-// 16-bit stores.  Same arithmetic, hence the same bytes, as k_quant_pack.
+// Row appends of up to a few dozen rows per sequence (decode steps, speculative
+// or chunked appends).  D threads (thread c = channel c) handle up to RW
+// consecutive new rows of one sequence and kv head: k'_c of every row as
+// interleaved independent sums, warp g quantizes group g of each row.  Only
+// the rows' own fields of their (page, kv head) blocks are written: key code
+// words (each holds codes of one token) with plain stores, value code fields
+// (words shared with neighbouring tokens) with atomic and/or, scale/min/
+// channel-0 entries with 16-bit stores.  Same arithmetic, hence the same
+// bytes, as k_quant_pack.
 // ---------------------------------------------------------------------------
 constexpr int kDirectMaxNew = 64;   // dqk_append uses k_append_rows up to this many rows per sequence
 constexpr int kRowsPerCta = 4;
 
+template <int D, int NS, int RW>
+struct RowStoreScratch {
+    static constexpr int NG = D / kGroup;
+    uint32_t kimg[RW][D], kmask[RW][D], vimg[RW][D], vmask[RW][D];   // code regions: D words each
+    float rng[NS == 1 ? RW : 1][4][NG];
+};
+
+// Quantize rows i < nr (key k'_c = kp[i], value xv[i] of channel c) at cache
+// positions pos0 + i (physical pages phys[i]) and store their fields.  sync()
+// synchronises the D threads.
+template <int D, int NS, int RW, typename Sync>
+__device__ __forceinline__ void quantize_store_rows(const float (&kp)[RW], const float (&xv)[RW], const int (&phys)[RW],
+                                                    int nr, int pos0, int c, uint8_t *__restrict__ pool,
+                                                    long long num_pages, int hkv, int j, int v_ch0,
+                                                    RowStoreScratch<D, NS, RW> &S, Sync sync) {
+    constexpr int NG = D / kGroup;
+    const int warp = c >> 5, lane = c & 31;
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        S.kimg[i][c] = 0u;
+        S.kmask[i][c] = 0u;
+        S.vimg[i][c] = 0u;
+        S.vmask[i][c] = 0u;
+    }
+    const Layout L = make_layout(D, v_ch0, NS);
+    // group ranges: per warp (32 channels); with one group per row, combined
+    // over the row's NG warps through shared memory
+    float klo[RW], khi[RW], vlo[RW], vhi[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        // channel 0 keeps its sign; ranges read -0 as +0
+        warp_minmax(kp[i] + 0.0f, c == 0, klo[i], khi[i]);
+        warp_minmax(xv[i] + 0.0f, v_ch0 != 0 && c == 0, vlo[i], vhi[i]);
+        if constexpr (NS == 1) {
+            if (lane == 0) {
+                S.rng[i][0][warp] = klo[i];
+                S.rng[i][1][warp] = khi[i];
+                S.rng[i][2][warp] = vlo[i];
+                S.rng[i][3][warp] = vhi[i];
+            }
+        }
+    }
+    sync();
+    if constexpr (NS == 1) {
+#pragma unroll
+        for (int i = 0; i < RW; ++i)
+#pragma unroll
+            for (int w = 0; w < NG; ++w) {
+                klo[i] = fminf(klo[i], S.rng[i][0][w]);
+                khi[i] = fmaxf(khi[i], S.rng[i][1][w]);
+                vlo[i] = fminf(vlo[i], S.rng[i][2][w]);
+                vhi[i] = fmaxf(vhi[i], S.rng[i][3][w]);
+            }
+    }
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        if (i >= nr) break;                   // uniform
+        if (phys[i] < 0 || phys[i] >= num_pages) {   // uniform
+            if (c == 0) dqk_flag_error(kErrBounds);
+            continue;
+        }
+        const int slot = (pos0 + i) % kPage;
+        uint16_t *h16 = reinterpret_cast<uint16_t *>(pool + ((size_t)phys[i] * hkv + j) * L.bytes);
+        uint16_t ksh, kmh, vsh, vmh;
+        const int kc = quant_code(kp[i] + 0.0f, c == 0, klo[i], khi[i], ksh, kmh);
+        const int vc = quant_code(xv[i] + 0.0f, v_ch0 != 0 && c == 0, vlo[i], vhi[i], vsh, vmh);
+        if (NS == 1 ? c == 0 : lane == 0) {
+            const int g = NS == 1 ? 0 : warp;
+            h16[(L.ks >> 1) + kscale_idx(NS, slot, g)] = ksh;
+            h16[(L.km >> 1) + kscale_idx(NS, slot, g)] = kmh;
+            h16[(L.vs >> 1) + vscale_idx(NS, slot, g)] = vsh;
+            h16[(L.vm >> 1) + vscale_idx(NS, slot, g)] = vmh;
+        }
+        if (c == 0) {
+            h16[(L.k0 >> 1) + k0_idx(slot)] = f32_to_bf16_rne(kp[i]);
+            if (v_ch0) h16[(L.v0 >> 1) + slot] = f32_to_bf16_rne(xv[i]);
+        }
+        int off, bit;
+        kcode_pos(NG, slot, c, off, bit);
+        atomicOr(&S.kimg[i][off >> 2], (uint32_t)kc << bit);
+        atomicOr(&S.kmask[i][off >> 2], 3u << bit);
+        vcode_pos(NG, slot, c, off, bit);
+        atomicOr(&S.vimg[i][off >> 2], (uint32_t)vc << bit);
+        atomicOr(&S.vmask[i][off >> 2], 3u << bit);
+    }
+    sync();
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+        if (i >= nr) break;
+        if (phys[i] < 0 || phys[i] >= num_pages) continue;
+        uint8_t *blk = pool + ((size_t)phys[i] * hkv + j) * L.bytes;
+        uint32_t *kw = reinterpret_cast<uint32_t *>(blk + L.kc);
+        uint32_t *vw = reinterpret_cast<uint32_t *>(blk + L.vc);
+        const uint32_t km = S.kmask[i][c], vm = S.vmask[i][c];
+        if (km == 0xffffffffu) {
+            kw[c] = S.kimg[i][c];             // a key word holds codes of this token only
+        } else if (km) {
+            atomicAnd(&kw[c], ~km);
+            atomicOr(&kw[c], S.kimg[i][c]);
+        }
+        if (vm) {                             // value words are shared with neighbouring tokens
+            atomicAnd(&vw[c], ~vm);
+            atomicOr(&vw[c], S.vimg[i][c]);
+        }
+    }
+}
+
+// One CTA of D threads per (group of RW consecutive new rows of a sequence,
+// kv head) -- RW = 1 when every sequence appends one row, else kRowsPerCta;
+// thread c reads T_K's row c straight from global memory (the loads issued
+// before any is used).
 template <int D, int NS, int RW>
 __global__ void __launch_bounds__(D) k_append_rows(
     const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin, int dtype,
     const int *__restrict__ new_lens, const int *__restrict__ seq_before, const int *__restrict__ page_table,
     int max_pages, int groups_per_seq, uint8_t *__restrict__ pool, long long num_pages, int hkv, int v_ch0,
     int early_release) {
-    constexpr int NG = D / kGroup;
     __shared__ double xs[RW][D];
-    __shared__ uint32_t kimg[RW][D], kmask[RW][D], vimg[RW][D], vmask[RW][D];   // code regions: D words each
+    __shared__ RowStoreScratch<D, NS, RW> S;
     const int j = blockIdx.y;
     const int b = blockIdx.x / groups_per_seq, t0 = (blockIdx.x - b * groups_per_seq) * RW;
-    const int c = threadIdx.x, warp = c >> 5, lane = c & 31;
+    const int c = threadIdx.x, lane = c & 31;
     if (early_release) grid_dependents_launch();
     // every load that depends only on (sequence, kv head, channel) is issued
     // before the first one is used: the lengths, the row offset of the
@@ -337,10 +446,6 @@ __global__ void __launch_bounds__(D) k_append_rows(
         xv[i] = load_elem(vin, dtype, base + c);
         const int page = (L0 + t) / kPage;
         phys[i] = (L0 >= 0 && page < max_pages) ? page_table[(size_t)b * max_pages + page] : -1;
-        kimg[i][c] = 0u;
-        kmask[i][c] = 0u;
-        vimg[i][c] = 0u;
-        vmask[i][c] = 0u;
     }
     __syncthreads();
     // k'_c = sum_i T_K[c][i] x_i, ascending i, exact products summed in fp64
@@ -355,88 +460,11 @@ __global__ void __launch_bounds__(D) k_append_rows(
 #pragma unroll
             for (int i = 0; i < RW; ++i) acc[i] = fma(t4[e], xs[i][4 * u + e], acc[i]);
     }
-    const Layout L = make_layout(D, v_ch0, NS);
-    // group ranges: per warp (32 channels); with one group per row, combined
-    // over the row's NG warps through shared memory
-    __shared__ float rng[NS == 1 ? RW : 1][4][NG];
-    float kp[RW], klo[RW], khi[RW], vlo[RW], vhi[RW];
+    float kp[RW];
 #pragma unroll
-    for (int i = 0; i < RW; ++i) {
-        kp[i] = __double2float_rn(acc[i]);    // channel 0 keeps its sign; ranges read -0 as +0
-        warp_minmax(kp[i] + 0.0f, c == 0, klo[i], khi[i]);
-        warp_minmax(xv[i] + 0.0f, v_ch0 != 0 && c == 0, vlo[i], vhi[i]);
-        if constexpr (NS == 1) {
-            if (lane == 0) {
-                rng[i][0][warp] = klo[i];
-                rng[i][1][warp] = khi[i];
-                rng[i][2][warp] = vlo[i];
-                rng[i][3][warp] = vhi[i];
-            }
-        }
-    }
-    if constexpr (NS == 1) {
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < RW; ++i)
-#pragma unroll
-            for (int w = 0; w < NG; ++w) {
-                klo[i] = fminf(klo[i], rng[i][0][w]);
-                khi[i] = fmaxf(khi[i], rng[i][1][w]);
-                vlo[i] = fminf(vlo[i], rng[i][2][w]);
-                vhi[i] = fmaxf(vhi[i], rng[i][3][w]);
-            }
-    }
-#pragma unroll
-    for (int i = 0; i < RW; ++i) {
-        if (i >= nr) break;                   // uniform
-        if (phys[i] < 0 || phys[i] >= num_pages) {   // uniform
-            if (c == 0) dqk_flag_error(kErrBounds);
-            continue;
-        }
-        const int slot = (L0 + t0 + i) % kPage;
-        uint16_t *h16 = reinterpret_cast<uint16_t *>(pool + ((size_t)phys[i] * hkv + j) * L.bytes);
-        uint16_t ksh, kmh, vsh, vmh;
-        const int kc = quant_code(kp[i] + 0.0f, c == 0, klo[i], khi[i], ksh, kmh);
-        const int vc = quant_code(xv[i] + 0.0f, v_ch0 != 0 && c == 0, vlo[i], vhi[i], vsh, vmh);
-        if (NS == 1 ? c == 0 : lane == 0) {
-            const int g = NS == 1 ? 0 : warp;
-            h16[(L.ks >> 1) + kscale_idx(NS, slot, g)] = ksh;
-            h16[(L.km >> 1) + kscale_idx(NS, slot, g)] = kmh;
-            h16[(L.vs >> 1) + vscale_idx(NS, slot, g)] = vsh;
-            h16[(L.vm >> 1) + vscale_idx(NS, slot, g)] = vmh;
-        }
-        if (c == 0) {
-            h16[(L.k0 >> 1) + k0_idx(slot)] = f32_to_bf16_rne(kp[i]);
-            if (v_ch0) h16[(L.v0 >> 1) + slot] = f32_to_bf16_rne(xv[i]);
-        }
-        int off, bit;
-        kcode_pos(NG, slot, c, off, bit);
-        atomicOr(&kimg[i][off >> 2], (uint32_t)kc << bit);
-        atomicOr(&kmask[i][off >> 2], 3u << bit);
-        vcode_pos(NG, slot, c, off, bit);
-        atomicOr(&vimg[i][off >> 2], (uint32_t)vc << bit);
-        atomicOr(&vmask[i][off >> 2], 3u << bit);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < RW; ++i) {
-        if (i >= nr) break;
-        if (phys[i] < 0 || phys[i] >= num_pages) continue;
-        uint8_t *blk = pool + ((size_t)phys[i] * hkv + j) * L.bytes;
-        uint32_t *kw = reinterpret_cast<uint32_t *>(blk + L.kc);
-        uint32_t *vw = reinterpret_cast<uint32_t *>(blk + L.vc);
-        const uint32_t km = kmask[i][c], vm = vmask[i][c];
-        if (km == 0xffffffffu) {
-            kw[c] = kimg[i][c];               // a key word holds codes of this token only
-        } else if (km) {
-            atomicAnd(&kw[c], ~km);
-            atomicOr(&kw[c], kimg[i][c]);
-        }
-        if (vm) {                             // value words are shared with neighbouring tokens
-            atomicAnd(&vw[c], ~vm);
-            atomicOr(&vw[c], vimg[i][c]);
-        }
-    }
+    for (int i = 0; i < RW; ++i) kp[i] = __double2float_rn(acc[i]);
+    quantize_store_rows<D, NS, RW>(kp, xv, phys, nr, L0 + t0, c, pool, num_pages, hkv, j, v_ch0, S,
+                                   [] { __syncthreads(); });
 }
 
 }  // namespace dqk

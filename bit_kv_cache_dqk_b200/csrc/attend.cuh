@@ -1,7 +1,9 @@
-// attend.cuh -- k_attend: split-K pruned-channel attention over the INT2 paged
-// cache ("Throughput on SGLang": pruning removes 40 % of key channels from
-// reads, quantization cuts storage to 2 bits per value), and k_combine, the
-// cross-split log-sum-exp merge.
+// attend.cuh -- the streaming part of the decode kernel: split-K
+// pruned-channel attention over the INT2 paged cache ("Throughput on SGLang":
+// pruning removes 40 % of key channels from reads, quantization cuts storage
+// to 2 bits per value) -- unit bookkeeping, the producer warp, and the
+// per-page consumer steps -- and k_merge, the merge of context-parallel
+// records.
 //
 // Work split: the cache is a sequence of units (pages of one run; a run is a
 // (sequence, chunk of <= 8 kv heads)).  CTA c of C owns units
@@ -154,7 +156,10 @@ __device__ __forceinline__ CtaUnits cta_units(const int *seq_lens, int nchunks, 
     return cu;
 }
 
-// Partial record of (slot = CTA + run, warp pair index pi, kv head jl, query head hh).
+// Partial record of (slot = CTA + run, warp pair index pi, kv head jl, query head hh):
+// kRecHead floats (m, l and two unused) then o[D], so o starts 16-byte aligned.
+constexpr int kRecHead = 4;
+__host__ __device__ constexpr int rec_stride(int D) { return kRecHead + D; }
 __host__ __device__ __forceinline__ size_t record_index(int slot, int pi, int jl, int hh, int pw, int hc, int G) {
     return (((size_t)slot * pw + pi) * hc + jl) * G + hh;
 }
@@ -529,7 +534,7 @@ __device__ __forceinline__ void init_records(const AttendParams &p, const CtaUni
     int np = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     while (r < R && ur < u1) {
         if (np > 0 && lane < G) {
-            float *rec = p.part + record_index(slot_base + r, pi, jl, lane, p.pw, p.hc, G) * (2 + D);
+            float *rec = p.part + record_index(slot_base + r, pi, jl, lane, p.pw, p.hc, G) * rec_stride(D);
             rec[0] = -INFINITY;
             rec[1] = 0.0f;
         }
@@ -539,7 +544,7 @@ __device__ __forceinline__ void init_records(const AttendParams &p, const CtaUni
     }
 }
 
-// The producer warp of the attend kernels: brings the CTA's units [u0, u1)
+// The producer warp of the decode kernels: brings the CTA's units [u0, u1)
 // into the ring, pps pages (each hc blocks, one bulk copy) per stage, marks
 // which page slots of a stage hold a page, and never leaves with copies in
 // flight.  Lane l fills page slots l and l + 32 of a stage (pps <= 64).  The
@@ -549,22 +554,38 @@ __device__ __forceinline__ void init_records(const AttendParams &p, const CtaUni
 // (the packed cache; the BF16 comparison streams without a policy, which
 // measured faster for it).  Waits are bounded; a stuck pipeline sets the
 // abort flag.
+//
+// The gate holds back two kinds of copies until the consumers have finished
+// the CTA's prologue (its `opened` mbarrier completes once): the first fill
+// of the stages from `scratch_first` on, whose memory the prologue works in,
+// and, when the same
+// launch appends rows to the cache (new_lens non-null), every page at or past
+// the first page an append of this call touches.
 constexpr int kMaxPagesPerStage = 64;
+
+struct ProducerGate {
+    uint64_t *opened;          // completed by the consumers at the end of the CTA's prologue
+    int scratch_first;         // first stage used as prologue scratch (>= the stage count: none)
+    const int *new_lens;       // rows this launch appends per sequence (null: none)
+    const int *seq_before;     // their first position
+    int stall;                 // test only: CTA 0 never arms its second stage
+    uint64_t wait_ns;          // bound of every wait
+};
 
 struct ProducerSlots {
     int phys[2], chunk[2];   // raw page-table entry and kv-head chunk of slot lane + 32k
     bool in[2];              // the slot holds a unit of the CTA that maps to a page-table entry
+    bool gated[2];           // the page is written by this launch's append
 };
 
 template <bool kEvictFirst>
 __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned char *stage_mem, uint64_t *full,
                                                 uint64_t *empty, unsigned char *valid, volatile int *abort_flag,
                                                 int S, uint32_t stage_bytes, int kStageBlocks, const CtaUnits &cu,
-                                                int iters, int lane) {
+                                                int iters, int lane, const ProducerGate &gate) {
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
     const int u0 = cu.u0, u1 = cu.u1;
-    grid_dependents_launch();   // the combine kernel may start its prologue
     if (iters == 0) return;
     if (pps < 1 || pps > kMaxPagesPerStage || pps > kStageBlocks) {   // host plans never do this
         if (lane == 0) {
@@ -586,6 +607,7 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
         for (int k = 0; k < 2; ++k) {
             const int slot = 32 * k + lane, u = base + slot;
             f.in[k] = false;
+            f.gated[k] = false;
             f.phys[k] = -1;
             f.chunk[k] = 0;
             if (slot < pps && u < u1) {
@@ -599,6 +621,7 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
                     f.chunk[k] = rr - b * p.nchunks;
                     f.in[k] = true;
                     if (page < p.max_pages) f.phys[k] = p.page_table[(size_t)b * p.max_pages + page];
+                    if (gate.new_lens && gate.new_lens[b] > 0) f.gated[k] = page >= gate.seq_before[b] / kPage;
                 }
             }
         }
@@ -612,17 +635,36 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
     ProducerSlots cur = fetch(0);
     int it = 0, stage = 0;
     uint32_t phase = 0;
+    bool opened = gate.opened == nullptr;
     for (; it < iters; ++it) {
         ProducerSlots nxt = cur;
         if (it + 1 < iters) nxt = fetch(it + 1);
         int good = 1;
-        if (lane == 0) good = mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs, 2000u) && !*abort_flag;
+        if (lane == 0) good = mbar_wait_bounded(&empty[stage], phase ^ 1u, gate.wait_ns, 2000u) && !*abort_flag;
+        const bool need_open =
+            !opened && (stage >= gate.scratch_first || __any_sync(0xffffffffu, cur.gated[0] || cur.gated[1]));
+        if (need_open && lane == 0 && good) good = mbar_wait_bounded(gate.opened, 0u, gate.wait_ns, 2000u);
         if (!__shfl_sync(0xffffffffu, good, 0)) {
             if (lane == 0) {
                 *abort_flag = 1;
                 dqk_flag_error(kErrTimeout);
             }
             break;
+        }
+        if (need_open) {
+            // the prologue's shared-memory scratch and the appended rows (global
+            // memory) were written through the generic proxy
+            fence_proxy_async_shared();
+            fence_proxy_async_global();
+            opened = true;
+        }
+        if (gate.stall && blockIdx.x == 0 && it == 1) {   // test only: this stage is never armed
+            cur = nxt;
+            if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+            }
+            continue;
         }
         long long off[2];
         bool have[2];
@@ -656,447 +698,7 @@ __device__ __forceinline__ void attend_producer(const AttendParams &p, unsigned 
     // never leave with copies in flight (exit path: wait, bounded, for the last round of each stage)
     if (lane == 0)
         for (int k = it - 1; k >= 0 && k >= it - S; --k)
-            (void)mbar_wait_bounded(&full[k % S], (uint32_t)(k / S) & 1u, kWaitLimitNs);
-}
-
-template <int D, int G, bool VCH0, int NS>
-__global__ void __launch_bounds__(attend_threads(G), 1) k_attend(const AttendParams p) {
-    using T = AttendTile<D, G>;
-    constexpr int kConsumerWarps = attend_warps(G), kStageBlocks = attend_stage_blocks(G);
-    constexpr int BPW = attend_pages_per_warp(G);
-    static_assert(BPW >= 2 && BPW <= 8, "pages per warp");
-    constexpr int NG = T::NG, NT = T::NT, NM = T::NM;
-    extern __shared__ __align__(128) unsigned char attend_smem[];
-    const int S = p.stages;
-    const uint32_t stage_bytes = (uint32_t)(kStageBlocks * p.bb);
-    unsigned char *stage_mem = attend_smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(attend_smem + (size_t)S * stage_bytes);
-    uint64_t *empty = full + kMaxStages;
-    unsigned char *valid = reinterpret_cast<unsigned char *>(empty + kMaxStages);   // [kMaxStages][kStageBlocks]
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(valid + kMaxStages * kStageBlocks);
-    // per consumer warp: QK B fragments [NT][NG][32] uint2, head constants [NT][NG][4] float4
-    unsigned char *frag_mem = valid + kMaxStages * kStageBlocks + 16;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int R = p.batch * p.nchunks;
-    const int pps = p.pps;
-
-    // The producer initialises the ring's barriers and announces them on named
-    // barrier 1 without waiting; every warp works out the CTA's unit range on
-    // its own, so the producer's first copies wait on nothing but the lengths
-    // and the page table.  Consumers wait on barrier 1 before their first use
-    // of the ring.
-    constexpr int kRingReady = 1;
-    if (warp == kConsumerWarps) {
-        if (lane == 0) {
-            for (int s = 0; s < S; ++s) {
-                mbar_init(&full[s], 1);
-                mbar_init(&empty[s], kConsumerWarps);
-            }
-            *abort_flag = 0;
-            fence_mbar_init();
-        }
-        __syncwarp();
-        named_bar_arrive(kRingReady, attend_threads(G));
-    }
-    const CtaUnits cu = cta_units(p.seq_lens, p.nchunks, R, blockIdx.x, p.num_ctas, lane);
-    const int u0 = cu.u0, u1 = cu.u1;
-    const int nunits = u1 - u0;
-    const int iters = (nunits + pps - 1) / pps;
-
-    if (warp == kConsumerWarps) {
-        attend_producer<true>(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kStageBlocks, cu, iters,
-                              lane);
-        return;
-    }
-
-    // ---------------------------------------------------------------- consumers
-    // warp: kv head jl of the chunk, page group pi of each stage (slots BPW*pi ..)
-    const int jl = warp % p.hc, pi = warp / p.hc;
-    const int gid = lane >> 2, tig = lane & 3;
-    const int slot_base = (int)blockIdx.x;
-
-    if (nunits > 0) init_records(p, cu, slot_base, pi, jl, G, D, lane);
-    named_bar_sync(kRingReady, attend_threads(G));
-    if (iters == 0) return;
-    grid_dependency_wait();     // query fragments come from k_qprep
-
-    int r = cu.r, ur = cu.ur;
-    int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-    int cur_run = -1, run_end = -1, partial_u = -1, nv_last = kPage;
-
-    WarpState<D, G> st;
-    LaneOffsets lo;
-    lo.lane16 = lane * 16;
-    lo.gid8 = gid * 8;
-    lo.kmin = gid * 2 * NG + (tig & (NG / 2 - 1)) * 4;   // in range for every lane (B rows past 2 NG are 0)
-    lo.gid4 = gid * 4;
-    lo.tig16 = tig * 16;
-    lo.vmin = (tig * NS + (gid < NS ? gid : 0)) * 4;
-    lo.srcA = (2 * tig) * 4 + (gid >> 1);
-    {
-        unsigned char *mine = frag_mem + (size_t)warp * NT * NG * (32 * 8 + 4 * 16);
-        lo.sq = smem_addr(mine) + lane * 8;
-        lo.sk = smem_addr(mine + NT * NG * 32 * 8) + tig * 16;
-    }
-    lo.ones_lane = gid == NS ? 0x3C003C00u : 0u;
-    lo.vmin_mask = gid < NS ? 0xffffffffu : 0u;
-
-    auto start_run = [&](int rr) {
-        const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
-        const int j = chunk * p.hc + jl;
-        const size_t bj = (size_t)b * p.hkv + j;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                const uint2 qb = p.qf[((bj * NT + nt) * NG + g) * 32 + lane];
-                const float pg = p.qk[((bj * NT + nt) * (NG + 1) + g) * 4 + tig];
-                const float2 kp = make_float2(pg, -(kMagicF + kMagicLoF) * pg);   // exact: power-of-two p_g
-                if constexpr (WarpState<D, G>::kRegFrags) {
-                    st.qb[g] = qb;
-                    st.kp[g] = kp;
-                } else {
-                    st_s64(lo.sq + (nt * NG + g) * 256, qb);
-                    if (gid == 0)
-                        st_s64(lo.sk + (nt * NG + g) * 64, make_uint2(__float_as_uint(kp.x), __float_as_uint(kp.y)));
-                }
-            }
-            st.sgh[nt] = p.qk[((bj * NT + nt) * (NG + 1) + NG) * 4 + tig];
-            __syncwarp();
-            st.qmin[nt] = p.qm[(bj * NT + nt) * 32 + lane];
-            const int hh = 4 * nt + tig;
-            st.q0v[nt] = hh < G ? p.q0[(size_t)b * p.hq + j * G + hh] : 0.0f;
-            st.m_run[nt] = -INFINITY;
-#pragma unroll
-            for (int m = 0; m < NM; ++m)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) st.oacc[nt][m][e] = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) st.macc[nt][e] = 0.0f;
-        }
-        cur_run = rr;
-    };
-
-    auto finish_run = [&](int rr) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            float minterm[NS];
-#pragma unroll
-            for (int g = 0; g < NS; ++g) minterm[g] = __shfl_sync(0xffffffffu, st.macc[nt][0], g * 4 + tig);
-            const float l = __shfl_sync(0xffffffffu, st.macc[nt][0], NS * 4 + tig);
-            const float v0t = __shfl_sync(0xffffffffu, st.macc[nt][0], (NS + 1) * 4 + tig);
-            const int hh = 4 * nt + tig;
-            if (hh < G) {
-                float *rec = p.part + record_index(slot_base + rr, pi, jl, hh, p.pw, p.hc, G) * (2 + D);
-                if (gid == 0) {
-                    rec[0] = st.m_run[nt];
-                    rec[1] = l;
-                }
-#pragma unroll
-                for (int m = 0; m < NM; ++m) {
-                    const int c0 = 16 * m + gid, c1 = c0 + 8;
-                    const float mt = minterm[NS == 1 ? 0 : (m >> 1)];
-                    const float f = vfield_scale<NG>(m);
-                    rec[2 + c0] = (VCH0 && c0 == 0) ? v0t : fmaf(st.oacc[nt][m][0], f, mt);
-                    rec[2 + c1] = fmaf(st.oacc[nt][m][2], f, mt);
-                }
-            }
-        }
-    };
-
-    // move to the run holding unit u (u >= run_end)
-    auto switch_run = [&](int u) {
-        if (cur_run >= 0) finish_run(cur_run);
-        while (r < R && u >= ur + npr) {
-            ur += npr;
-            ++r;
-            npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
-        }
-        start_run(r);
-        run_end = ur + npr;
-        const int Lb = p.seq_lens[r / p.nchunks];
-        partial_u = (Lb & (kPage - 1)) ? run_end - 1 : -1;
-        nv_last = Lb - (npr - 1) * kPage;
-    };
-
-    // the first run's query fragments load while the first pages are in flight
-    switch_run(u0 + BPW * pi < u1 ? u0 + BPW * pi : u0);
-
-    bool ok = true;
-    int stage = 0;
-    uint32_t phase = 0;
-    const uint32_t blk_a = smem_addr(stage_mem) + (uint32_t)((BPW * pi * p.hc + jl) * p.bb);
-    const uint32_t page_gap = (uint32_t)(p.hc * p.bb);
-    // n (1 .. BPW-1) full pages of one run at shared addresses base + q * page_gap
-    auto consume_batch = [&](int n, uint32_t base) {
-        if constexpr (BPW == 4) {
-            if (n == 3) {
-                const uint32_t sb3[3] = {base, base + page_gap, base + 2 * page_gap};
-                consume<D, G, VCH0, NS, 3, false>(sb3, kPage, st, lane, lo);
-                return;
-            }
-            if (n == 2) {
-                const uint32_t sb2[2] = {base, base + page_gap};
-                consume<D, G, VCH0, NS, 2, false>(sb2, kPage, st, lane, lo);
-                return;
-            }
-        }
-        const uint32_t sb1[1] = {base};
-        consume<D, G, VCH0, NS, 1, false>(sb1, kPage, st, lane, lo);
-    };
-
-    const uint32_t valid_addr = smem_addr(valid) + BPW * pi;
-    constexpr uint32_t kAllValid = (1u << BPW) - 1u;
-    for (int it = 0; it < iters; ++it) {
-        if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
-            if (lane == 0) {
-                *abort_flag = 1;
-                dqk_flag_error(kErrTimeout);
-            }
-            ok = false;
-            break;
-        }
-        const int ua = u0 + it * pps + BPW * pi;
-        if (ua < u1) {
-            const uint32_t sa = blk_a + (uint32_t)stage * stage_bytes;
-            const int ul = ua + BPW - 1;
-            // flags of the warp's page slots (one byte each), as a bit mask
-            const uint32_t va = valid_addr + stage * kStageBlocks;
-            uint32_t vv = 0;
-            if constexpr (BPW == 4) {
-                const uint32_t w = ld_s32(va);
-                vv = (w & 1u) | ((w >> 7) & 2u) | ((w >> 14) & 4u) | ((w >> 21) & 8u);
-            } else if constexpr (BPW == 2) {
-                const uint32_t w = ld_s16(va);
-                vv = (w & 1u) | ((w >> 7) & 2u);
-            } else {
-#pragma unroll
-                for (int q = 0; q < BPW; ++q) vv |= ld_s8(va + q) << q;
-            }
-            if (ua >= run_end) switch_run(ua);
-            if (ul < run_end && ul < u1 && !(partial_u >= ua && partial_u <= ul) && vv == kAllValid) {
-                uint32_t sbb[BPW];
-#pragma unroll
-                for (int q = 0; q < BPW; ++q) sbb[q] = sa + q * page_gap;
-                consume<D, G, VCH0, NS, BPW, false>(sbb, kPage, st, lane, lo);
-            } else if (vv == kAllValid && ul < u1 && run_end <= ul && partial_u < 0) {
-                // the pages cross one run boundary, the run's last page is full:
-                // the pages of each run as one batch
-                const int k = run_end - ua;   // 1 .. BPW-1 pages of the current run
-                consume_batch(k, sa);
-                switch_run(run_end);
-                if (ul < run_end && !(partial_u >= ua + k && partial_u <= ul)) {
-                    consume_batch(BPW - k, sa + (uint32_t)k * page_gap);
-                } else {
-#pragma unroll
-                    for (int q = 1; q < BPW; ++q) {
-                        if (q < k) continue;
-                        const int uq = ua + q;
-                        if (uq >= run_end) switch_run(uq);
-                        const uint32_t s1[1] = {sa + q * page_gap};
-                        if (uq == partial_u) consume<D, G, VCH0, NS, 1, true>(s1, nv_last, st, lane, lo);
-                        else consume<D, G, VCH0, NS, 1, false>(s1, kPage, st, lane, lo);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < BPW; ++q) {
-                    const int uq = ua + q;
-                    if (uq >= u1) break;
-                    if (uq >= run_end) switch_run(uq);
-                    if ((vv >> q) & 1u) {
-                        const uint32_t s1[1] = {sa + q * page_gap};
-                        if (uq == partial_u) consume<D, G, VCH0, NS, 1, true>(s1, nv_last, st, lane, lo);
-                        else consume<D, G, VCH0, NS, 1, false>(s1, kPage, st, lane, lo);
-                    }
-                }
-            }
-        }
-        __syncwarp();
-        mbar_arrive_if(&empty[stage], lane == 0);
-        if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-        }
-    }
-    if (ok && cur_run >= 0) finish_run(cur_run);
-}
-
-// ---------------------------------------------------------------------------
-// log-sum-exp combine: out[b][h] = sum_i o_i 2^(m_i - m*) / sum_i l_i 2^(m_i - m*)
-// over the records of every CTA (and page slot) that held pages of (b, h).
-// ---------------------------------------------------------------------------
-constexpr int kCombineChunk = 96;      // records read per pass
-constexpr int kCombineThreads = 256;
-
-// One CTA per (sequence, query head).  The record indices are worked out
-// before the attend kernel has finished.  Each pass then reads a chunk of
-// records in one round -- (m_i, l_i) into shared memory, and thread (slice,
-// channel) the channel of records i = slice (mod slices) into registers --
-// forms the weights 2^(m_i - m*) once per record, and accumulates.  The
-// running max moves from chunk to chunk with an exact rescale.  Maxima and
-// denominators are reduced in a fixed order, so the result does not depend on
-// scheduling.
-//
-// partial_out: instead of the normalized output, the merged record itself --
-// (m, l, o[D]) per (sequence, query head), m in log2 units -- for a later merge
-// with the records of other context ranges (dqk_merge_partials).
-template <int D>
-__global__ void __launch_bounds__(kCombineThreads) k_combine(const int *__restrict__ seq_lens, int batch, int hq,
-                                                             int hkv, int hc, int pw, int nchunks, int num_ctas,
-                                                             const float *__restrict__ part, float *__restrict__ out,
-                                                             int partial_out) {
-    constexpr int kSlices = kCombineThreads / D;
-    constexpr int kPer = kCombineChunk / kSlices;   // records of a chunk per thread
-    constexpr int kWarps = kCombineThreads / 32;
-    static_assert(kCombineChunk <= kCombineThreads, "one record per thread when forming weights");
-    __shared__ long long sh_U, sh_ur;
-    __shared__ int sh_np;
-    __shared__ int sh_rec[kCombineChunk];   // record index of slot i of the chunk, -1 for none
-    __shared__ float sh_m[kCombineChunk], sh_l[kCombineChunk], sh_w[kCombineChunk];
-    __shared__ float sh_red[kWarps];
-    __shared__ float sh_acc[kSlices][D];
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int G = hq / hkv, j = h / G, chunk = j / hc, jl = j % hc, hh = h % G;
-    const int r = b * nchunks + chunk, R = batch * nchunks;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int ch = threadIdx.x % D, slice = threadIdx.x / D;
-    if (warp == 0) {
-        const long long U = warp_total_units(seq_lens, nchunks, R, lane);
-        long long base = 0;   // start unit of run r
-        for (int r0 = 0; r0 < r; r0 += 32) {
-            const int rr = r0 + lane;
-            long long np = rr < r ? run_pages(seq_lens, nchunks, rr) : 0;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) np += __shfl_xor_sync(0xffffffffu, np, o);
-            base += np;
-        }
-        if (lane == 0) {
-            sh_U = U;
-            sh_ur = base;
-            sh_np = run_pages(seq_lens, nchunks, r);
-        }
-    }
-    __syncthreads();
-    const long long U = sh_U, ur = sh_ur;
-    const int np = sh_np;
-    float *o = out + ((size_t)b * hq + h) * D;
-    // records of this (run, head): CTAs cf..cl that own units of the run (CTAs
-    // with an empty unit range wrote none), each with pw page-slot records
-    const int cf = np > 0 ? (int)cta_of_unit(ur, U, num_ctas) : 0;
-    const int cl = np > 0 ? (int)cta_of_unit(ur + np - 1, U, num_ctas) : -1;
-    const int nrec = (cl - cf + 1) * pw;
-    auto index_chunk = [&](int i0) {
-        for (int i = threadIdx.x; i < kCombineChunk; i += blockDim.x) {
-            int ri = -1;
-            if (i0 + i < nrec) {
-                const int c = cf + (i0 + i) / pw, s = (i0 + i) % pw;
-                if ((long long)c * U / num_ctas < ((long long)c + 1) * U / num_ctas)
-                    ri = (int)record_index(c + r, s, jl, hh, pw, hc, G);
-            }
-            sh_rec[i] = ri;
-        }
-    };
-    index_chunk(0);
-    __syncthreads();
-    {   // the first chunk's record lines (and their address translations)
-        // are requested while k_attend finishes; values are read after the wait
-        const int n0 = min(kCombineChunk, nrec);
-        if (threadIdx.x < n0 && sh_rec[threadIdx.x] >= 0) prefetch_l2(part + (size_t)sh_rec[threadIdx.x] * (2 + D));
-        if (lane == 0 || lane == 31)
-            for (int k = 0; k < kPer; ++k) {
-                const int i = slice + kSlices * k;
-                if (i < n0 && sh_rec[i] >= 0) prefetch_l2(part + (size_t)sh_rec[i] * (2 + D) + 2 + ch);
-            }
-    }
-    grid_dependency_wait();     // partial records come from k_attend
-    float *pr = out + ((size_t)b * hq + h) * (D + 2);   // partial record of (b, h)
-    if (np == 0) {
-        if (slice == 0) {
-            if (partial_out) {
-                pr[2 + ch] = 0.0f;
-                if (ch == 0) {
-                    pr[0] = -INFINITY;
-                    pr[1] = 0.0f;
-                }
-            } else {
-                o[ch] = 0.0f;
-            }
-        }
-        return;
-    }
-    float mrun = -INFINITY, acc = 0.0f, dsum = 0.0f;
-    for (int i0 = 0; i0 < nrec; i0 += kCombineChunk) {
-        const int n = min(kCombineChunk, nrec - i0);
-        if (i0 > 0) {
-            __syncthreads();   // the previous chunk has been read
-            index_chunk(i0);
-            __syncthreads();
-        }
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const int ri = sh_rec[i];
-            sh_m[i] = ri >= 0 ? part[(size_t)ri * (2 + D)] : -INFINITY;
-            sh_l[i] = ri >= 0 ? part[(size_t)ri * (2 + D) + 1] : 0.0f;
-        }
-        float ov[kPer];
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            const int i = slice + kSlices * k;
-            const int ri = i < n ? sh_rec[i] : -1;
-            ov[k] = ri >= 0 ? part[(size_t)ri * (2 + D) + 2 + ch] : 0.0f;
-        }
-        __syncthreads();
-        // chunk max (every warp, same order), weights once per record
-        float cm = -INFINITY;
-        for (int i = lane; i < n; i += 32) cm = fmaxf(cm, sh_m[i]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
-        const float mnew = fmaxf(mrun, cm);
-        if (mnew == -INFINITY) continue;   // no tokens yet (uniform)
-        float dpart = 0.0f;
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const float mi = sh_m[i];
-            const float wi = mi == -INFINITY ? 0.0f : exp2f(mi - mnew);
-            sh_w[i] = wi;
-            dpart = fmaf(wi, sh_l[i], dpart);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) dpart += __shfl_xor_sync(0xffffffffu, dpart, off);
-        if (lane == 0) sh_red[warp] = dpart;
-        __syncthreads();
-        float dchunk = 0.0f;
-#pragma unroll
-        for (int k = 0; k < kWarps; ++k) dchunk += sh_red[k];
-        const float alpha = exp2f(mrun - mnew);   // 0 while mrun is -inf
-        dsum = dsum * alpha + dchunk;
-        acc *= alpha;
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            const int i = slice + kSlices * k;
-            if (i < n) {
-                const float wi = sh_w[i];
-                if (wi != 0.0f) acc = fmaf(wi, ov[k], acc);   // empty records hold no o values
-            }
-        }
-        mrun = mnew;
-    }
-    sh_acc[slice][ch] = acc;
-    __syncthreads();
-    if (slice == 0) {
-        float num = 0.0f;
-#pragma unroll
-        for (int k = 0; k < kSlices; ++k) num += sh_acc[k][ch];
-        if (partial_out) {
-            pr[2 + ch] = num;
-            if (ch == 0) {
-                pr[0] = mrun;
-                pr[1] = dsum;
-            }
-        } else {
-            o[ch] = dsum > 0.0f ? num / dsum : 0.0f;
-        }
-    }
+            (void)mbar_wait_bounded(&full[k % S], (uint32_t)(k / S) & 1u, gate.wait_ns);
 }
 
 // ---------------------------------------------------------------------------

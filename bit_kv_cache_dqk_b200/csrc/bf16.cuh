@@ -11,6 +11,7 @@
 
 #include "attend.cuh"
 #include "common.cuh"
+#include "decode.cuh"
 #include "ptx.cuh"
 
 namespace dqk {
@@ -71,33 +72,16 @@ __global__ void __launch_bounds__(2 * D / 8) k_append_b16(const void *__restrict
 
 // ---------------------------------------------------------------------------
 // query fragments: qs = q * log2(e)/sqrt(d) as bf16 hi + lo pieces in the
-// B operand of the m16n8k16 score tiles: qb [B*Hkv][NT][D/16][32] uint2, per
-// lane the registers of k-step s (channels 16s + 2*tig (+1), +8) for column
-// n = gid: query head 4*nt + gid/2, piece gid & 1.
+// B operand of the m16n8k16 score tiles: per lane the registers of k-step s
+// (channels 16s + 2*tig (+1), +8) for column n = gid: query head 4*nt + gid/2,
+// piece gid & 1.
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128) k_qprep_b16(const void *__restrict__ q, int dtype, int hq, int hkv,
-                                                  float qscale, uint2 *__restrict__ qb) {
-    const int j = blockIdx.x, b = blockIdx.y;
-    const int G = hq / hkv, NT = G > 4 ? 2 : 1;
-    const size_t bj = (size_t)b * hkv + j;
-    auto piece = [&](int hl, int c, int pc) -> uint32_t {
-        if (hl >= G) return 0u;
-        const size_t idx = ((size_t)b * hq + (size_t)j * G + hl) * D + c;
-        const float x = ((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[idx])
-                                             : reinterpret_cast<const float *>(q)[idx]) * qscale;
-        const uint32_t hi = f32_to_bf16_rne(x);
-        if (pc == 0) return hi;
-        return f32_to_bf16_rne(x - __uint_as_float(hi << 16));
-    };
-    for (int idx = threadIdx.x; idx < NT * (D / 16) * 32; idx += blockDim.x) {
-        const int L = idx & 31, s = (idx >> 5) % (D / 16), nt = (idx >> 5) / (D / 16);
-        const int gid = L >> 2, tig = L & 3, hl = 4 * nt + (gid >> 1), pc = gid & 1;
-        const int c0 = 16 * s + 2 * tig;
-        const uint32_t b0 = piece(hl, c0, pc) | (piece(hl, c0 + 1, pc) << 16);
-        const uint32_t b1 = piece(hl, c0 + 8, pc) | (piece(hl, c0 + 9, pc) << 16);
-        qb[((bj * NT + nt) * (D / 16) + s) * 32 + L] = make_uint2(b0, b1);
-    }
+__device__ __forceinline__ uint32_t b16_query_piece(const void *q, int dtype, size_t idx, float qscale, int pc) {
+    const float x = ((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[idx])
+                                         : reinterpret_cast<const float *>(q)[idx]) * qscale;
+    const uint32_t hi = f32_to_bf16_rne(x);
+    if (pc == 0) return hi;
+    return f32_to_bf16_rne(x - __uint_as_float(hi << 16));
 }
 
 // ---------------------------------------------------------------------------
@@ -209,7 +193,8 @@ __device__ __forceinline__ void consume_b16(uint32_t blk, int nv, B16State<D, G>
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParams p) {
+__global__ void __launch_bounds__(kB16Threads, 1) k_decode_b16(const __grid_constant__ DecodeParams dp) {
+    const AttendParams &p = dp.a;
     using St = B16State<D, G>;
     constexpr int NT = St::NT, NM = St::NM;
     extern __shared__ __align__(128) unsigned char b16_smem[];
@@ -218,12 +203,14 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     unsigned char *stage_mem = b16_smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(b16_smem + (size_t)S * stage_bytes);
     uint64_t *empty = full + kMaxStages;
-    unsigned char *valid = reinterpret_cast<unsigned char *>(empty + kMaxStages);   // [kMaxStages][kB16StageBlocks]
+    unsigned char *valid = reinterpret_cast<unsigned char *>(full) + kBarBytes;   // [kMaxStages][kB16StageBlocks]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(valid + kMaxStages * kB16StageBlocks);
+    MergeHead *plan = reinterpret_cast<MergeHead *>(valid + kMaxStages * kB16StageBlocks + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
+    grid_dependency_wait();
     __shared__ CtaUnits sh_cu;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -242,8 +229,9 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     const int u0 = cu.u0, u1 = cu.u1;
     const int iters = (u1 - u0 + pps - 1) / pps;
     if (warp == kB16Warps) {
+        const ProducerGate gate{nullptr, kMaxStages, nullptr, nullptr, 0, dp.ring_wait_ns};
         attend_producer<false>(p, stage_mem, full, empty, valid, abort_flag, S, stage_bytes, kB16StageBlocks, cu, iters,
-                               lane);
+                               lane, gate);
         return;
     }
     // consumer warp: kv head jl of the chunk, page slot pi of each stage
@@ -251,8 +239,10 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     const int gid = lane >> 2, tig = lane & 3;
     const int slot_base = (int)blockIdx.x;
     if (u1 > u0) init_records(p, cu, slot_base, pi, jl, G, D, lane);
-    if (iters == 0) return;
-    grid_dependency_wait();     // query fragments come from k_qprep_b16
+    {
+        const MergeHead mh = merge_head_of(p, cu.U, kB16Warps, warp, lane, 0);
+        if (lane == 0) plan[warp] = mh;
+    }
 
     int r = cu.r, ur = cu.ur;
     int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
@@ -260,11 +250,23 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     St st;
     auto start_run = [&](int rr) {
         const int b = rr / p.nchunks, chunk = rr - b * p.nchunks;
-        const size_t bj = (size_t)b * p.hkv + chunk * p.hc + jl;
+        const int j = chunk * p.hc + jl;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
+            const int hl = 4 * nt + (gid >> 1), pc = gid & 1;
+            const size_t row = ((size_t)b * p.hq + (size_t)j * G + hl) * D;
 #pragma unroll
-            for (int s = 0; s < D / 16; ++s) st.qf[nt][s] = p.qf[((bj * NT + nt) * (D / 16) + s) * 32 + lane];
+            for (int s = 0; s < D / 16; ++s) {
+                const int c0 = 16 * s + 2 * tig;
+                uint2 f = make_uint2(0u, 0u);
+                if (hl < G) {
+                    f.x = b16_query_piece(dp.q, dp.q_dtype, row + c0, dp.qscale, pc) |
+                          (b16_query_piece(dp.q, dp.q_dtype, row + c0 + 1, dp.qscale, pc) << 16);
+                    f.y = b16_query_piece(dp.q, dp.q_dtype, row + c0 + 8, dp.qscale, pc) |
+                          (b16_query_piece(dp.q, dp.q_dtype, row + c0 + 9, dp.qscale, pc) << 16);
+                }
+                st.qf[nt][s] = f;
+            }
             st.m_run[nt] = -INFINITY;
 #pragma unroll
             for (int m = 0; m < NM; ++m)
@@ -281,15 +283,15 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
             const float l = __shfl_sync(0xffffffffu, st.lacc[nt][0] + st.lacc[nt][1], tig);
             const int hh = 4 * nt + tig;
             if (hh < G) {
-                float *rec = p.part + record_index(slot_base + rr, pi, jl, hh, p.pw, p.hc, G) * (2 + D);
+                float *rec = p.part + record_index(slot_base + rr, pi, jl, hh, p.pw, p.hc, G) * rec_stride(D);
                 if (gid == 0) {
                     rec[0] = st.m_run[nt];
                     rec[1] = l;
                 }
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
-                    rec[2 + 16 * m + gid] = st.oacc[nt][m][0] + st.oacc[nt][m][1];
-                    rec[2 + 16 * m + gid + 8] = st.oacc[nt][m][2] + st.oacc[nt][m][3];
+                    rec[kRecHead + 16 * m + gid] = st.oacc[nt][m][0] + st.oacc[nt][m][1];
+                    rec[kRecHead + 16 * m + gid + 8] = st.oacc[nt][m][2] + st.oacc[nt][m][3];
                 }
             }
         }
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
     uint32_t phase = 0;
     const uint32_t blk0 = smem_addr(stage_mem) + (uint32_t)((pi * p.hc + jl) * p.bb);
     for (int it = 0; it < iters; ++it) {
-        if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
+        if (!mbar_wait_bounded(&full[stage], phase, dp.ring_wait_ns)) {
             if (lane == 0) {
                 *abort_flag = 1;
                 dqk_flag_error(kErrTimeout);
@@ -336,6 +338,10 @@ __global__ void __launch_bounds__(kB16Threads, 1) k_attend_b16(const AttendParam
         }
     }
     if (ok && cur_run >= 0) finish_run(cur_run);
+
+    consumers_grid_sync<kB16Warps>(dp.grid_wait_ns, nullptr);
+    grid_dependents_launch();
+    merge_heads<D>(dp, cu.U, kB16Warps, warp, lane, reinterpret_cast<float *>(stage_mem), plan);
 }
 
 }  // namespace dqk

@@ -1,18 +1,22 @@
 // dualqk.cu -- libdualqk: host side of the C ABI declared in include/dualqk.h
 // (argument checks, launch planning) and the single translation unit that
 // holds every kernel of the decode hot path.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
 #include "append.cuh"
 #include "attend.cuh"
 #include "bf16.cuh"
+#include "decode.cuh"
 #include "qprep.cuh"
 
 namespace {
@@ -21,6 +25,8 @@ using namespace dqk;
 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kMaxDevices = 64;
 
 dqk_status check_layer(const dqk_layer_desc *L) {
     if (!L) return DQK_ERR_INVALID_ARG;
@@ -37,21 +43,34 @@ dqk_status check_layer(const dqk_layer_desc *L) {
     return DQK_OK;
 }
 
-int device_sms() {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+int current_device() {
+    int dev = -1;
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+int device_sms(int dev) {
+    int sms = 0;
+    if (dev < 0 || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
     return sms;
 }
 
-// Decode plan and workspace layout: [header | qf | qm | q0 | partial records],
-// every section 256-byte aligned.
+// Decode plan and workspace layout: [header | qf | qk | qm | q0 | split
+// records], every section 256-byte aligned.
 struct DecodePlan {
-    int d, G, NT, NG, hc, pps, pw, nchunks, num_ctas, stages, bb;
+    int d, G, NT, NG, hc, pps, pw, nchunks, num_ctas, stages, bb, threads;
     size_t off_qf, off_qk, off_qm, off_q0, off_part, bytes, smem;
 };
 
 constexpr int kMaxAttendCtas = 160;   // >= the 148 SMs of a B200; larger parts run 160 persistent CTAs
+
+size_t records_bytes(size_t runs, int pw, int hc, int G, int d) {
+    return ((size_t)kMaxAttendCtas + runs - 1) * pw * hc * G * rec_stride(d) * sizeof(float);
+}
+
+size_t prologue_scratch(int d, int ns, int G) {
+    if (d == 128) return ns == 1 ? prologue_scratch_bytes<128, 1>(G) : prologue_scratch_bytes<128, 4>(G);
+    return ns == 1 ? prologue_scratch_bytes<64, 1>(G) : prologue_scratch_bytes<64, 2>(G);
+}
 
 bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.d = L->head_dim;
@@ -60,6 +79,7 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.NG = P.d / kGroup;
     const int hkv = L->num_kv_heads;
     const int warps = attend_warps(P.G), stage_blocks = attend_stage_blocks(P.G);
+    P.threads = attend_threads(P.G);
     // kv heads per chunk: the largest divisor of Hkv that divides the warp count
     P.hc = 0;
     for (int c = std::min(hkv, warps); c >= 1; --c)
@@ -73,18 +93,22 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.pw = warps / P.hc;            // warps per kv head (each takes attend_pages_per_warp pages of a stage)
     P.nchunks = hkv / P.hc;
     if ((long long)batch * P.nchunks * (L->num_pages + 1) >= (1LL << 31)) return false;
+    if ((long long)batch * L->num_q_heads >= (1LL << 31) / 2) return false;
     // Records are sized for kMaxAttendCtas so the workspace size does not depend
-    // on the device; the launch (check_decode) uses one CTA per SM up to that bound.
+    // on the device; the launch uses one CTA per SM up to that bound.
     P.num_ctas = kMaxAttendCtas;
-    P.bb = make_layout(P.d, L->v_ch0_protect, P.d / L->group_size).bytes;
-    // shared memory: ring stages | mbarriers | valid flags | abort flag | per-warp query fragments
+    const int ns = P.d / L->group_size;
+    P.bb = make_layout(P.d, L->v_ch0_protect, ns).bytes;
     const size_t stage_bytes = (size_t)stage_blocks * P.bb;
-    // (score fragments live in shared memory only for two query-head tiles)
-    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * stage_blocks + 16 +
-                         (P.NT > 1 ? (size_t)warps * P.NT * P.NG * (32 * 8 + 4 * 16) : 0);
+    const size_t fixed = decode_fixed_smem(stage_blocks, warps, P.NT, P.NG);
     const size_t budget = 227 * 1024;
     P.stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / stage_bytes);
     if (P.stages < 2) return false;
+    // the prologue works in the last stages (one at least stays free for the
+    // producer), the merge in the first
+    const size_t scratch_stages = (prologue_scratch(P.d, ns, P.G) + stage_bytes - 1) / stage_bytes;
+    if (scratch_stages >= (size_t)P.stages) return false;
+    if ((size_t)warps * (P.d + 4) * sizeof(float) > stage_bytes) return false;
     P.smem = P.stages * stage_bytes + fixed;
     const size_t R = (size_t)batch * P.nchunks;
     const size_t bj = (size_t)batch * hkv;
@@ -93,13 +117,111 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.off_qm = round_up(P.off_qk + bj * P.NT * (P.NG + 1) * 4 * sizeof(float), 256);
     P.off_q0 = round_up(P.off_qm + bj * P.NT * 32 * sizeof(uint32_t), 256);
     P.off_part = round_up(P.off_q0 + (size_t)batch * L->num_q_heads * sizeof(float), 256);
-    const size_t records = ((size_t)kMaxAttendCtas + R - 1) * P.pw * P.hc * P.G;
-    P.bytes = round_up(P.off_part + records * (2 + P.d) * sizeof(float), 256);
+    P.bytes = round_up(P.off_part + records_bytes(R, P.pw, P.hc, P.G, P.d), 256);
     return true;
 }
 
 dqk_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? DQK_OK : DQK_ERR_CUDA;
+}
+
+// Once per (kernel instance, device): the dynamic shared-memory bound, the
+// largest carveout (consecutive kernels then do not make the SMs switch their
+// L1 / shared split), and a check that one CTA fits on an SM (a cooperative
+// launch needs every CTA resident).  Thread-safe; later calls cost a lookup.
+template <auto Kernel>
+dqk_status prepare_kernel(int dev, size_t smem, int threads) {
+    static std::mutex mu;
+    static size_t set_smem[kMaxDevices] = {};
+    if (dev < 0 || dev >= kMaxDevices) return DQK_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (set_smem[dev] != 0 && set_smem[dev] >= smem) return DQK_OK;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return DQK_ERR_CUDA;
+    (void)cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, Kernel, threads, smem) != cudaSuccess)
+        return DQK_ERR_CUDA;
+    if (per_sm < 1) return DQK_ERR_UNSUPPORTED;
+    set_smem[dev] = smem;
+    return DQK_OK;
+}
+
+// The same for kernels launched without a shared-memory bound beyond the
+// default: only the carveout.
+template <auto Kernel>
+void prefer_max_shared(int dev) {
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
+    if (dev < 0 || dev >= kMaxDevices) return;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev]) return;
+    (void)cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    done[dev] = true;
+}
+
+// Cooperative launch (every CTA resident: the kernels' grid barriers rely on
+// it), with programmatic stream serialization when the device accepts the
+// two together: the kernel may then start while the previous kernel of the
+// stream finishes; it waits for it (griddepcontrol.wait) before reading
+// anything.
+std::atomic<int> g_pdl_refused[kMaxDevices];
+
+template <typename... KArgs, typename... Args>
+dqk_status launch_cooperative(void (*kernel)(KArgs...), int dev, unsigned grid, unsigned block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    const bool pdl = g_pdl_refused[dev].load(std::memory_order_relaxed) == 0;
+    cfg.numAttrs = pdl ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    if (e != cudaSuccess && pdl) {
+        (void)cudaGetLastError();   // a refused launch configuration is not sticky
+        g_pdl_refused[dev].store(1, std::memory_order_relaxed);
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    }
+    return e == cudaSuccess ? DQK_OK : DQK_ERR_CUDA;
+}
+
+// Tensor map of a layer's transforms [Hkv * d rows][d columns] fp32 for the
+// decode prologue's 2-D bulk tensor copies: boxes of 32 columns x d rows
+// with the 128-byte swizzle.  The encoder is the driver's, found through the
+// runtime's entry-point query (no link against the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+bool encode_transform_map(CUtensorMap *map, const float *t, int hkv, int d) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode || !t) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)hkv * d};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * sizeof(float)};
+    const cuuint32_t box[2] = {32, (cuuint32_t)d};
+    const cuuint32_t elem[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(t), dims, strides, box, elem,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct DecodeArgs {
@@ -114,80 +236,48 @@ struct DecodeArgs {
     void *ws;
     size_t ws_bytes;
     cudaStream_t stream;
-    bool partial = false;      // the combine writes (m, l, o) records instead of outputs
-    bool after_append = false; // the query kernel directly follows a step's append (writes first, waits last)
+    bool partial = false;            // write (m, l, o) records instead of outputs
+    // a decode step's append, done inside the kernel (max_new in 1..kFuseMaxNew)
+    const void *k = nullptr, *v = nullptr;
+    dqk_dtype kv_dtype = DQK_BF16;
+    const int *new_lens = nullptr, *seq_before = nullptr;
+    int max_new = 0;
+    // test only: the producer of CTA 0 never arms its second stage; short ring waits
+    bool stall = false;
 };
 
-dqk_status check_decode(const DecodeArgs &a, DecodePlan &P) {
+constexpr unsigned long long kRingWaitNs = kWaitLimitNs;   // 1 s
+constexpr unsigned long long kGridWaitNs = kWaitLimitNs;
+constexpr unsigned long long kStallWaitNs = 1000000ull;     // 1 ms
+
+dqk_status check_decode(const DecodeArgs &a, DecodePlan &P, int &dev) {
     dqk_status st = check_layer(a.L);
     if (st != DQK_OK) return st;
     if (!a.L->t_q || !a.q || !a.seq_lens || !a.page_table || !a.out || !a.ws) return DQK_ERR_INVALID_ARG;
+    // the transforms' rows are staged with 16-byte bulk copies
+    if (!aligned(a.L->t_q, 16) || (a.max_new > 0 && !aligned(a.L->t_k, 16))) return DQK_ERR_INVALID_ARG;
     if (a.q_dtype != DQK_F32 && a.q_dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
     if (a.batch <= 0 || a.max_pages <= 0 || a.pct < 0 || a.pct > 99) return DQK_ERR_INVALID_ARG;
     if (!aligned(a.ws, 256) || !aligned(a.out, 16)) return DQK_ERR_INVALID_ARG;
     if (!plan_decode(a.L, a.batch, P)) return DQK_ERR_UNSUPPORTED;
     if (a.ws_bytes < P.bytes) return DQK_ERR_WORKSPACE_TOO_SMALL;
-    P.num_ctas = std::min(device_sms(), kMaxAttendCtas);
+    dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return DQK_ERR_CUDA;
+    P.num_ctas = std::min(device_sms(dev), kMaxAttendCtas);
     if (P.num_ctas <= 0) return DQK_ERR_CUDA;
     return DQK_OK;
 }
 
-// Every kernel of the path prefers the largest shared-memory carveout, so that
-// consecutive kernels do not make the SMs switch their L1 / shared split.
-// Attributes are per function (one flag per kernel instance); setting one
-// twice is harmless.
-template <auto Kernel>
-void prefer_max_shared() {
-    static bool done = false;
-    if (!done) {
-        (void)cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                   (int)cudaSharedmemCarveoutMaxShared);
-        done = true;
-    }
-}
-
-// Launch with programmatic stream serialization: the kernel may start while
-// the previous kernel of the stream finishes; it orders itself with
-// griddepcontrol.wait before touching that kernel's outputs.
-template <typename... KArgs, typename... Args>
-dqk_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                      Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? DQK_OK : DQK_ERR_CUDA;
-}
-
-template <int D>
-dqk_status run_prepare(const DecodeArgs &a, const DecodePlan &P) {
-    const size_t smem = qprep_smem_bytes(D, P.G);
-    prefer_max_shared<k_qprep<D>>();
-    if (cudaFuncSetAttribute(k_qprep<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return DQK_ERR_CUDA;
-    char *ws = static_cast<char *>(a.ws);
-    const float qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
-    return launch_pdl(k_qprep<D>, dim3(a.L->num_kv_heads, a.batch), dim3(kQprepThreads), smem, a.stream, a.L->t_q,
-                      a.q, (int)a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, a.pct, qscale,
-                      reinterpret_cast<uint2 *>(ws + P.off_qf), reinterpret_cast<float *>(ws + P.off_qk),
-                      reinterpret_cast<uint32_t *>(ws + P.off_qm), reinterpret_cast<float *>(ws + P.off_q0),
-                      a.sel_out, a.after_append ? 1 : 0);
-}
-
 template <int D, int G, bool VCH0, int NS>
-dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
-    prefer_max_shared<k_attend<D, G, VCH0, NS>>();
-    if (cudaFuncSetAttribute(k_attend<D, G, VCH0, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
-        cudaSuccess)
-        return DQK_ERR_CUDA;
+dqk_status run_decode_g(const DecodeArgs &a, const DecodePlan &P, int dev) {
+    auto kernel = k_decode<D, G, VCH0, NS>;
+    dqk_status st = prepare_kernel<k_decode<D, G, VCH0, NS>>(dev, P.smem, P.threads);
+    if (st != DQK_OK) return st;
     char *ws = static_cast<char *>(a.ws);
-    AttendParams prm;
+    DecodeParams dp = {};
+    if (!encode_transform_map(&dp.tmap_q, a.L->t_q, a.L->num_kv_heads, D)) return DQK_ERR_CUDA;
+    if (a.max_new > 0 && !encode_transform_map(&dp.tmap_k, a.L->t_k, a.L->num_kv_heads, D)) return DQK_ERR_CUDA;
+    AttendParams &prm = dp.a;
     prm.pool = static_cast<const uint8_t *>(a.L->pool);
     prm.num_pages = a.L->num_pages;
     prm.seq_lens = a.seq_lens;
@@ -209,69 +299,62 @@ dqk_status run_attend_g(const DecodeArgs &a, const DecodePlan &P) {
     prm.v_ch0 = a.L->v_ch0_protect;
     prm.stages = P.stages;
     prm.num_ctas = P.num_ctas;
-    return launch_pdl(k_attend<D, G, VCH0, NS>, dim3(P.num_ctas), dim3(attend_threads(G)), P.smem, a.stream, prm);
+    dp.pool_w = static_cast<uint8_t *>(a.L->pool);
+    dp.t_q = a.L->t_q;
+    dp.q = a.q;
+    dp.q_dtype = (int)a.q_dtype;
+    dp.pct = a.pct;
+    dp.qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
+    dp.sel_out = a.sel_out;
+    dp.out = a.out;
+    dp.partial_out = a.partial ? 1 : 0;
+    dp.t_k = a.L->t_k;
+    dp.k_in = a.k;
+    dp.v_in = a.v;
+    dp.kv_dtype = (int)a.kv_dtype;
+    dp.max_new = a.max_new;
+    dp.new_lens = a.new_lens;
+    dp.seq_before = a.seq_before;
+    dp.ring_wait_ns = a.stall ? kStallWaitNs : kRingWaitNs;
+    dp.grid_wait_ns = kGridWaitNs;
+    dp.stall = a.stall ? 1 : 0;
+    return launch_cooperative(kernel, dev, (unsigned)P.num_ctas, (unsigned)P.threads, P.smem, a.stream, dp);
 }
 
 template <int D, bool VCH0, int NS>
-dqk_status run_attend_s(const DecodeArgs &a, const DecodePlan &P) {
+dqk_status run_decode_s(const DecodeArgs &a, const DecodePlan &P, int dev) {
     switch (P.G) {
-        case 1: return run_attend_g<D, 1, VCH0, NS>(a, P);
-        case 2: return run_attend_g<D, 2, VCH0, NS>(a, P);
-        case 4: return run_attend_g<D, 4, VCH0, NS>(a, P);
-        default: return run_attend_g<D, 8, VCH0, NS>(a, P);
+        case 1: return run_decode_g<D, 1, VCH0, NS>(a, P, dev);
+        case 2: return run_decode_g<D, 2, VCH0, NS>(a, P, dev);
+        case 4: return run_decode_g<D, 4, VCH0, NS>(a, P, dev);
+        default: return run_decode_g<D, 8, VCH0, NS>(a, P, dev);
     }
 }
 
 template <int D, bool VCH0>
-dqk_status run_attend_v(const DecodeArgs &a, const DecodePlan &P) {
-    return a.L->group_size == D ? run_attend_s<D, VCH0, 1>(a, P) : run_attend_s<D, VCH0, D / kGroup>(a, P);
+dqk_status run_decode_v(const DecodeArgs &a, const DecodePlan &P, int dev) {
+    return a.L->group_size == D ? run_decode_s<D, VCH0, 1>(a, P, dev) : run_decode_s<D, VCH0, D / kGroup>(a, P, dev);
 }
 
-template <int D>
-dqk_status run_attend(const DecodeArgs &a, const DecodePlan &P) {
-    return a.L->v_ch0_protect ? run_attend_v<D, true>(a, P) : run_attend_v<D, false>(a, P);
-}
-
-template <int D>
-dqk_status run_combine(const DecodeArgs &a, const DecodePlan &P) {
-    char *ws = static_cast<char *>(a.ws);
-    prefer_max_shared<k_combine<D>>();
-    return launch_pdl(k_combine<D>, dim3(a.L->num_q_heads, a.batch), dim3(kCombineThreads), 0, a.stream, a.seq_lens,
-                      a.batch,
-                      a.L->num_q_heads, a.L->num_kv_heads, P.hc, P.pw, P.nchunks, P.num_ctas,
-                      reinterpret_cast<const float *>(ws + P.off_part), a.out, (int)a.partial);
-}
-
-enum Stage { kPrepare = 1, kAttend = 2, kCombine = 4 };
-
-dqk_status decode_stages(const DecodeArgs &a, int stages) {
+dqk_status run_decode(const DecodeArgs &a) {
     DecodePlan P;
-    dqk_status st = check_decode(a, P);
+    int dev = -1;
+    dqk_status st = check_decode(a, P, dev);
     if (st != DQK_OK) return st;
-    const bool d128 = a.L->head_dim == 128;
-    if (stages & kPrepare) {
-        st = d128 ? run_prepare<128>(a, P) : run_prepare<64>(a, P);
-        if (st != DQK_OK) return st;
-    }
-    if (stages & kAttend) {
-        st = d128 ? run_attend<128>(a, P) : run_attend<64>(a, P);
-        if (st != DQK_OK) return st;
-    }
-    if (stages & kCombine) {
-        st = d128 ? run_combine<128>(a, P) : run_combine<64>(a, P);
-        if (st != DQK_OK) return st;
-    }
-    return DQK_OK;
+    if (a.L->head_dim == 128)
+        return a.L->v_ch0_protect ? run_decode_v<128, true>(a, P, dev) : run_decode_v<128, false>(a, P, dev);
+    return a.L->v_ch0_protect ? run_decode_v<64, true>(a, P, dev) : run_decode_v<64, false>(a, P, dev);
 }
 
 template <int D, int NS>
 dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk_dtype dtype, int batch,
                       const int *new_lens, const int *seq_before, int max_new, const int *page_table,
-                      int max_pages, int early_release, cudaStream_t stream) {
+                      int max_pages, cudaStream_t stream) {
+    const int dev = current_device();
     if (max_new <= kDirectMaxNew) {
-        // one row per sequence (a decode step): one row per CTA, no idle row slots
-        if (max_new == 1) prefer_max_shared<k_append_rows<D, NS, 1>>();
-        else prefer_max_shared<k_append_rows<D, NS, kRowsPerCta>>();
+        // one row per sequence: one row per CTA, no idle row slots
+        if (max_new == 1) prefer_max_shared<k_append_rows<D, NS, 1>>(dev);
+        else prefer_max_shared<k_append_rows<D, NS, kRowsPerCta>>(dev);
         auto kernel = max_new == 1 ? k_append_rows<D, NS, 1> : k_append_rows<D, NS, kRowsPerCta>;
         const int rw = max_new == 1 ? 1 : kRowsPerCta;
         const int groups = (max_new + rw - 1) / rw;
@@ -279,24 +362,21 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
         if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
         kernel<<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
             L->t_k, k, v, dtype, new_lens, seq_before, page_table, max_pages, groups,
-            static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
+            static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, 0);
         return launch_status();
     }
     const size_t smem = sizeof(AppendSmem<D>);
-    if (cudaFuncSetAttribute(k_quant_pack<D, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return DQK_ERR_CUDA;
+    dqk_status st = prepare_kernel<k_quant_pack<D, NS>>(dev, smem, 512);
+    if (st != DQK_OK) return st;
     const int slots = (max_new + kPage - 1) / kPage + 1;
     const long long items = (long long)batch * slots;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = std::max(device_sms(dev), 1);
     long long gx = ((long long)sms + L->num_kv_heads - 1) / L->num_kv_heads;   // ~1 CTA per SM (fp64 T_K in smem)
     if (gx > items) gx = items;
     if (gx < 1) gx = 1;
     k_quant_pack<D, NS><<<dim3((unsigned)gx, L->num_kv_heads), 512, smem, stream>>>(
         L->t_k, k, v, dtype, batch, new_lens, seq_before, page_table, max_pages, slots,
-        static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, early_release);
+        static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, 0);
     return launch_status();
 }
 
@@ -328,17 +408,17 @@ dqk_status check_append(const dqk_layer_desc *layer, const void *k, const void *
 
 dqk_status launch_append(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype dtype, int batch,
                          const int *new_lens, const int *seq_lens_before, int max_new, const int *page_table,
-                         int max_pages, int early_release, cudaStream_t s) {
+                         int max_pages, cudaStream_t s) {
     const bool one = layer->group_size == layer->head_dim;   // one scale group per token
     if (layer->head_dim == 128)
         return one ? run_append<128, 1>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
-                                        max_pages, early_release, s)
+                                        max_pages, s)
                    : run_append<128, 4>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
-                                        max_pages, early_release, s);
+                                        max_pages, s);
     return one ? run_append<64, 1>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
-                                   max_pages, early_release, s)
+                                   max_pages, s)
                : run_append<64, 2>(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table,
-                                   max_pages, early_release, s);
+                                   max_pages, s);
 }
 }  // namespace
 
@@ -349,8 +429,7 @@ dqk_status dqk_append(const dqk_layer_desc *layer, const void *k, const void *v,
                       int max_pages, dqk_stream_t stream) {
     dqk_status st = check_append(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages);
     if (st != DQK_OK || max_new == 0) return st;
-    // whatever follows may read the cache at once: release it only at exit
-    return launch_append(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages, 0,
+    return launch_append(layer, k, v, dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -371,8 +450,9 @@ size_t dqk_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max
 
 dqk_status dqk_decode(DQK_DECODE_ARGS) {
     DQK_DECODE_PACK;
-    return decode_stages(a, kPrepare | kAttend | kCombine);
+    return run_decode(a);
 }
+
 dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const void *v, dqk_dtype kv_dtype,
                            const int *new_lens, const int *seq_lens_before, int max_new, const void *q,
                            dqk_dtype q_dtype, int batch, const int *seq_lens, const int *page_table, int max_pages,
@@ -384,22 +464,35 @@ dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const voi
     DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out, sel_out,
                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};
     DecodePlan P;
-    st = check_decode(a, P);
+    int dev = -1;
+    st = check_decode(a, P, dev);
     if (st != DQK_OK) return st;
-    if (max_new > 0) {
-        // the query kernel (next on the stream) may start at once: it reads only
-        // q and T_Q before its grid-dependency wait
+    if (max_new > kFuseMaxNew) {
+        // longer appends run as their own kernel first
         st = launch_append(layer, k, v, kv_dtype, batch, new_lens, seq_lens_before, max_new, page_table, max_pages,
-                           1, a.stream);
+                           a.stream);
         if (st != DQK_OK) return st;
-        a.after_append = true;
+    } else if (max_new > 0) {
+        a.k = k;
+        a.v = v;
+        a.kv_dtype = kv_dtype;
+        a.new_lens = new_lens;
+        a.seq_before = seq_lens_before;
+        a.max_new = max_new;
     }
-    return decode_stages(a, kPrepare | kAttend | kCombine);
+    return run_decode(a);
 }
+
 dqk_status dqk_decode_partial(DQK_DECODE_ARGS) {
     DQK_DECODE_PACK;
     a.partial = true;
-    return decode_stages(a, kPrepare | kAttend | kCombine);
+    return run_decode(a);
+}
+
+dqk_status dqk_test_decode_stall(DQK_DECODE_ARGS) {
+    DQK_DECODE_PACK;
+    a.stall = true;
+    return run_decode(a);
 }
 
 dqk_status dqk_merge_partials(const float *parts, int n_parts, int batch, int num_q_heads, int head_dim,
@@ -417,19 +510,6 @@ dqk_status dqk_merge_partials(const float *parts, int n_parts, int batch, int nu
     return launch_status();
 }
 
-dqk_status dqk_decode_prepare(DQK_DECODE_ARGS) {
-    DQK_DECODE_PACK;
-    return decode_stages(a, kPrepare);
-}
-dqk_status dqk_decode_attend(DQK_DECODE_ARGS) {
-    DQK_DECODE_PACK;
-    return decode_stages(a, kAttend);
-}
-dqk_status dqk_decode_combine(DQK_DECODE_ARGS) {
-    DQK_DECODE_PACK;
-    return decode_stages(a, kCombine);
-}
-
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -443,7 +523,6 @@ dqk_status dqk_decode_combine(DQK_DECODE_ARGS) {
 static __device__ __align__(256) unsigned char g_dqk_noalloc_ws[DQK_NOALLOC_WORKSPACE_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[kMaxDevices] = {};
 
@@ -478,7 +557,7 @@ dqk_status dqk_decode_noalloc(const dqk_layer_desc *layer, const void *q, dqk_dt
     if (st != DQK_OK) return st;
     DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out, sel_out,
                  ws, (size_t)DQK_NOALLOC_WORKSPACE_BYTES, static_cast<cudaStream_t>(stream)};
-    return decode_stages(a, kPrepare | kAttend | kCombine);
+    return run_decode(a);
 }
 
 dqk_status dqk_last_device_error(dqk_stream_t stream) {
@@ -529,6 +608,7 @@ bool plan_b16(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.G = L->num_q_heads / L->num_kv_heads;
     P.NT = P.G > 4 ? 2 : 1;
     P.NG = P.d / kGroup;
+    P.threads = kB16Threads;
     const int hkv = L->num_kv_heads;
     if (hkv <= kB16Warps) {
         if (kB16Warps % hkv) return false;
@@ -541,35 +621,33 @@ bool plan_b16(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     P.pw = kB16Warps / P.hc;
     P.nchunks = hkv / P.hc;
     if ((long long)batch * P.nchunks * (L->num_pages + 1) >= (1LL << 31)) return false;
+    if ((long long)batch * L->num_q_heads >= (1LL << 31) / 2) return false;
     P.num_ctas = kMaxAttendCtas;
     P.bb = b16_block_bytes(P.d);
     const size_t stage_bytes = (size_t)kB16StageBlocks * P.bb;
-    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + (size_t)kMaxStages * kB16StageBlocks + 16;
+    const size_t fixed = decode_fixed_smem(kB16StageBlocks, kB16Warps, 1, 0);
     P.stages = (int)std::min<size_t>(kMaxStages, (227 * 1024 - fixed) / stage_bytes);
     if (P.stages < 2) return false;
+    if ((size_t)kB16Warps * (P.d + 4) * sizeof(float) > stage_bytes) return false;   // the merge's scratch
     P.smem = P.stages * stage_bytes + fixed;
     const size_t R = (size_t)batch * P.nchunks;
-    const size_t bj = (size_t)batch * hkv;
-    P.off_qf = 256;
-    P.off_qk = P.off_qm = P.off_q0 = 0;
-    P.off_part = round_up(P.off_qf + bj * P.NT * (P.d / 16) * 32 * sizeof(uint2), 256);
-    const size_t records = ((size_t)kMaxAttendCtas + R - 1) * P.pw * P.hc * P.G;
-    P.bytes = round_up(P.off_part + records * (2 + P.d) * sizeof(float), 256);
+    P.off_qf = P.off_qk = P.off_qm = P.off_q0 = 0;
+    P.off_part = 256;
+    P.bytes = round_up(P.off_part + records_bytes(R, P.pw, P.hc, P.G, P.d), 256);
     return true;
 }
 
 template <int D, int G>
-dqk_status run_attend_b16(const DecodeArgs &a, const DecodePlan &P) {
-    if (cudaFuncSetAttribute(k_attend_b16<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) !=
-        cudaSuccess)
-        return DQK_ERR_CUDA;
+dqk_status run_decode_b16_g(const DecodeArgs &a, const DecodePlan &P, int dev) {
+    dqk_status st = prepare_kernel<k_decode_b16<D, G>>(dev, P.smem, P.threads);
+    if (st != DQK_OK) return st;
     char *ws = static_cast<char *>(a.ws);
-    AttendParams prm = {};
+    DecodeParams dp = {};
+    AttendParams &prm = dp.a;
     prm.pool = static_cast<const uint8_t *>(a.L->pool);
     prm.num_pages = a.L->num_pages;
     prm.seq_lens = a.seq_lens;
     prm.page_table = a.page_table;
-    prm.qf = reinterpret_cast<const uint2 *>(ws + P.off_qf);
     prm.part = reinterpret_cast<float *>(ws + P.off_part);
     prm.batch = a.batch;
     prm.hq = a.L->num_q_heads;
@@ -583,25 +661,24 @@ dqk_status run_attend_b16(const DecodeArgs &a, const DecodePlan &P) {
     prm.v_ch0 = 0;
     prm.stages = P.stages;
     prm.num_ctas = P.num_ctas;
-    return launch_pdl(k_attend_b16<D, G>, dim3(P.num_ctas), dim3(kB16Threads), P.smem, a.stream, prm);
+    dp.q = a.q;
+    dp.q_dtype = (int)a.q_dtype;
+    dp.qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
+    dp.out = a.out;
+    dp.ring_wait_ns = kRingWaitNs;
+    dp.grid_wait_ns = kGridWaitNs;
+    return launch_cooperative(k_decode_b16<D, G>, dev, (unsigned)P.num_ctas, (unsigned)P.threads, P.smem, a.stream,
+                              dp);
 }
 
 template <int D>
-dqk_status run_decode_b16(const DecodeArgs &a, const DecodePlan &P) {
-    char *ws = static_cast<char *>(a.ws);
-    const float qscale = (float)(1.4426950408889634 / std::sqrt((double)D));
-    k_qprep_b16<D><<<dim3(a.L->num_kv_heads, a.batch), 128, 0, a.stream>>>(
-        a.q, (int)a.q_dtype, a.L->num_q_heads, a.L->num_kv_heads, qscale, reinterpret_cast<uint2 *>(ws + P.off_qf));
-    dqk_status st = launch_status();
-    if (st != DQK_OK) return st;
+dqk_status run_decode_b16(const DecodeArgs &a, const DecodePlan &P, int dev) {
     switch (P.G) {
-        case 1: st = run_attend_b16<D, 1>(a, P); break;
-        case 2: st = run_attend_b16<D, 2>(a, P); break;
-        case 4: st = run_attend_b16<D, 4>(a, P); break;
-        default: st = run_attend_b16<D, 8>(a, P); break;
+        case 1: return run_decode_b16_g<D, 1>(a, P, dev);
+        case 2: return run_decode_b16_g<D, 2>(a, P, dev);
+        case 4: return run_decode_b16_g<D, 4>(a, P, dev);
+        default: return run_decode_b16_g<D, 8>(a, P, dev);
     }
-    if (st != DQK_OK) return st;
-    return run_combine<D>(a, P);
 }
 
 }  // namespace
@@ -657,11 +734,13 @@ dqk_status dqk_bf16_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype
     DecodePlan P;
     if (!plan_b16(layer, batch, P)) return DQK_ERR_UNSUPPORTED;
     if (workspace_bytes < P.bytes) return DQK_ERR_WORKSPACE_TOO_SMALL;
-    P.num_ctas = std::min(device_sms(), kMaxAttendCtas);
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return DQK_ERR_CUDA;
+    P.num_ctas = std::min(device_sms(dev), kMaxAttendCtas);
     if (P.num_ctas <= 0) return DQK_ERR_CUDA;
     DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, 0, out, nullptr,
                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};
-    return layer->head_dim == 128 ? run_decode_b16<128>(a, P) : run_decode_b16<64>(a, P);
+    return layer->head_dim == 128 ? run_decode_b16<128>(a, P, dev) : run_decode_b16<64>(a, P, dev);
 }
 
 }  // extern "C"

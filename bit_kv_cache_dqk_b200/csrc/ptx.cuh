@@ -104,6 +104,14 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return pol;
 }
 
+// L2 policy for small tensors every launch re-reads (the transforms): kept
+// in L2 ahead of the streamed pages.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // 1-D bulk copy global -> shared, completion counted on `bar` (no multicast).
 __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -119,6 +127,17 @@ __device__ __forceinline__ void bulk_copy_g2s_hint(void *dst, const void *src, u
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
             "r"(smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// 2-D tiled bulk tensor copy global -> shared of the box at (x, y) of the
+// tensor map at `tmap` (a kernel-parameter address) with an L2 cache policy,
+// completion counted on `bar` (no multicast).
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+        "%3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
 }
 
@@ -155,6 +174,56 @@ __device__ __forceinline__ void stage_f64_padded(double *dst, const float *src) 
                 d[2] = (double)v[u].z;
                 d[3] = (double)v[u].w;
             }
+        }
+    }
+}
+
+// Generic-proxy accesses made before these fences are ordered before the
+// async-proxy (bulk copy) accesses issued after them: shared memory of this
+// CTA, and global memory.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Address of the grid-wide barrier word that the driver sets up for a
+// cooperative launch (the word cooperative groups' grid sync uses): the grid
+// workspace { size, barrier } sits at the address held in environment
+// registers 1 (high half) and 2 (low half).  Null when the launch was not
+// cooperative.
+__device__ __forceinline__ unsigned int *coop_barrier_word() {
+    unsigned int hi, lo;
+    asm volatile("mov.u32 %0, %%envreg1;" : "=r"(hi));
+    asm volatile("mov.u32 %0, %%envreg2;" : "=r"(lo));
+    const unsigned long long ws = ((unsigned long long)hi << 32) | lo;
+    return ws ? reinterpret_cast<unsigned int *>(ws + 4) : nullptr;
+}
+
+// Grid barrier, called by one thread of every CTA.  CTA 0 adds 2^31 - (C - 1),
+// the others add 1: the top bit of the word flips when the last CTA arrives
+// and the low bits return to their value, so the word needs no reset between
+// barriers or launches as long as every CTA arrives once at each of them.  The
+// release add publishes what the CTA wrote before (and, through the CTA
+// barrier that precedes the call, what its other threads wrote); the acquire
+// polls make the other CTAs' writes visible.  Gives up after limit_ns (false).
+__device__ __forceinline__ bool grid_sync_bounded(unsigned int *word, uint64_t limit_ns) {
+    const unsigned int add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1u) : 1u;
+    unsigned int old;
+    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(word), "r"(add) : "memory");
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if ((old ^ ld_acquire_gpu(word)) & 0x80000000u) return true;
+        if (it >= 64u) {
+            if ((it & 31u) == 0u && global_timer_ns() - t0 > limit_ns) return false;
+            __nanosleep(40);
         }
     }
 }

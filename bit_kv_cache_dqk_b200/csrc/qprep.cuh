@@ -1,9 +1,10 @@
-// qprep.cuh -- k_qprep: query transform q' = T_Q q and dynamic channel
-// selection (keep channel 0 and the largest-|q'| channels; "Why the cache
-// becomes a bottleneck": query-channel pruning; "Throughput on SGLang": 40 %
-// of key channels removed from reads).  One CTA per (sequence, kv head), one
-// warp per query head of the group.  Also lays the kept, scaled q' out as the
-// B operands of the attend kernel's tensor-core tiles.
+// qprep.cuh -- query transform q' = T_Q q and dynamic channel selection (keep
+// channel 0 and the largest-|q'| channels; "Why the cache becomes a
+// bottleneck": query-channel pruning; "Throughput on SGLang": 40 % of key
+// channels removed from reads), run for the G query heads of one (sequence,
+// kv head) by the consumer warps of one CTA in the decode kernel's prologue.
+// The kept, scaled q' is laid out as the B operands of the attend loop's
+// tensor-core tiles.
 #pragma once
 
 #include "common.cuh"
@@ -11,45 +12,8 @@
 
 namespace dqk {
 
-// Warp-wide bitonic sort, descending, of 32*E distinct 64-bit keys; element
-// index lane*E + e.  Stages whose partner distance is below E stay in
-// registers, the others exchange through shuffles.
-template <int E>
-__device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[E], int lane) {
-    constexpr int N = 32 * E;
-#pragma unroll
-    for (int k = 2; k <= N; k <<= 1) {
-#pragma unroll
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            if (jj >= E) {
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const int i = lane * E + e;
-                    const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[e], jj / E);
-                    const bool keep_max = ((i & jj) == 0) == ((i & k) == 0);
-                    v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const int pe = e ^ jj;
-                    if (pe > e) {
-                        const int i = lane * E + e;
-                        const unsigned long long a = v[e], b = v[pe];
-                        const bool desc = (i & k) == 0;
-                        if (desc ? (a < b) : (a > b)) {
-                            v[e] = b;
-                            v[pe] = a;
-                        }
-                    }
-                }
-            }
-        }
-    }
-}
-
-// Query fragments of one (sequence, kv head), consumed by k_attend, with
-// qs = q'_c * log2(e)/sqrt(d) on kept channels c >= 1 (0 elsewhere):
+// Query fragments of one (sequence, kv head), consumed by the attend loop,
+// with qs = q'_c * log2(e)/sqrt(d) on kept channels c >= 1 (0 elsewhere):
 //   qf  [B*Hkv][NT][NG][32] uint2      per lane: the two s8x4 registers of the
 //       m16n8k32 B operand of group g: rows (channels of the group) 4*tig..+3
 //       and 16+4*tig..+3, column n = gid -> query head 4*nt + gid/2; gid even:
@@ -66,230 +30,301 @@ __device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[E], in
 //       the low part (the key mins repeat in those A columns), so one tile
 //       sums both; column 2h holds query head 4*nt + h, odd columns are zero.
 //   q0  [B][Hq] float                  qs of channel 0 (always kept).
+// Query heads a tile of 4 leaves empty (G < 4) hold zeros everywhere.
+struct QueryOut {
+    uint2 *qf;
+    float *qk;
+    uint32_t *qm;
+    float *q0;
+    int16_t *sel;   // nullable: [B][Hq][n_keep] kept channels, ascending
+};
+
 __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
     const __half hi = __float2half_rn(x);
     if (piece == 0) return __half_as_ushort(hi);
     return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
 }
 
-constexpr int kQprepThreads = 512;
-
-// Shared memory of k_qprep: T_Q[j] in fp32 with rows padded to D+4 floats
-// (conflict-free 16-byte row reads), the query rows in fp64, per-head sort
-// buffers and the outputs before they are laid out.  (T_Q held in fp64 would
-// double this; the larger CTAs then slow a co-running append.)
-__host__ __device__ constexpr size_t qprep_smem_bytes(int D, int G) {
-    return (size_t)D * (D + 4) * 4 + (size_t)G * D * 8 + (size_t)kQprepThreads * 8 + (size_t)G * (D / 32) * 8 +
-           (size_t)G * (D / 32 + 1) * 4 + (size_t)G * D * 3 + 64;
+// A [D][D] fp32 transform staged by 2-D tensor copies: D/32 boxes of 32
+// columns x D rows, each row of a box 128 bytes whose 16-byte chunks are
+// XOR-permuted by (row mod 8) (the tensor map's 128-byte swizzle), so that
+// one thread per row reads 16-byte chunks without bank conflicts.  Byte
+// offset of columns 4u..4u+3 of box k, row r; the base is 1024-byte aligned.
+template <int D>
+__device__ __forceinline__ uint32_t swz_offset(int k, int r, int u) {
+    return (uint32_t)(k * D * 128 + r * 128 + ((u ^ (r & 7)) << 4));
 }
 
-// One thread per (query head, channel), kQprepThreads / D heads per pass.
-// Launched with programmatic stream serialization: it reads its inputs and
-// computes q' and the selection while an earlier append may still be running,
-// waits for the earlier work before writing anything, then releases the
-// attend kernel.
+// Issue the copies of matrix j (rows j*D ..) of the tensor map into dst; the
+// transforms are re-read by every launch, so they are kept in L2.
 template <int D>
-__global__ void __launch_bounds__(kQprepThreads) k_qprep(const float *__restrict__ t_q, const void *__restrict__ q,
-                                                        int dtype, int hq, int hkv, int pct, float qscale,
-                                                        uint2 *__restrict__ qf, float *__restrict__ qk,
-                                                        uint32_t *__restrict__ qm, float *__restrict__ q0,
-                                                        int16_t *__restrict__ sel_out, int write_first) {
+__device__ __forceinline__ void stage_matrix(unsigned char *dst, const void *tmap, int j, uint64_t *bar) {
+    const uint64_t keep = l2_policy_evict_last();
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) tma_load_2d(dst + (size_t)k * D * 128, tmap, 32 * k, j * D, bar, keep);
+}
+
+// Sum over i ascending of (double)T[row][i] * x[i * xs + n], one fused
+// multiply-add after the other for each of the NX vectors (fp32 x fp32
+// products are exact in fp64, so the result does not depend on contraction).
+// x is i-major (row stride xs doubles), so the NX values of a column come in
+// 16-byte loads.  Eight 16-byte chunks of the row per iteration.
+template <int D, int NX>
+__device__ __forceinline__ void dot_rows_swz(const unsigned char *sT, int row, const double *x, int xs,
+                                             double (&acc)[NX]) {
+#pragma unroll
+    for (int n = 0; n < NX; ++n) acc[n] = 0.0;
+    const int sw = row & 7;
+    const unsigned char *base = sT + row * 128;
+#pragma unroll 1
+    for (int k = 0; k < D / 32; ++k) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float4 tv = *reinterpret_cast<const float4 *>(base + k * D * 128 + ((u ^ sw) << 4));
+            const double te[4] = {(double)tv.x, (double)tv.y, (double)tv.z, (double)tv.w};
+            const double *xi = x + (32 * k + 4 * u) * xs;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int n = 0; n < NX; ++n) acc[n] = fma(te[e], xi[e * xs + n], acc[n]);
+        }
+    }
+}
+
+// Shared memory of one query task (1024-byte aligned): T_Q[j] [D][D] fp32
+// (swizzled boxes; the q' values [G][D] reuse it once the sums are done), the
+// query rows [D][G] fp64 (i-major), the int8 pieces [G][2][D].
+template <int D>
+__host__ __device__ constexpr size_t qprep_scratch_bytes(int G) {
+    return (size_t)D * D * 4 + (size_t)G * D * 8 + (size_t)G * 2 * D;
+}
+
+// Channels (of this warp's NG per lane, channel 0 excluded) whose magnitude
+// bit pattern is >= cand.
+template <int NG>
+__device__ __forceinline__ int count_ge(const uint32_t (&mag)[NG], bool ch0, uint32_t cand) {
+    uint32_t n = 0;
+#pragma unroll
+    for (int g = 0; g < NG; ++g) n += (mag[g] >= cand && !(g == 0 && ch0)) ? 1u : 0u;
+    return (int)__reduce_add_sync(0xffffffffu, n);
+}
+
+// x * 2^e, exact: an exponent-field addition when x and the result are
+// normal, the library function otherwise.
+__device__ __forceinline__ float scale_pow2(float x, int e) {
+    const uint32_t b = __float_as_uint(x);
+    const int ex = (int)((b >> 23) & 0xffu) + e;
+    if (((b >> 23) & 0xffu) != 0u && ((b >> 23) & 0xffu) != 0xffu && ex >= 1 && ex <= 254)
+        return __uint_as_float((b & 0x807fffffu) | ((uint32_t)ex << 23));
+    return ldexpf(x, e);
+}
+
+// The G query heads of (sequence b, kv head j), by the nthreads threads of
+// the calling group (t = 0..nthreads-1; G <= nthreads / 32, D <= nthreads),
+// which synchronise on named barrier `bar` (all) and `busy_bar` (the first
+// max(D/32, G) warps, which do the work; the others run meanwhile() and
+// return):
+//   q'_c = fp32(fp64 sequential sum_i T_Q[j][c][i] q_i)   (thread c, all heads);
+//   kept = {0} + the n_keep - 1 largest |q'_c| of c >= 1 (fp32 magnitudes,
+//   ties to the lower index): warp h selects head h's channels by a bitwise
+//   threshold search, then writes head h's fragments and kept channels
+//   (ascending).
+// meanwhile(): work of the caller's that overlaps the loads of the task.
+template <int D, int G, typename Meanwhile>
+__device__ void qprep_kv(const void *tmap_q, const void *__restrict__ q, int dtype, int hq, int hkv, int pct,
+                         float qscale, int b, int j, int t, int nthreads, int bar, int busy_bar, unsigned char *scratch,
+                         uint64_t *tbar, uint32_t &tphase, uint64_t wait_ns, const QueryOut &qo, Meanwhile meanwhile) {
     constexpr int NG = D / 32;
-    constexpr int kRow = D + 4;                       // padded fp32 row of T_Q
-    constexpr int kHeadsPerPass = kQprepThreads / D;
-    constexpr int kWarpsPerHead = D / 32;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int G = hq / hkv;
-    const int NT = G > 4 ? 2 : 1;
-    float *tq = reinterpret_cast<float *>(smem_raw);                                  // [D][D+4]
-    double *qin = reinterpret_cast<double *>(tq + D * kRow);                         // [G][D]
-    unsigned long long *xbuf = reinterpret_cast<unsigned long long *>(qin + G * D);  // [threads] sort exchange
-    float *qsum = reinterpret_cast<float *>(xbuf + kQprepThreads);                   // [G][NG]
-    float *sig = qsum + G * NG;                                                       // [G][NG]  p_g
-    float *gmax = sig + G * NG;                                                       // [G][NG]  largest |qs|
-    float *shd = gmax + G * NG;                                                       // [G]      sigma_h
-    signed char *q8 = reinterpret_cast<signed char *>(shd + G);                      // [G][2][D] pieces
-    unsigned char *mask = reinterpret_cast<unsigned char *>(q8 + G * 2 * D);         // [G][D]
-    int *wcount = reinterpret_cast<int *>(mask + G * D + ((16 - (G * D) % 16) % 16)); // [threads/32] kept per warp
-    const int j = blockIdx.x, b = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = threadIdx.x % D, hp = threadIdx.x / D;   // channel, head slot of the pass
+    constexpr int NT = G > 4 ? 2 : 1;
+    const int warp = t >> 5, lane = t & 31;
     const int nk = keep_count(D, pct);
+    double *qin = reinterpret_cast<double *>(scratch + (size_t)D * D * 4);
+    signed char *q8 = reinterpret_cast<signed char *>(qin + (size_t)G * D);
+    float *qpv = reinterpret_cast<float *>(scratch);   // [G][D] after the sums
 
-    {   // stage T_Q[j] (fp32, padded rows) and the query rows (fp64)
-        constexpr int n4 = D * D / 4, kIn = (n4 + kQprepThreads - 1) / kQprepThreads;
-        const float4 *src = reinterpret_cast<const float4 *>(t_q + (size_t)j * D * D);
-        float4 v[kIn];
-#pragma unroll
-        for (int u = 0; u < kIn; ++u) {
-            const int i4 = threadIdx.x + u * kQprepThreads;
-            if (i4 < n4) v[u] = src[i4];
-        }
-        const size_t qbase = ((size_t)b * hq + (size_t)j * G) * D;
-        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x)
-            qin[idx] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[qbase + idx])
-                                                    : reinterpret_cast<const float *>(q)[qbase + idx]);
-#pragma unroll
-        for (int u = 0; u < kIn; ++u) {
-            const int i4 = threadIdx.x + u * kQprepThreads;
-            if (i4 < n4) {
-                const int e = 4 * i4, row = e / D, col = e % D;
-                *reinterpret_cast<float4 *>(&tq[row * kRow + col]) = v[u];
-            }
-        }
+    // stage T_Q[j] and the G query rows
+    named_bar_sync(bar, nthreads);   // the previous task is done with the scratch
+    if (t == 0) {
+        fence_proxy_async_shared();   // earlier generic accesses to the scratch come first
+        mbar_arrive_expect_tx(tbar, D * D * 4);
+        stage_matrix<D>(scratch, tmap_q, j, tbar);
     }
-    __syncthreads();
+    const size_t qbase = ((size_t)b * hq + (size_t)j * G) * D;
+    for (int i = t; i < G * D; i += nthreads) {   // query h, channel c -> qin[c][h]
+        const int h = i / D, c = i - h * D;
+        qin[c * G + h] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[qbase + i])
+                                                      : reinterpret_cast<const float *>(q)[qbase + i]);
+    }
+    named_bar_sync(bar, nthreads);   // the query rows are in
+    // the warps the task leaves idle run the caller's `meanwhile` work
+    constexpr int kBusy = (D / 32 > G ? D / 32 : G);
+    if (warp >= kBusy) {
+        meanwhile();
+        return;
+    }
+    if (!mbar_wait_bounded(tbar, tphase, wait_ns)) dqk_flag_error(kErrTimeout);
+    tphase ^= 1u;
 
-    // write_first: the kernel before this one on the stream (a cache append
-    // launched without programmatic serialization) writes nothing this kernel
-    // reads or writes, and everything before it has finished, so the outputs
-    // are written at once and the wait for it comes last (this kernel's
-    // completion then implies the append's).  Otherwise the outputs wait for
-    // every earlier kernel of the stream.
-    bool waited = write_first != 0;
-    for (int h0 = 0; h0 < G; h0 += kHeadsPerPass) {
-        const int hl = h0 + hp;                 // local query head of this thread
-        const bool active = hl < G;
-        const int h = j * G + hl;
-        // q'_c = sum_i T_Q[c][i] q_i, ascending i, exact fp32 x fp32 products
-        // accumulated in fp64, rounded once to fp32
-        float qp = 0.0f;
-        if (active) {
-            const float *row = &tq[c * kRow];
-            const double *x = &qin[hl * D];
-            double acc = 0.0;
+    // q'_c of every head: G interleaved sums per thread (thread c = row c),
+    // ascending i, exact fp32 x fp32 products accumulated in fp64, one
+    // rounding each
+    double acc[G];
+    if (t < D) dot_rows_swz<D, G>(scratch, t, qin, G, acc);
+    named_bar_sync(busy_bar, 32 * kBusy);   // T_Q is dead
+    if (t < D) {
 #pragma unroll
-            for (int i = 0; i < D; i += 4) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(&row[i]);
-                acc = fma((double)t4.x, x[i + 0], acc);
-                acc = fma((double)t4.y, x[i + 1], acc);
-                acc = fma((double)t4.z, x[i + 2], acc);
-                acc = fma((double)t4.w, x[i + 3], acc);
+        for (int n = 0; n < G; ++n) qpv[n * D + t] = __double2float_rn(acc[n]);
+    }
+    named_bar_sync(busy_bar, 32 * kBusy);
+
+    if (warp < G) {
+        const int h = warp, hl = h, nt = hl >> 2, hh = hl & 3;
+        const int hg = j * G + h;   // query head index
+        // selection of the nk - 1 channels c >= 1 with the largest |q'_c|
+        // (fp32 magnitudes as bit patterns), ties to the lower index; lane owns
+        // channels lane + 32 g.  T = the (nk-1)-th largest magnitude, found bit
+        // by bit from the top (the largest T with at least nk - 1 magnitudes >=
+        // T); then every channel above T is kept, and of those equal to T the
+        // lowest-indexed ones that complete the count.
+        const int m = nk - 1;
+        uint32_t mag[NG];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const int c = lane + 32 * g;
+            mag[g] = c == 0 ? 0u : (__float_as_uint(qpv[h * D + c]) & 0x7fffffffu);
+        }
+        const bool ch0 = lane == 0;   // channel 0 (g = 0) takes no part
+        uint32_t T = 0;
+        // bit 30 alone, then two bits per step (three candidates counted at once)
+        if (count_ge<NG>(mag, ch0, 1u << 30) >= m) T = 1u << 30;
+#pragma unroll 1
+        for (int bit = 28; bit >= 0; bit -= 2) {
+            const int n3 = count_ge<NG>(mag, ch0, T | (3u << bit)), n2 = count_ge<NG>(mag, ch0, T | (2u << bit)),
+                      n1 = count_ge<NG>(mag, ch0, T | (1u << bit));
+            T |= (n3 >= m ? 3u : n2 >= m ? 2u : n1 >= m ? 1u : 0u) << bit;
+        }
+        int need = m - (T == 0x7fffffffu ? 0 : count_ge<NG>(mag, ch0, T + 1u));   // equal to T, still to keep
+        uint32_t kmask[NG];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const bool eq = mag[g] == T && !(g == 0 && ch0) && m > 0;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const int rank = __popc(eqm & ((1u << lane) - 1u));   // equal channels of lower index in this group
+            const bool keep = (mag[g] > T && !(g == 0 && ch0) && m > 0) || (eq && rank < need);
+            kmask[g] = __ballot_sync(0xffffffffu, keep);
+            need -= __popc(eqm);
+        }
+        kmask[0] |= 1u;   // channel 0 is always kept
+
+        // lane owns channels lane + 32 g: scaled q' on kept channels >= 1, group
+        // sums and maxima, sigma_h, and the two int8 pieces relative to sigma_g =
+        // sigma_h * 2^-e, the smallest such value not below the group's largest
+        // |qs| / 127, so that sigma_g / sigma_h is a power of two
+        float qs[NG], v[NG], gs[NG], gm[NG];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const int c = lane + 32 * g;
+            qs[g] = qpv[h * D + c] * qscale;
+            v[g] = (((kmask[g] >> lane) & 1u) && c != 0) ? qs[g] : 0.0f;
+            gs[g] = v[g];
+            gm[g] = fabsf(v[g]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                gs[g] += __shfl_xor_sync(0xffffffffu, gs[g], o);
+                gm[g] = fmaxf(gm[g], __shfl_xor_sync(0xffffffffu, gm[g], o));
             }
-            qp = __double2float_rn(acc);
         }
-        // selection: bitonic sort (descending) of the head's D keys, one per
-        // thread: |q'| bits, then ascending channel; channel 0 sorts last
-        unsigned long long key = (c == 0) ? 0ull
-                                          : (((unsigned long long)(__float_as_uint(qp) & 0x7fffffffu) << 32) |
-                                             (unsigned long long)(0xffffffffu - (unsigned)c));
-#pragma unroll
-        for (int k = 2; k <= D; k <<= 1) {
-#pragma unroll
-            for (int jj = k >> 1; jj > 0; jj >>= 1) {
-                unsigned long long o;
-                if (jj < 32) {
-                    o = __shfl_xor_sync(0xffffffffu, key, jj);
-                } else {
-                    xbuf[threadIdx.x] = key;
-                    __syncthreads();
-                    o = xbuf[threadIdx.x ^ jj];
-                    __syncthreads();
-                }
-                const bool keep_max = ((c & jj) == 0) == ((c & k) == 0);
-                key = keep_max ? (key > o ? key : o) : (key < o ? key : o);
-            }
-        }
-        // position c of the sorted order holds the c-th largest key
-        if (active) mask[hl * D + c] = 0;
-        __syncthreads();
-        if (active && c < nk - 1) mask[hl * D + (int)(0xffffffffu - (unsigned)(key & 0xffffffffull))] = 1;
-        if (active && c == 0) mask[hl * D] = 1;
-        __syncthreads();
-        const bool keep = active && mask[hl * D + c] != 0;
-        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-        if (lane == 0) wcount[warp] = __popc(bal);
-        // scaled q' on kept channels >= 1; group sums and two int8 pieces
-        // (warp = one group of one head) relative to sigma_g = sigma_h * 2^-e,
-        // the smallest such value not below the group's largest |qs| / 127, so
-        // that sigma_g / sigma_h is a power of two
-        const float qs = qp * qscale;
-        const float v = (keep && c != 0) ? qs : 0.0f;
-        float gs = v, gm = fabsf(v);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            gs += __shfl_xor_sync(0xffffffffu, gs, o);
-            gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
-        }
-        const int g = c >> 5;
-        if (active && lane == 0) gmax[hl * NG + g] = gm;
-        __syncthreads();
         float hm = 0.0f;
-        if (active)
-            for (int gg = 0; gg < NG; ++gg) hm = fmaxf(hm, gmax[hl * NG + gg]);
-        const float sh = hm / 127.0f, tg = gm / 127.0f;
-        int e = 0;
-        if (tg > 0.0f) {
-            e = ilogbf(sh) - ilogbf(tg);   // >= 0: sh >= tg
-            if (ldexpf(sh, -e) < tg) --e;
-        }
-        const float sgm = ldexpf(sh, -e);   // in [tg, 2 tg)
-        int q1 = 0, q2 = 0;
-        if (sgm > 0.0f) {
-            const float x = v / sgm;
-            q1 = max(-127, min(127, __float2int_rn(x)));
-            q2 = max(-128, min(127, __float2int_rn((x - (float)q1) * 256.0f)));
-        }
-        if (active) {
-            q8[(hl * 2 + 0) * D + c] = (signed char)q1;
-            q8[(hl * 2 + 1) * D + c] = (signed char)q2;
-            if (lane == 0) {
-                qsum[hl * NG + g] = gs;
-                sig[hl * NG + g] = ldexpf(1.0f, -e - 2 * g);
+#pragma unroll
+        for (int g = 0; g < NG; ++g) hm = fmaxf(hm, gm[g]);
+        constexpr float kInv127 = 1.0f / 127.0f;
+        const float sh = hm * kInv127;
+        const float rsh = sh > 0.0f ? 1.0f / sh : 0.0f;   // 1 / sigma_g = 2^e / sh
+        float sig[NG];
+        int before = 0;   // kept channels in earlier groups
+        const uint32_t shb = __float_as_uint(sh);
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            // sigma_g = sh * 2^-e with e >= 0 the largest such that sigma_g >= tg:
+            // sh = 2^Es ms, tg = 2^Et mt (normal, ms, mt in [1, 2)) give
+            // e = Es - Et - [ms < mt]; exponent-field arithmetic, the library
+            // functions for the rare subnormal operand
+            const float tg = gm[g] * kInv127;
+            const uint32_t tgb = __float_as_uint(tg);
+            int e = 0;
+            if (tg > 0.0f) {
+                if ((shb >> 23) != 0u && (tgb >> 23) != 0u) {
+                    e = (int)(shb >> 23) - (int)(tgb >> 23) - ((shb & 0x7fffffu) < (tgb & 0x7fffffu) ? 1 : 0);
+                } else {
+                    e = ilogbf(sh) - ilogbf(tg);
+                    if (ldexpf(sh, -e) < tg) --e;
+                }
             }
-            if (c == 0) shd[hl] = sh;
+            int q1 = 0, q2 = 0;
+            if (sh > 0.0f) {
+                const float x = v[g] * scale_pow2(rsh, e);   // v / sigma_g
+                q1 = max(-127, min(127, __float2int_rn(x)));
+                q2 = max(-128, min(127, __float2int_rn((x - (float)q1) * 256.0f)));
+            }
+            // p_g = 2^(-e - 2g), a normal number unless the query is degenerate
+            const int pe = 127 - e - 2 * g;
+            sig[g] = pe >= 1 ? __uint_as_float((uint32_t)pe << 23) : ldexpf(1.0f, -e - 2 * g);
+            const int c = lane + 32 * g;
+            q8[(h * 2 + 0) * D + c] = (signed char)q1;
+            q8[(h * 2 + 1) * D + c] = (signed char)q2;
+            // kept channels ascending: earlier groups, then lanes below
+            if (qo.sel && ((kmask[g] >> lane) & 1u))
+                qo.sel[((size_t)b * hq + hg) * nk + before + __popc(kmask[g] & ((1u << lane) - 1u))] = (int16_t)c;
+            before += __popc(kmask[g]);
         }
-        __syncthreads();
-        if (!waited) {
-            grid_dependency_wait();     // earlier work on the stream (e.g. a cache append) is complete
-            grid_dependents_launch();   // the attend kernel may start streaming pages now
-            waited = true;
-        }
-        if (active) {
-            // kept channels before c: earlier warps of this head, then lanes below
-            int before = __popc(bal & ((1u << lane) - 1u));
-            for (int w = warp - (warp % kWarpsPerHead); w < warp; ++w) before += wcount[w];
-            if (sel_out && keep) sel_out[((size_t)b * hq + h) * nk + before] = (int16_t)c;
-            if (c == 0) q0[(size_t)b * hq + h] = qs;
-        }
-        __syncthreads();
-    }
-    // lay out the B-operand fragments
-    const size_t bj = (size_t)b * hkv + j;
-    for (int idx = threadIdx.x; idx < NT * NG * 32; idx += blockDim.x) {
-        const int L = idx & 31, g = (idx >> 5) % NG, nt = (idx >> 5) / NG;
-        const int gid = L >> 2, tig = L & 3, hl = 4 * nt + (gid >> 1), piece = gid & 1;
-        uint32_t w0 = 0, w1 = 0;
-        if (hl < G) {
-            const unsigned char *r = reinterpret_cast<const unsigned char *>(&q8[(hl * 2 + piece) * D + 32 * g]);
+        if (lane == 0) qo.q0[(size_t)b * hq + hg] = qs[0];
+        __syncwarp();
+
+        // this head's lanes of the fragments: 8 lanes (gid = 2 hh + piece) per group
+        const size_t bj = (size_t)b * hkv + j;
+        for (int idx = lane; idx < 8 * NG; idx += 32) {
+            const int L = 8 * hh + (idx & 7), gg = idx >> 3;
+            const int gid = L >> 2, tig = L & 3, piece = gid & 1;
+            const unsigned char *r = reinterpret_cast<const unsigned char *>(&q8[(h * 2 + piece) * D + 32 * gg]);
+            uint32_t w0 = 0, w1 = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 w0 |= (uint32_t)r[4 * tig + i] << (8 * i);
                 w1 |= (uint32_t)r[16 + 4 * tig + i] << (8 * i);
             }
+            qo.qf[((bj * NT + nt) * NG + gg) * 32 + L] = make_uint2(w0, w1);
         }
-        qf[((bj * NT + nt) * NG + g) * 32 + L] = make_uint2(w0, w1);
-    }
-    for (int idx = threadIdx.x; idx < NT * (NG + 1) * 4; idx += blockDim.x) {
-        const int hh = idx & 3, g = (idx >> 2) % (NG + 1), nt = (idx >> 2) / (NG + 1), hl = 4 * nt + hh;
-        qk[((bj * NT + nt) * (NG + 1) + g) * 4 + hh] = hl < G ? (g < NG ? sig[hl * NG + g] : shd[hl]) : 0.0f;
-    }
-    for (int idx = threadIdx.x; idx < NT * 32; idx += blockDim.x) {
-        const int L = idx & 31, nt = idx >> 5;
-        const int gid = L >> 2, tig = L & 3, hl = 4 * nt + (gid >> 1);
-        uint32_t w = 0;
-        if (hl < G && (gid & 1) == 0) {
-            // rows k = 2*tig, 2*tig + 1: piece k / NG (0 high, 1 low) of group k % NG
-            const int k0 = 2 * tig, k1 = 2 * tig + 1;
-            const uint32_t r0 = k0 < 2 * NG ? f16_piece(qsum[hl * NG + k0 % NG], k0 / NG) : 0u;
-            const uint32_t r1 = k1 < 2 * NG ? f16_piece(qsum[hl * NG + k1 % NG], k1 / NG) : 0u;
-            w = r0 | (r1 << 16);
+#pragma unroll
+        for (int g = 0; g <= NG; ++g)
+            if (lane == g) qo.qk[((bj * NT + nt) * (NG + 1) + g) * 4 + hh] = g < NG ? sig[g] : sh;
+        if (lane < 8) {
+            const int L = 8 * hh + lane, gid = L >> 2, tig = L & 3;
+            uint32_t w = 0;
+            if ((gid & 1) == 0) {
+                // rows k = 2*tig, 2*tig + 1: piece k / NG (0 high, 1 low) of group k % NG
+                const int k0 = 2 * tig, k1 = 2 * tig + 1;
+                float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+                for (int g = 0; g < NG; ++g) {
+                    if (k0 % NG == g) s0 = gs[g];
+                    if (k1 % NG == g) s1 = gs[g];
+                }
+                const uint32_t r0 = k0 < 2 * NG ? f16_piece(s0, k0 / NG) : 0u;
+                const uint32_t r1 = k1 < 2 * NG ? f16_piece(s1, k1 / NG) : 0u;
+                w = r0 | (r1 << 16);
+            }
+            qo.qm[(bj * NT + nt) * 32 + L] = w;
         }
-        qm[(bj * NT + nt) * 32 + L] = w;
-    }
-    if (write_first) {
-        grid_dependency_wait();     // the append is complete
-        grid_dependents_launch();   // the attend kernel may start streaming pages now
+        // the head slots of a 4-head tile that no query head fills (G < 4)
+        if (G < 4 && h == 0) {
+            for (int idx = lane; idx < (4 - G) * 8 * (NG + 2); idx += 32) {
+                const int hs = G + idx / (8 * (NG + 2)), rem = idx % (8 * (NG + 2));
+                const int L = 8 * hs + (rem & 7), part = rem >> 3;   // part < NG: qf of group part
+                if (part < NG) qo.qf[((bj * NT) * NG + part) * 32 + L] = make_uint2(0u, 0u);
+                else if (part == NG) qo.qm[(bj * NT) * 32 + L] = 0u;
+                else if ((rem & 7) <= NG) qo.qk[((bj * NT) * (NG + 1) + (rem & 7)) * 4 + hs] = 0.0f;
+            }
+        }
     }
 }
 

@@ -24,7 +24,7 @@ DQK_ERR_CUDA, DQK_ERR_DEVICE_BOUNDS, DQK_ERR_TIMEOUT = 4, 5, 6
 DQK_F32, DQK_BF16 = 0, 1
 
 EXPORTED = ["dqk_block_bytes", "dqk_append", "dqk_decode_workspace_size", "dqk_decode",
-            "dqk_decode_step", "dqk_decode_partial", "dqk_merge_partials", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine",
+            "dqk_decode_step", "dqk_decode_partial", "dqk_merge_partials", "dqk_test_decode_stall",
             "dqk_decode_noalloc", "dqk_bf16_block_bytes", "dqk_bf16_append",
             "dqk_bf16_decode_workspace_size", "dqk_bf16_decode", "dqk_last_device_error", "dqk_status_string"]
 
@@ -46,7 +46,7 @@ _lib.dqk_append.restype = C.c_int
 _lib.dqk_append.argtypes = [_D, _P, _P, C.c_int, C.c_int, _P, _P, C.c_int, _P, C.c_int, _P]
 _lib.dqk_decode_workspace_size.restype = C.c_size_t
 _lib.dqk_decode_workspace_size.argtypes = [_D, C.c_int, C.c_int]
-for _n in ("dqk_decode", "dqk_decode_partial", "dqk_decode_prepare", "dqk_decode_attend", "dqk_decode_combine"):
+for _n in ("dqk_decode", "dqk_decode_partial", "dqk_test_decode_stall"):
     getattr(_lib, _n).restype = C.c_int
     getattr(_lib, _n).argtypes = [_D, _P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P,
                                   C.c_size_t, _P]
@@ -155,23 +155,11 @@ def dqk_merge_partials(parts, n_parts, batch, num_q_heads, head_dim, out, stream
     return _check(st, "dqk_merge_partials", raise_on_error)
 
 
-def dqk_decode_prepare(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out,
-                       sel_out, workspace, workspace_bytes, stream=None, raise_on_error=True) -> int:
-    return _decode(_lib.dqk_decode_prepare, "dqk_decode_prepare", layer, q, q_dtype, batch, seq_lens,
-                   page_table, max_pages, sparsity_pct, out, sel_out, workspace, workspace_bytes, stream,
-                   raise_on_error)
-
-
-def dqk_decode_attend(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out,
-                      sel_out, workspace, workspace_bytes, stream=None, raise_on_error=True) -> int:
-    return _decode(_lib.dqk_decode_attend, "dqk_decode_attend", layer, q, q_dtype, batch, seq_lens,
-                   page_table, max_pages, sparsity_pct, out, sel_out, workspace, workspace_bytes, stream,
-                   raise_on_error)
-
-
-def dqk_decode_combine(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out,
-                       sel_out, workspace, workspace_bytes, stream=None, raise_on_error=True) -> int:
-    return _decode(_lib.dqk_decode_combine, "dqk_decode_combine", layer, q, q_dtype, batch, seq_lens,
+def dqk_test_decode_stall(layer, q, q_dtype, batch, seq_lens, page_table, max_pages, sparsity_pct, out,
+                          sel_out, workspace, workspace_bytes, stream=None, raise_on_error=True) -> int:
+    """Test only: dqk_decode with a stalled ring stage and 1 ms ring waits
+    (see include/dualqk.h); the device error word then reads DQK_ERR_TIMEOUT."""
+    return _decode(_lib.dqk_test_decode_stall, "dqk_test_decode_stall", layer, q, q_dtype, batch, seq_lens,
                    page_table, max_pages, sparsity_pct, out, sel_out, workspace, workspace_bytes, stream,
                    raise_on_error)
 

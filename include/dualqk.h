@@ -166,9 +166,14 @@ size_t dqk_decode_workspace_size(const dqk_layer_desc *layer, int batch, int max
  *               initialisation and are scratch after the call.
  * q' = fp32(fp64 sequential T_Q q); s_t = q'_S . k^'_t / sqrt(d) over the
  * kept channels with k^' = min + code*scale (BF16 value for channel 0);
- * out = softmax(s) . v^.  Computed as split-K flash decoding: per split an
- * online softmax with fp32 partials (m, l, o), then a log-sum-exp combine.
- * Equal to dqk_decode_prepare + dqk_decode_attend + dqk_decode_combine.
+ * out = softmax(s) . v^.  Computed as split-K flash decoding in one
+ * cooperative kernel launch (one CTA per SM): the query transform and
+ * selection of every head spread over the CTAs, a grid barrier, the online
+ * softmax over each CTA's share of the pages with fp32 partials (m, l, o),
+ * a second grid barrier, then the log-sum-exp merge of each head's
+ * partials.  The kernel is launched with programmatic stream serialization
+ * where the device accepts it together with the cooperative attribute; it
+ * waits for the previous kernel of the stream before reading anything.
  */
 dqk_status dqk_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype, int batch,
                       const int *seq_lens, const int *page_table, int max_pages,
@@ -183,11 +188,11 @@ dqk_status dqk_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dt
  *  seq_lens must already count the new rows.  All arguments of both parts are
  *  checked before anything is launched.
  *  Result: the same bytes as dqk_append followed by dqk_decode on `stream`.
- *  The difference is on the GPU: the query transform and selection run while
- *  the append is still writing the cache (the query kernel reads only q and
- *  T_Q and writes only the workspace, so it writes its results at once and
- *  waits for the append as its last step), and the attention kernel starts
- *  streaming pages as soon as both have finished. */
+ *  With max_new <= 4 the append runs inside the decode kernel: its rows are
+ *  transformed and packed by the CTAs' prologues next to the query work, and
+ *  every page at or past the first page an append touches is read only
+ *  after the grid barrier that follows them; longer appends run as their
+ *  own kernel first. */
 dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const void *v,
                            dqk_dtype kv_dtype, const int *new_lens, const int *seq_lens_before,
                            int max_new, const void *q, dqk_dtype q_dtype, int batch,
@@ -198,8 +203,9 @@ dqk_status dqk_decode_step(const dqk_layer_desc *layer, const void *k, const voi
 /* Context-parallel decode (one sequence's pages spread over several GPUs):
  * each rank decodes the pages it holds with dqk_decode_partial, the ranks
  * exchange their records (an all-gather over NCCL), and dqk_merge_partials
- * forms the output.  Passage: the split-K combine of the decode path, taken
- * across ranks; the pages' attention is over the whole context.
+ * forms the output.  The pages say nothing about splitting the context or
+ * merging partial softmax results; this is flash decoding's log-sum-exp
+ * merge carried across ranks, exact up to fp32 rounding.
  *
  * dqk_decode_partial -- dqk_decode over the cached tokens this caller holds
  * (its own pool, page table and token counts seq_lens), writing instead of
@@ -220,20 +226,18 @@ dqk_status dqk_decode_partial(const dqk_layer_desc *layer, const void *q, dqk_dt
 dqk_status dqk_merge_partials(const float *parts, int n_parts, int batch, int num_q_heads,
                               int head_dim, float *out, dqk_stream_t stream);
 
-/* The three stages of dqk_decode, exported so callers can place or time them
- * separately.  Same arguments; each uses the ones its stage needs. */
-dqk_status dqk_decode_prepare(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
-                              int batch, const int *seq_lens, const int *page_table,
-                              int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
-                              void *workspace, size_t workspace_bytes, dqk_stream_t stream);
-dqk_status dqk_decode_attend(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
-                             int batch, const int *seq_lens, const int *page_table,
-                             int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
-                             void *workspace, size_t workspace_bytes, dqk_stream_t stream);
-dqk_status dqk_decode_combine(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
-                              int batch, const int *seq_lens, const int *page_table,
-                              int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
-                              void *workspace, size_t workspace_bytes, dqk_stream_t stream);
+/* dqk_test_decode_stall -- TEST ONLY: dqk_decode with a fault injected on
+ * the host's request, to exercise the bounded waits.  The producer warp of
+ * CTA 0 never arms its second ring stage and every ring wait gives up after
+ * 1 ms instead of 1 s: the consumers of CTA 0 stop waiting, the producer
+ * drains the copies it issued, every CTA still takes part in both grid
+ * barriers, and dqk_last_device_error() then returns DQK_ERR_TIMEOUT.  The
+ * outputs are undefined; nothing stays in flight and the next call is
+ * unaffected.  Arguments as dqk_decode.  The pages have no counterpart. */
+dqk_status dqk_test_decode_stall(const dqk_layer_desc *layer, const void *q, dqk_dtype q_dtype,
+                                 int batch, const int *seq_lens, const int *page_table,
+                                 int max_pages, int sparsity_pct, float *out, int16_t *sel_out,
+                                 void *workspace, size_t workspace_bytes, dqk_stream_t stream);
 
 /* Largest workspace dqk_decode_noalloc can serve: 8 MiB of static device
  * memory per device that loads the library. */

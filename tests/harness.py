@@ -10,6 +10,8 @@ for the same seeded workload.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -18,6 +20,7 @@ from bit_kv_cache_dqk_b200 import inputs as I
 from oracle import oracle as O
 
 ATOL = 2e-3          # max abs error on fp32 outputs
+PARITY_RECORDS = []  # (test, max abs error, max row-relative error) of every output comparison
 RTOL_ROW = 1e-2      # relative error per output row (||o - o_ref|| / ||o_ref||)
 
 
@@ -260,13 +263,17 @@ def assert_cache_matches_oracle(run: DeviceRun, ref: dict):
 
 def assert_outputs_close(out: np.ndarray, ref: np.ndarray, atol: float = ATOL, rtol_row: float = RTOL_ROW):
     err = np.abs(out - ref)
-    assert np.isfinite(out).all(), "non-finite outputs"
-    assert err.max() <= atol, f"max abs error {err.max():.3e} > {atol}"
     num = np.linalg.norm((out - ref).reshape(-1, out.shape[-1]), axis=1)
     den = np.linalg.norm(ref.reshape(-1, ref.shape[-1]), axis=1)
     rel = num / np.maximum(den, 1e-30)
     ok = den > 0
+    worst_abs = float(np.nanmax(err)) if err.size else 0.0
+    worst_rel = float(np.nanmax(rel[ok])) if ok.any() else 0.0
+    name = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    PARITY_RECORDS.append((name, worst_abs, worst_rel))
+    print(f"[parity] max abs err {worst_abs:.3e}, max row rel err {worst_rel:.3e}")
+    assert np.isfinite(out).all(), "non-finite outputs"
+    assert err.max() <= atol, f"max abs error {err.max():.3e} > {atol}"
     if ok.any():
         assert rel[ok].max() <= rtol_row, f"row relative error {rel[ok].max():.3e} > {rtol_row}"
-    print(f"[parity] max abs err {err.max():.3e}, max row rel err {rel[ok].max() if ok.any() else 0.0:.3e}")
-    return float(err.max()), float(rel[ok].max()) if ok.any() else 0.0
+    return worst_abs, worst_rel

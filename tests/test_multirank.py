@@ -90,3 +90,21 @@ def test_reference_arm_line():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gpus_flag_launches_ranks_and_reports_max_over_ranks():
+    """`bench.py --gpus 2` with no outer launcher runs two ranks itself (under
+    torch.distributed.run); the CPU self-test step sleeps (rank + 1) ms, so the
+    slowest rank sets the time and rank 0 alone prints one JSON line."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                           "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--cpu-selftest",
+                        "--steps", "20", "--warmup", "3"], capture_output=True, text=True, timeout=300, env=env,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stdout + r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2
+    assert line["ms_per_step"] >= 2.0          # rank 1's 2 ms steps, not rank 0's 1 ms
+    assert line["value"] == pytest.approx(2 * 1000 / (line["ms_per_step"] / 1e3), rel=1e-6)
