@@ -3,12 +3,12 @@
 Each rank holds a contiguous range of every sequence's logical pages (its own
 pool and page table), decodes them with ``dqk_decode_partial`` into one
 (m, l, o) record per (sequence, query head), the ranks all-gather the records
-over NCCL, and ``dqk_merge_partials`` forms the output on every rank.  This is
-the split-K combine of the decode path ("How does Dual-QK compress KV caches
-to 2-bit while keeping accuracy at 128K context?", decode section: split-K
-attention over the pruned channels with a log-sum-exp combine) carried across
-GPUs; the exchange is B * Hq * (d + 2) * 4 bytes per rank, so it is latency-
-bound and NCCL's all-gather is the whole of it.
+over NCCL, and ``dqk_merge_partials`` forms the output on every rank.  The
+pages say nothing about how the context is split or where; the merge is the
+log-sum-exp combination of partial softmax results that the single-GPU decode
+already uses between its CTAs, carried across GPUs.  The exchange is
+B * Hq * (d + 2) * 4 bytes per rank, so it is latency-bound and NCCL's
+all-gather is the whole of it.
 
 Host logic only: every step of the decode and the merge runs in libdualqk.
 """

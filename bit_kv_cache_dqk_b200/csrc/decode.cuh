@@ -23,8 +23,6 @@
 // workspace needs no initialisation.
 #pragma once
 
-#include <cuda.h>
-
 #include "append.cuh"
 #include "attend.cuh"
 #include "common.cuh"
@@ -37,8 +35,6 @@ namespace dqk {
 // kernels take it as a __grid_constant__ parameter: the tensor maps of the
 // transforms are read from parameter space by the bulk tensor copies.
 struct DecodeParams {
-    CUtensorMap tmap_q;          // T_Q [Hkv * D rows][D] fp32: 32 x D boxes, 128-byte swizzle
-    CUtensorMap tmap_k;          // T_K, the same (used by the step's appends)
     AttendParams a;
     uint8_t *pool_w;             // the pool, for the step's appends
     // query prep
@@ -58,13 +54,15 @@ struct DecodeParams {
     // bounds of the ring waits and of the grid barriers; test-only stall
     unsigned long long ring_wait_ns, grid_wait_ns;
     int stall;
+    // shared memory between the ring and the barriers (bytes, a multiple of 16)
+    int tail;
 };
 
 constexpr int kBarRing = 1, kBarConsumers = 2, kBarSlot0 = 3, kBarBusy = 4;   // named barriers (0 is __syncthreads)
 constexpr int kFuseMaxNew = 4;   // decode steps append up to this many rows per sequence inside the kernel
 
-// Shared memory besides the ring: full[kMaxStages], empty[kMaxStages], opened,
-// tbar, valid flags [kMaxStages][stage blocks], abort flag (16 B), the merge
+// Shared memory besides the ring: full[kMaxStages], empty[kMaxStages], opened
+// (and one spare word), valid flags [kMaxStages][stage blocks], abort flag (16 B), the merge
 // plan (one MergeHead per consumer warp), then the per-warp score fragments
 // of two-tile (G = 8) kernels.
 constexpr int kBarBytes = (2 * kMaxStages + 2) * 8;
@@ -74,42 +72,37 @@ __host__ __device__ constexpr size_t decode_fixed_smem(int stage_blocks, int war
            (NT > 1 ? (size_t)warps * NT * NG * (32 * 8 + 4 * 16) : 0);
 }
 
-// Shared memory of an append task (1024-byte aligned): T_K[j] [D][D] fp32
-// (swizzled boxes), the key rows [D][kFuseMaxNew] fp64 (i-major), the store
-// images of one row.
+// Shared memory of an append task (16-byte aligned): T_K[j] in padded rows,
+// the key rows [D][kFuseMaxNew] fp64 (i-major), the store images of one row.
 template <int D, int NS>
 __host__ __device__ constexpr size_t append_scratch_bytes() {
-    return (size_t)D * D * 4 + (size_t)kFuseMaxNew * D * 8 + sizeof(RowStoreScratch<D, NS, 1>);
+    return (size_t)D * pad_row_bytes<D>() + (size_t)kFuseMaxNew * D * 8 + sizeof(RowStoreScratch<D, NS, 1>);
 }
 
-// Prologue scratch of one task (the largest of the two kinds) plus the
-// 1024-byte alignment of the swizzled boxes.
+// Prologue scratch of one task (the largest of the two kinds) plus its
+// 16-byte alignment.
 template <int D, int NS>
 __host__ __device__ constexpr size_t prologue_scratch_bytes(int G) {
     const size_t a = qprep_scratch_bytes<D>(G), b = append_scratch_bytes<D, NS>();
-    return (a > b ? a : b) + 1024;
+    return (a > b ? a : b) + 16;
 }
 
 // The rows sequence b appends in this launch (at most kFuseMaxNew), kv head
-// j, by the nthreads consumer threads of the CTA: T_K[j] staged like T_Q in
-// the query task, then thread c < D computes k'_c of every row (interleaved
-// fp64 sequential sums) and the D threads quantize and store the rows one
-// after the other -- the arithmetic, hence the bytes, of k_append_rows.
-template <int D, int NS, typename Meanwhile>
-__device__ void append_kv(const DecodeParams &dp, int b, int j, int t, int nthreads, unsigned char *scratch,
-                          uint64_t *tbar, uint32_t &tphase, Meanwhile meanwhile) {
+// j, by the NTH consumer threads of the CTA: T_K[j] staged like T_Q in the
+// query task, then thread c < D computes k'_c of every row (interleaved fp64
+// sequential sums) and the D threads quantize and store the rows one after
+// the other -- the arithmetic, hence the bytes, of k_append_rows.
+template <int D, int NS, int NTH, typename Meanwhile>
+__device__ void append_kv(const DecodeParams &dp, int b, int j, int t, unsigned char *scratch, Meanwhile meanwhile) {
     const AttendParams &p = dp.a;
+    constexpr int nthreads = NTH;
     const int n = min(dp.new_lens[b], kFuseMaxNew);
     if (n <= 0) return;   // uniform over the CTA
     const int L0 = dp.seq_before[b], lane = t & 31;
-    double *xs = reinterpret_cast<double *>(scratch + (size_t)D * D * 4);   // [D][kFuseMaxNew]
+    double *xs = reinterpret_cast<double *>(scratch + (size_t)D * pad_row_bytes<D>());   // [D][kFuseMaxNew]
     RowStoreScratch<D, NS, 1> &S = *reinterpret_cast<RowStoreScratch<D, NS, 1> *>(xs + kFuseMaxNew * D);
     named_bar_sync(kBarConsumers, nthreads);   // the previous task is done with the scratch
-    if (t == 0) {
-        fence_proxy_async_shared();
-        mbar_arrive_expect_tx(tbar, D * D * 4);
-        stage_matrix<D>(scratch, &dp.tmap_k, j, tbar);
-    }
+    stage_rows<D, NTH>(scratch, dp.t_k + (size_t)j * D * D, t);
     int row0 = 0;   // rows of sequences 0..b-1 come first
     for (int bb = lane; bb < b; bb += 32) row0 += dp.new_lens[bb];
 #pragma unroll
@@ -119,8 +112,6 @@ __device__ void append_kv(const DecodeParams &dp, int b, int j, int t, int nthre
         xs[c * kFuseMaxNew + r] =
             r < n ? (double)load_elem(dp.k_in, dp.kv_dtype, (((size_t)row0 + r) * p.hkv + j) * D + c) : 0.0;
     }
-    if (!mbar_wait_bounded(tbar, tphase, dp.ring_wait_ns)) dqk_flag_error(kErrTimeout);
-    tphase ^= 1u;
     named_bar_sync(kBarConsumers, nthreads);
     if (t >= D) {
         meanwhile();
@@ -128,7 +119,7 @@ __device__ void append_kv(const DecodeParams &dp, int b, int j, int t, int nthre
     }
     const int c = t;
     double acc[kFuseMaxNew];
-    dot_rows_swz<D, kFuseMaxNew>(scratch, c, xs, kFuseMaxNew, acc);
+    dot_rows_pad<D, kFuseMaxNew>(scratch, c, xs, kFuseMaxNew, acc);
 #pragma unroll
     for (int r = 0; r < kFuseMaxNew; ++r) {
         if (r >= n) break;   // uniform
@@ -384,10 +375,9 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
     const int S = p.stages;
     const uint32_t stage_bytes = (uint32_t)(kStageBlocks * p.bb);
     unsigned char *stage_mem = attend_smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(attend_smem + (size_t)S * stage_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(attend_smem + (size_t)S * stage_bytes + dp.tail);
     uint64_t *empty = full + kMaxStages;
     uint64_t *opened = empty + kMaxStages;
-    uint64_t *tbar = opened + 1;   // the prologue's staged matrix rows
     unsigned char *valid = reinterpret_cast<unsigned char *>(full) + kBarBytes;   // [kMaxStages][kStageBlocks]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(valid + kMaxStages * kStageBlocks);
     MergeHead *plan = reinterpret_cast<MergeHead *>(valid + kMaxStages * kStageBlocks + 16);
@@ -397,6 +387,21 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
+    // The transforms this CTA's prologue tasks stage (task k runs on CTA k mod
+    // C): into L2 and the descriptor cache already, while the kernel before
+    // this one may still run (a prefetch returns no data).
+    if (threadIdx.x == 0) {
+        const int n_app = dp.max_new > 0 ? p.batch * p.hkv : 0;
+        const int n_tasks = n_app + p.batch * p.hkv;
+        if ((int)blockIdx.x < n_tasks) {
+            const uint64_t keep = l2_policy_evict_last();
+            for (int k = (int)blockIdx.x; k < n_tasks; k += (int)gridDim.x) {
+                const bool app = k < n_app;
+                const int j = (app ? k : k - n_app) % p.hkv;
+                bulk_prefetch_l2((app ? dp.t_k : dp.t_q) + (size_t)j * D * D, D * D * 4, keep);
+            }
+        }
+    }
     // launched with programmatic serialization: everything read below may come
     // from the kernel before this one on the stream
     grid_dependency_wait();
@@ -418,13 +423,14 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
         __syncwarp();
         named_bar_arrive(kBarRing, attend_threads(G));
     }
-    // the prologue works in the last ring stages, which the producer fills only
-    // once `opened` completes
+    // the prologue works in the last ring stages and the tail after them; the
+    // producer fills those stages only once `opened` completes
     const uint32_t scratch_bytes = (uint32_t)prologue_scratch_bytes<D, NS>(G);
-    const int scratch_stages = (int)((scratch_bytes + stage_bytes - 1) / stage_bytes);
+    const uint32_t tail = (uint32_t)dp.tail;
+    const int scratch_stages =
+        scratch_bytes > tail ? (int)((scratch_bytes - tail + stage_bytes - 1) / stage_bytes) : 0;
     unsigned char *scratch_raw = stage_mem + (size_t)(S - scratch_stages) * stage_bytes;
-    // (aligned in the shared window: the swizzle pattern follows shared-address bits)
-    unsigned char *scratch = scratch_raw + ((1024u - (smem_addr(scratch_raw) & 1023u)) & 1023u);
+    unsigned char *scratch = scratch_raw + ((16u - (smem_addr(scratch_raw) & 15u)) & 15u);
 
     if (warp == kConsumerWarps) {
         const CtaUnits cu = cta_units(p.seq_lens, p.nchunks, R, blockIdx.x, p.num_ctas, lane);
@@ -439,8 +445,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
     // ------------------------------------------------------------- prologue
     // tasks = [the step's appends (sequence, kv head)] + [query prep (sequence,
     // kv head)], task k on CTA k mod C, each by all consumer warps of the CTA;
-    // they start at once (their own barrier, tbar, is set up here), and the
-    // CTA's bookkeeping (unit range, empty records, merge plan; results in
+    // the CTA's bookkeeping (unit range, empty records, merge plan; results in
     // shared memory) runs while the first task's loads are in flight
     CtaUnits *cu_sm = reinterpret_cast<CtaUnits *>(plan + 16);
     {
@@ -450,26 +455,20 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
         // after the tasks)
         constexpr int kFirst = (D / 32 > G ? D / 32 : G);
         constexpr int kThreads = 32 * kConsumerWarps;
-        if (threadIdx.x == 0) {
-            mbar_init(tbar, 1);
-            fence_mbar_init();
-        }
         const QueryOut qo{const_cast<uint2 *>(p.qf), const_cast<float *>(p.qk), const_cast<uint32_t *>(p.qm),
                           const_cast<float *>(p.q0), dp.sel_out};
         const int n_app = dp.max_new > 0 ? p.batch * p.hkv : 0;
         const int n_tasks = n_app + p.batch * p.hkv;
-        uint32_t tphase = 0;
         bool done = false;
         for (int k = (int)blockIdx.x; k < n_tasks; k += (int)gridDim.x) {
             const Bookkeeping<D, G> bkk{&p, cu_sm, plan, R, warp, lane, k < n_app ? D / 32 : kFirst};
             const BookkeepingOnce<D, G> once{&bkk, !done && bkk.first < kConsumerWarps};
             if (k < n_app) {
-                append_kv<D, NS>(dp, k / p.hkv, k % p.hkv, threadIdx.x, kThreads, scratch, tbar, tphase, once);
+                append_kv<D, NS, kThreads>(dp, k / p.hkv, k % p.hkv, threadIdx.x, scratch, once);
             } else {
                 const int u = k - n_app;
-                qprep_kv<D, G>(&dp.tmap_q, dp.q, dp.q_dtype, p.hq, p.hkv, dp.pct, dp.qscale, u / p.hkv, u % p.hkv,
-                               threadIdx.x, kThreads, kBarConsumers, kBarBusy, scratch, tbar, tphase, dp.ring_wait_ns,
-                               qo, once);
+                qprep_kv<D, G, kThreads>(dp.t_q, dp.q, dp.q_dtype, p.hq, p.hkv, dp.pct, dp.qscale, u / p.hkv,
+                                         u % p.hkv, threadIdx.x, kBarConsumers, kBarBusy, scratch, qo, once);
             }
             done = done || bkk.first < kConsumerWarps;
         }
@@ -602,12 +601,14 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
         const uint32_t page_gap = (uint32_t)(p.hc * p.bb);
         // n (1 .. BPW-1) full pages of one run at shared addresses base + q * page_gap
         auto consume_batch = [&](int n, uint32_t base) {
-            if constexpr (BPW == 4) {
+            if constexpr (BPW >= 4) {
                 if (n == 3) {
                     const uint32_t sb3[3] = {base, base + page_gap, base + 2 * page_gap};
                     consume<D, G, VCH0, NS, 3, false>(sb3, kPage, st, lane, lo);
                     return;
                 }
+            }
+            if constexpr (BPW >= 3) {
                 if (n == 2) {
                     const uint32_t sb2[2] = {base, base + page_gap};
                     consume<D, G, VCH0, NS, 2, false>(sb2, kPage, st, lane, lo);

@@ -1,8 +1,6 @@
 // dualqk.cu -- libdualqk: host side of the C ABI declared in include/dualqk.h
 // (argument checks, launch planning) and the single translation unit that
 // holds every kernel of the decode hot path.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -57,7 +55,7 @@ int device_sms(int dev) {
 // Decode plan and workspace layout: [header | qf | qk | qm | q0 | split
 // records], every section 256-byte aligned.
 struct DecodePlan {
-    int d, G, NT, NG, hc, pps, pw, nchunks, num_ctas, stages, bb, threads;
+    int d, G, NT, NG, hc, pps, pw, nchunks, num_ctas, stages, bb, threads, tail;
     size_t off_qf, off_qk, off_qm, off_q0, off_part, bytes, smem;
 };
 
@@ -104,12 +102,16 @@ bool plan_decode(const dqk_layer_desc *L, int batch, DecodePlan &P) {
     const size_t budget = 227 * 1024;
     P.stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / stage_bytes);
     if (P.stages < 2) return false;
-    // the prologue works in the last stages (one at least stays free for the
-    // producer), the merge in the first
-    const size_t scratch_stages = (prologue_scratch(P.d, ns, P.G) + stage_bytes - 1) / stage_bytes;
+    // the shared memory left after the ring (a multiple of 16 bytes) follows
+    // it; the prologue works in the last stages and that tail (one stage at
+    // least stays free for the producer), the merge in the first stage
+    const size_t tail = P.stages == kMaxStages ? 0 : (budget - fixed - P.stages * stage_bytes) & ~(size_t)15;
+    P.tail = (int)tail;
+    const size_t scratch = prologue_scratch(P.d, ns, P.G);
+    const size_t scratch_stages = scratch > tail ? (scratch - tail + stage_bytes - 1) / stage_bytes : 0;
     if (scratch_stages >= (size_t)P.stages) return false;
     if ((size_t)warps * (P.d + 4) * sizeof(float) > stage_bytes) return false;
-    P.smem = P.stages * stage_bytes + fixed;
+    P.smem = P.stages * stage_bytes + tail + fixed;
     const size_t R = (size_t)batch * P.nchunks;
     const size_t bj = (size_t)batch * hkv;
     P.off_qf = 256;
@@ -195,34 +197,6 @@ dqk_status launch_cooperative(void (*kernel)(KArgs...), int dev, unsigned grid, 
     return e == cudaSuccess ? DQK_OK : DQK_ERR_CUDA;
 }
 
-// Tensor map of a layer's transforms [Hkv * d rows][d columns] fp32 for the
-// decode prologue's 2-D bulk tensor copies: boxes of 32 columns x d rows
-// with the 128-byte swizzle.  The encoder is the driver's, found through the
-// runtime's entry-point query (no link against the driver library).
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static std::once_flag once;
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    std::call_once(once, [] {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    });
-    return fn;
-}
-
-bool encode_transform_map(CUtensorMap *map, const float *t, int hkv, int d) {
-    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-    if (!encode || !t) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)hkv * d};
-    const cuuint64_t strides[1] = {(cuuint64_t)d * sizeof(float)};
-    const cuuint32_t box[2] = {32, (cuuint32_t)d};
-    const cuuint32_t elem[2] = {1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(t), dims, strides, box, elem,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 struct DecodeArgs {
     const dqk_layer_desc *L;
@@ -275,8 +249,6 @@ dqk_status run_decode_g(const DecodeArgs &a, const DecodePlan &P, int dev) {
     if (st != DQK_OK) return st;
     char *ws = static_cast<char *>(a.ws);
     DecodeParams dp = {};
-    if (!encode_transform_map(&dp.tmap_q, a.L->t_q, a.L->num_kv_heads, D)) return DQK_ERR_CUDA;
-    if (a.max_new > 0 && !encode_transform_map(&dp.tmap_k, a.L->t_k, a.L->num_kv_heads, D)) return DQK_ERR_CUDA;
     AttendParams &prm = dp.a;
     prm.pool = static_cast<const uint8_t *>(a.L->pool);
     prm.num_pages = a.L->num_pages;
@@ -318,6 +290,7 @@ dqk_status run_decode_g(const DecodeArgs &a, const DecodePlan &P, int dev) {
     dp.ring_wait_ns = a.stall ? kStallWaitNs : kRingWaitNs;
     dp.grid_wait_ns = kGridWaitNs;
     dp.stall = a.stall ? 1 : 0;
+    dp.tail = P.tail;
     return launch_cooperative(kernel, dev, (unsigned)P.num_ctas, (unsigned)P.threads, P.smem, a.stream, dp);
 }
 

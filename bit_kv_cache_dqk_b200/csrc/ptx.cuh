@@ -86,6 +86,13 @@ __device__ __forceinline__ void prefetch_l2(const void *ptr) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
 }
 
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) of global
+// memory into L2 with a cache policy; no data is returned.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *ptr, uint32_t bytes, uint64_t policy) {
+    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(ptr), "r"(bytes), "l"(policy)
+                 : "memory");
+}
+
 // Named barrier `id` over `n` threads: arrive without waiting, or arrive and
 // wait.  (Barrier 0 is __syncthreads.)
 __device__ __forceinline__ void named_bar_arrive(int id, int n) {
@@ -130,16 +137,6 @@ __device__ __forceinline__ void bulk_copy_g2s_hint(void *dst, const void *src, u
         : "memory");
 }
 
-// 2-D tiled bulk tensor copy global -> shared of the box at (x, y) of the
-// tensor map at `tmap` (a kernel-parameter address) with an L2 cache policy,
-// completion counted on `bar` (no multicast).
-__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
-        "%3}], [%4], %5;" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
-}
 
 // 4-byte asynchronous global -> shared copy (no register round trip), and the
 // wait for all of this thread's outstanding copies.
@@ -400,6 +397,9 @@ __device__ __forceinline__ uint32_t ld_s8(uint32_t a) {
     return v;
 }
 
+__device__ __forceinline__ void st_s32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v));
+}
 __device__ __forceinline__ void st_s64(uint32_t a, uint2 v) {
     asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(v.x), "r"(v.y));
 }

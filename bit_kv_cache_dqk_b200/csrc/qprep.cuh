@@ -45,42 +45,51 @@ __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
     return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
 }
 
-// A [D][D] fp32 transform staged by 2-D tensor copies: D/32 boxes of 32
-// columns x D rows, each row of a box 128 bytes whose 16-byte chunks are
-// XOR-permuted by (row mod 8) (the tensor map's 128-byte swizzle), so that
-// one thread per row reads 16-byte chunks without bank conflicts.  Byte
-// offset of columns 4u..4u+3 of box k, row r; the base is 1024-byte aligned.
+// A [D][D] fp32 transform staged in shared memory by the nthreads threads of
+// the caller (NTH of them, a compile-time count), with coalesced 16-byte
+// loads -- a warp reads 512 contiguous bytes, all of a thread's loads are in
+// flight before its first store -- into rows padded to D*4 + 16 bytes, so that
+// one thread per row then reads 16-byte chunks without bank conflicts (eight
+// consecutive rows cover the 32 banks).
 template <int D>
-__device__ __forceinline__ uint32_t swz_offset(int k, int r, int u) {
-    return (uint32_t)(k * D * 128 + r * 128 + ((u ^ (r & 7)) << 4));
-}
+__host__ __device__ constexpr int pad_row_bytes() { return D * 4 + 16; }
 
-// Issue the copies of matrix j (rows j*D ..) of the tensor map into dst; the
-// transforms are re-read by every launch, so they are kept in L2.
-template <int D>
-__device__ __forceinline__ void stage_matrix(unsigned char *dst, const void *tmap, int j, uint64_t *bar) {
-    const uint64_t keep = l2_policy_evict_last();
+template <int D, int NTH>
+__device__ __forceinline__ void stage_rows(unsigned char *dst, const float *__restrict__ src, int t) {
+    constexpr int Q = D / 4;                     // 16-byte chunks per row
+    constexpr int N = (D * Q + NTH - 1) / NTH;   // chunks per thread
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    float4 v[N];
 #pragma unroll
-    for (int k = 0; k < D / 32; ++k) tma_load_2d(dst + (size_t)k * D * 128, tmap, 32 * k, j * D, bar, keep);
+    for (int i = 0; i < N; ++i) {
+        const int q = t + i * NTH;
+        if (q < D * Q) v[i] = __ldg(s4 + q);
+    }
+    const uint32_t base = smem_addr(dst);
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int q = t + i * NTH;
+        if (q < D * Q) st_s128(base + (uint32_t)((q / Q) * pad_row_bytes<D>() + (q % Q) * 16), *reinterpret_cast<uint4 *>(&v[i]));
+    }
 }
 
 // Sum over i ascending of (double)T[row][i] * x[i * xs + n], one fused
 // multiply-add after the other for each of the NX vectors (fp32 x fp32
-// products are exact in fp64, so the result does not depend on contraction).
-// x is i-major (row stride xs doubles), so the NX values of a column come in
-// 16-byte loads.  Eight 16-byte chunks of the row per iteration.
+// products are exact in fp64, so the result does not depend on contraction),
+// T staged by stage_rows.  x is i-major (row stride xs doubles), so the NX
+// values of a column come in 16-byte loads.  Eight 16-byte chunks of the row
+// per iteration.
 template <int D, int NX>
-__device__ __forceinline__ void dot_rows_swz(const unsigned char *sT, int row, const double *x, int xs,
+__device__ __forceinline__ void dot_rows_pad(const unsigned char *sT, int row, const double *x, int xs,
                                              double (&acc)[NX]) {
 #pragma unroll
     for (int n = 0; n < NX; ++n) acc[n] = 0.0;
-    const int sw = row & 7;
-    const unsigned char *base = sT + row * 128;
+    const unsigned char *base = sT + row * pad_row_bytes<D>();
 #pragma unroll 1
     for (int k = 0; k < D / 32; ++k) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const float4 tv = *reinterpret_cast<const float4 *>(base + k * D * 128 + ((u ^ sw) << 4));
+            const float4 tv = *reinterpret_cast<const float4 *>(base + (32 * k + 4 * u) * 4);
             const double te[4] = {(double)tv.x, (double)tv.y, (double)tv.z, (double)tv.w};
             const double *xi = x + (32 * k + 4 * u) * xs;
 #pragma unroll
@@ -91,12 +100,12 @@ __device__ __forceinline__ void dot_rows_swz(const unsigned char *sT, int row, c
     }
 }
 
-// Shared memory of one query task (1024-byte aligned): T_Q[j] [D][D] fp32
-// (swizzled boxes; the q' values [G][D] reuse it once the sums are done), the
-// query rows [D][G] fp64 (i-major), the int8 pieces [G][2][D].
+// Shared memory of one query task (16-byte aligned): T_Q[j] in padded rows
+// (the q' values [G][D] fp32 reuse it once the sums are done), the query rows
+// [D][G] fp64 (i-major), the int8 pieces [G][2][D].
 template <int D>
 __host__ __device__ constexpr size_t qprep_scratch_bytes(int G) {
-    return (size_t)D * D * 4 + (size_t)G * D * 8 + (size_t)G * 2 * D;
+    return (size_t)D * pad_row_bytes<D>() + (size_t)G * D * 8 + (size_t)G * 2 * D;
 }
 
 // Channels (of this warp's NG per lane, channel 0 excluded) whose magnitude
@@ -130,46 +139,41 @@ __device__ __forceinline__ float scale_pow2(float x, int e) {
 //   threshold search, then writes head h's fragments and kept channels
 //   (ascending).
 // meanwhile(): work of the caller's that overlaps the loads of the task.
-template <int D, int G, typename Meanwhile>
-__device__ void qprep_kv(const void *tmap_q, const void *__restrict__ q, int dtype, int hq, int hkv, int pct,
-                         float qscale, int b, int j, int t, int nthreads, int bar, int busy_bar, unsigned char *scratch,
-                         uint64_t *tbar, uint32_t &tphase, uint64_t wait_ns, const QueryOut &qo, Meanwhile meanwhile) {
+template <int D, int G, int NTH, typename Meanwhile>
+__device__ void qprep_kv(const float *__restrict__ t_q, const void *__restrict__ q, int dtype, int hq, int hkv, int pct,
+                         float qscale, int b, int j, int t, int bar, int busy_bar, unsigned char *scratch,
+                         const QueryOut &qo, Meanwhile meanwhile) {
     constexpr int NG = D / 32;
     constexpr int NT = G > 4 ? 2 : 1;
+    constexpr int nthreads = NTH;
     const int warp = t >> 5, lane = t & 31;
     const int nk = keep_count(D, pct);
-    double *qin = reinterpret_cast<double *>(scratch + (size_t)D * D * 4);
+    double *qin = reinterpret_cast<double *>(scratch + (size_t)D * pad_row_bytes<D>());
     signed char *q8 = reinterpret_cast<signed char *>(qin + (size_t)G * D);
     float *qpv = reinterpret_cast<float *>(scratch);   // [G][D] after the sums
 
     // stage T_Q[j] and the G query rows
     named_bar_sync(bar, nthreads);   // the previous task is done with the scratch
-    if (t == 0) {
-        fence_proxy_async_shared();   // earlier generic accesses to the scratch come first
-        mbar_arrive_expect_tx(tbar, D * D * 4);
-        stage_matrix<D>(scratch, tmap_q, j, tbar);
-    }
+    stage_rows<D, NTH>(scratch, t_q + (size_t)j * D * D, t);
     const size_t qbase = ((size_t)b * hq + (size_t)j * G) * D;
     for (int i = t; i < G * D; i += nthreads) {   // query h, channel c -> qin[c][h]
         const int h = i / D, c = i - h * D;
         qin[c * G + h] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[qbase + i])
                                                       : reinterpret_cast<const float *>(q)[qbase + i]);
     }
-    named_bar_sync(bar, nthreads);   // the query rows are in
+    named_bar_sync(bar, nthreads);   // T_Q[j] and the query rows are in
     // the warps the task leaves idle run the caller's `meanwhile` work
     constexpr int kBusy = (D / 32 > G ? D / 32 : G);
     if (warp >= kBusy) {
         meanwhile();
         return;
     }
-    if (!mbar_wait_bounded(tbar, tphase, wait_ns)) dqk_flag_error(kErrTimeout);
-    tphase ^= 1u;
 
     // q'_c of every head: G interleaved sums per thread (thread c = row c),
     // ascending i, exact fp32 x fp32 products accumulated in fp64, one
     // rounding each
     double acc[G];
-    if (t < D) dot_rows_swz<D, G>(scratch, t, qin, G, acc);
+    if (t < D) dot_rows_pad<D, G>(scratch, t, qin, G, acc);
     named_bar_sync(busy_bar, 32 * kBusy);   // T_Q is dead
     if (t < D) {
 #pragma unroll
