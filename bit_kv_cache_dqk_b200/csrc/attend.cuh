@@ -25,11 +25,10 @@
 //                + sum_g min[t, g] * Qsum[g, h]   (one extra m16n8k16; the high and
 //                                                  low fp16 parts of Qsum in separate rows)
 //                + qs_0[h] * k0[t]                (BF16 channel 0, fp32)
-//        with p_g = 2^-e_g / 4^g.  The piece-1 accumulators start at 1.5 * 2^23
-//        and the piece-2 ones at 1.5 * 2^15, so as floats they read
-//        M1 + D1 and M2 + D2/256 exactly, and two FFMAs give
-//        p_g (D1 + D2/256) with one rounding: (M1 + D1) p - (M1 + M2) p is exact,
-//        then (M2 + D2/256) p is added.
+//        with p_g = 2^-e_g / 4^g.  256 D1 + D2 is exact in int32 (below 2^28);
+//        it becomes fp32 with one rounding, and scale[t, g] * p_g / 256 is
+//        exact (p_g a power of two), so one FFMA adds
+//        scale * p_g (D1 + D2/256) with the roundings of the definition.
 //   online softmax in base 2 (running max per head, exact rescale on growth)
 //   PV   O^T[c, h] += sum_t code_v[t, c] * (p~[t, h] * vscale[t, g(c)])
 //        with p~ = fp16(p); one extra m16n8k16 gives sum_t p~ * vmin[t, g] and
@@ -188,7 +187,7 @@ struct WarpState {
     using T = AttendTile<D, G>;
     static constexpr bool kRegFrags = T::NT == 1;   // score fragments in registers (else per-warp shared memory)
     uint2 qb[kRegFrags ? T::NG : 1];                // score B fragments of group g
-    float2 kp[kRegFrags ? T::NG : 1];               // p_g and -(M1 + M2) p_g of group g
+    float kq[kRegFrags ? T::NG : 1];                // p_g / 256 of group g
     float sgh[T::NT];              // sigma_h of this thread's head
     uint32_t qmin[T::NT];          // min-term B fragment
     float q0v[T::NT];              // scaled q'_0 of this thread's head
@@ -207,7 +206,7 @@ struct LaneOffsets {
     uint32_t vmin;     // V min pair of row min(gid, NG-1), tokens 2tig, 2tig+1
     int srcA;          // lane holding p of (token 2tig, head gid/2); +4: token 2tig+1
     uint32_t sq;       // shared address of this lane's QK B fragments: [NT][NG][32 lanes] uint2
-    uint32_t sk;       // shared address of this thread's head constants: [NT][NG][4 heads] 16-byte slots (p_g pair)
+    uint32_t sk;       // shared address of this thread's head constants: [NT][NG][4 heads] 16-byte slots (p_g / 256)
     uint32_t ones_lane, vmin_mask;
 };
 
@@ -280,16 +279,15 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
     for (int g = 0; g < NG; ++g) {
         const uint32_t msk = 0x03030303u << (2 * g);   // group g's field in every byte: code * 4^g
         uint2 qb[NT];
-        float2 kp[NT];
+        float kq[NT];
         if constexpr (WarpState<D, G>::kRegFrags) {
             qb[0] = st.qb[g];
-            kp[0] = st.kp[g];
+            kq[0] = st.kq[g];
         } else {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 qb[nt] = ld_s64(o.sq + (nt * NG + g) * 256);
-                const uint2 kpu = ld_s64(o.sk + (nt * NG + g) * 64);
-                kp[nt] = make_float2(__uint_as_float(kpu.x), __uint_as_float(kpu.y));
+                kq[nt] = __uint_as_float(ld_s32(o.sk + (nt * NG + g) * 64));
             }
         }
 #pragma unroll
@@ -313,13 +311,11 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 int dg[4];
-                mma_u8s8_c2(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y, kMagicI, kMagicLoI);
-                // p (D1 + D2/256): (M1 + D1) p - (M1 + M2) p exact, + (M2 + D2/256) p, one rounding
-                const float2 k2 = kp[nt];
-                const float x0 = fmaf(__int_as_float(dg[1]), k2.x, fmaf(__int_as_float(dg[0]), k2.x, k2.y));
-                const float x1 = fmaf(__int_as_float(dg[3]), k2.x, fmaf(__int_as_float(dg[2]), k2.x, k2.y));
-                a0[b][nt] = fmaf(sa, x0, a0[b][nt]);
-                a1[b][nt] = fmaf(sbv, x1, a1[b][nt]);
+                mma_u8s8(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y, 0);
+                // rows gid, gid + 8: 256 D1 + D2 (exact), one rounding to fp32
+                const float y0 = (float)(dg[0] * 256 + dg[1]), y1 = (float)(dg[2] * 256 + dg[3]);
+                a0[b][nt] = fmaf(sa * kq[nt], y0, a0[b][nt]);
+                a1[b][nt] = fmaf(sbv * kq[nt], y1, a1[b][nt]);
             }
         }
     }

@@ -522,15 +522,13 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
                 const uint2 qb = __ldcg(&p.qf[((bj * NT + nt) * NG + g) * 32 + lane]);
-                const float pg = __ldcg(&p.qk[((bj * NT + nt) * (NG + 1) + g) * 4 + tig]);
-                const float2 kp = make_float2(pg, -(kMagicF + kMagicLoF) * pg);   // exact: power-of-two p_g
+                const float kq = __ldcg(&p.qk[((bj * NT + nt) * (NG + 1) + g) * 4 + tig]) * (1.0f / 256.0f);
                 if constexpr (WarpState<D, G>::kRegFrags) {
                     st.qb[g] = qb;
-                    st.kp[g] = kp;
+                    st.kq[g] = kq;
                 } else {
                     st_s64(lo.sq + (nt * NG + g) * 256, qb);
-                    if (gid == 0)
-                        st_s64(lo.sk + (nt * NG + g) * 64, make_uint2(__float_as_uint(kp.x), __float_as_uint(kp.y)));
+                    if (gid == 0) st_s32(lo.sk + (nt * NG + g) * 64, __float_as_uint(kq));
                 }
             }
             st.sgh[nt] = __ldcg(&p.qk[((bj * NT + nt) * (NG + 1) + NG) * 4 + tig]);
