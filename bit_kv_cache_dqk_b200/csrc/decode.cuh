@@ -494,6 +494,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
     int r = cu.r, ur = cu.ur;
     int npr = r < R ? run_pages(p.seq_lens, p.nchunks, r) : 0;
     int cur_run = -1, run_end = -1, partial_u = -1, nv_last = kPage;
+    int fast_end = -1;   // a stage's pages below this unit are full pages of the current run and the CTA
 
     WarpState<D, G> st;
     LaneOffsets lo;
@@ -587,6 +588,7 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
         const int Lb = p.seq_lens[r / p.nchunks];
         partial_u = (Lb & (kPage - 1)) ? run_end - 1 : -1;
         nv_last = Lb - (npr - 1) * kPage;
+        fast_end = min(partial_u >= 0 ? partial_u : run_end, u1);
     };
 
     if (iters > 0) {
@@ -634,19 +636,21 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
                 const int ul = ua + BPW - 1;
                 // flags of the warp's page slots (one byte each), as a bit mask
                 const uint32_t va = valid_addr + stage * kStageBlocks;
-                uint32_t vv = 0;
+                uint32_t vv = 0, vw = 0;
                 if constexpr (BPW == 4) {
-                    const uint32_t w = ld_s32(va);
-                    vv = (w & 1u) | ((w >> 7) & 2u) | ((w >> 14) & 4u) | ((w >> 21) & 8u);
+                    vw = ld_s32(va);
+                    vv = (vw & 1u) | ((vw >> 7) & 2u) | ((vw >> 14) & 4u) | ((vw >> 21) & 8u);
                 } else if constexpr (BPW == 2) {
-                    const uint32_t w = ld_s16(va);
-                    vv = (w & 1u) | ((w >> 7) & 2u);
+                    vw = ld_s16(va);
+                    vv = (vw & 1u) | ((vw >> 7) & 2u);
                 } else {
 #pragma unroll
                     for (int q = 0; q < BPW; ++q) vv |= ld_s8(va + q) << q;
+                    vw = vv == kAllValid ? 0x01010101u : 0u;
                 }
+                constexpr uint32_t kAllValidBytes = BPW == 4 ? 0x01010101u : BPW == 2 ? 0x0101u : 0x01010101u;
                 if (ua >= run_end) switch_run(ua);
-                if (ul < run_end && ul < u1 && !(partial_u >= ua && partial_u <= ul) && vv == kAllValid) {
+                if (ul < fast_end && vw == kAllValidBytes) {
                     uint32_t sbb[BPW];
 #pragma unroll
                     for (int q = 0; q < BPW; ++q) sbb[q] = sa + q * page_gap;

@@ -118,6 +118,16 @@ __device__ __forceinline__ int count_ge(const uint32_t (&mag)[NG], bool ch0, uin
     return (int)__reduce_add_sync(0xffffffffu, n);
 }
 
+// The rare paths of the piece arithmetic (subnormal operands), kept out of
+// line: the prologue runs once per launch, so its code is fetched cold and
+// every inlined instruction costs.
+__device__ __noinline__ float ldexp_rare(float x, int e) { return ldexpf(x, e); }
+__device__ __noinline__ int exp_offset_rare(float sh, float tg) {
+    int e = ilogbf(sh) - ilogbf(tg);
+    if (ldexpf(sh, -e) < tg) --e;
+    return e;
+}
+
 // x * 2^e, exact: an exponent-field addition when x and the result are
 // normal, the library function otherwise.
 __device__ __forceinline__ float scale_pow2(float x, int e) {
@@ -125,7 +135,7 @@ __device__ __forceinline__ float scale_pow2(float x, int e) {
     const int ex = (int)((b >> 23) & 0xffu) + e;
     if (((b >> 23) & 0xffu) != 0u && ((b >> 23) & 0xffu) != 0xffu && ex >= 1 && ex <= 254)
         return __uint_as_float((b & 0x807fffffu) | ((uint32_t)ex << 23));
-    return ldexpf(x, e);
+    return ldexp_rare(x, e);
 }
 
 // The G query heads of (sequence b, kv head j), by the nthreads threads of
@@ -199,22 +209,37 @@ __device__ void qprep_kv(const float *__restrict__ t_q, const void *__restrict__
         }
         const bool ch0 = lane == 0;   // channel 0 (g = 0) takes no part
         uint32_t T = 0;
-        // bit 30 alone, then two bits per step (three candidates counted at once)
-        if (count_ge<NG>(mag, ch0, 1u << 30) >= m) T = 1u << 30;
+        int cnt = D - 1;   // channels >= T
+        // bit 30 alone, then two bits per step (three candidates counted at
+        // once); done as soon as exactly m channels are >= T (the prefix then
+        // separates the kept channels from the others)
+        {
+            const int n = count_ge<NG>(mag, ch0, 1u << 30);
+            if (n >= m) {
+                T = 1u << 30;
+                cnt = n;
+            }
+        }
 #pragma unroll 1
-        for (int bit = 28; bit >= 0; bit -= 2) {
+        for (int bit = 28; bit >= 0 && cnt != m; bit -= 2) {
             const int n3 = count_ge<NG>(mag, ch0, T | (3u << bit)), n2 = count_ge<NG>(mag, ch0, T | (2u << bit)),
                       n1 = count_ge<NG>(mag, ch0, T | (1u << bit));
-            T |= (n3 >= m ? 3u : n2 >= m ? 2u : n1 >= m ? 1u : 0u) << bit;
+            const uint32_t d = n3 >= m ? 3u : n2 >= m ? 2u : n1 >= m ? 1u : 0u;
+            T |= d << bit;
+            cnt = d == 3u ? n3 : d == 2u ? n2 : d == 1u ? n1 : cnt;
         }
-        int need = m - (T == 0x7fffffffu ? 0 : count_ge<NG>(mag, ch0, T + 1u));   // equal to T, still to keep
+        // with cnt > m, T is the m-th largest magnitude itself and ties at T
+        // go to the lower channel indices
+        const bool exact = cnt == m;
+        int need = exact ? 0 : m - (T == 0x7fffffffu ? 0 : count_ge<NG>(mag, ch0, T + 1u));
         uint32_t kmask[NG];
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-            const bool eq = mag[g] == T && !(g == 0 && ch0) && m > 0;
+            const bool eq = !exact && mag[g] == T && !(g == 0 && ch0) && m > 0;
             const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
             const int rank = __popc(eqm & ((1u << lane) - 1u));   // equal channels of lower index in this group
-            const bool keep = (mag[g] > T && !(g == 0 && ch0) && m > 0) || (eq && rank < need);
+            const bool above = exact ? mag[g] >= T : mag[g] > T;
+            const bool keep = (above && !(g == 0 && ch0) && m > 0) || (eq && rank < need);
             kmask[g] = __ballot_sync(0xffffffffu, keep);
             need -= __popc(eqm);
         }
@@ -260,8 +285,7 @@ __device__ void qprep_kv(const float *__restrict__ t_q, const void *__restrict__
                 if ((shb >> 23) != 0u && (tgb >> 23) != 0u) {
                     e = (int)(shb >> 23) - (int)(tgb >> 23) - ((shb & 0x7fffffu) < (tgb & 0x7fffffu) ? 1 : 0);
                 } else {
-                    e = ilogbf(sh) - ilogbf(tg);
-                    if (ldexpf(sh, -e) < tg) --e;
+                    e = exp_offset_rare(sh, tg);
                 }
             }
             int q1 = 0, q2 = 0;
@@ -272,7 +296,7 @@ __device__ void qprep_kv(const float *__restrict__ t_q, const void *__restrict__
             }
             // p_g = 2^(-e - 2g), a normal number unless the query is degenerate
             const int pe = 127 - e - 2 * g;
-            sig[g] = pe >= 1 ? __uint_as_float((uint32_t)pe << 23) : ldexpf(1.0f, -e - 2 * g);
+            sig[g] = pe >= 1 ? __uint_as_float((uint32_t)pe << 23) : ldexp_rare(1.0f, -e - 2 * g);
             const int c = lane + 32 * g;
             q8[(h * 2 + 0) * D + c] = (signed char)q1;
             q8[(h * 2 + 1) * D + c] = (signed char)q2;
