@@ -102,15 +102,27 @@ __device__ void append_kv(const DecodeParams &dp, int b, int j, int t, unsigned 
     double *xs = reinterpret_cast<double *>(scratch + (size_t)D * pad_row_bytes<D>());   // [D][kFuseMaxNew]
     RowStoreScratch<D, NS, 1> &S = *reinterpret_cast<RowStoreScratch<D, NS, 1> *>(xs + kFuseMaxNew * D);
     named_bar_sync(kBarConsumers, nthreads);   // the previous task is done with the scratch
-    stage_rows<D, NTH>(scratch, dp.t_k + (size_t)j * D * D, t);
+    // T_K[j] and the key rows: every load in flight before the first store
+    RowStage<D, NTH> rows;
+    rows.load(dp.t_k + (size_t)j * D * D, t);
     int row0 = 0;   // rows of sequences 0..b-1 come first
     for (int bb = lane; bb < b; bb += 32) row0 += dp.new_lens[bb];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) row0 += __shfl_xor_sync(0xffffffffu, row0, o);
-    for (int i = t; i < kFuseMaxNew * D; i += nthreads) {
-        const int r = i / D, c = i - r * D;
-        xs[c * kFuseMaxNew + r] =
-            r < n ? (double)load_elem(dp.k_in, dp.kv_dtype, (((size_t)row0 + r) * p.hkv + j) * D + c) : 0.0;
+    constexpr int XN = (kFuseMaxNew * D + NTH - 1) / NTH;
+    float xv[XN];
+#pragma unroll
+    for (int k = 0; k < XN; ++k) {
+        const int i = t + k * NTH, r = i / D, c = i - r * D;
+        xv[k] = (i < kFuseMaxNew * D && r < n)
+                    ? load_elem_vol(dp.k_in, dp.kv_dtype, (((size_t)row0 + r) * p.hkv + j) * D + c)
+                    : 0.0f;
+    }
+    rows.store(scratch, t);
+#pragma unroll
+    for (int k = 0; k < XN; ++k) {
+        const int i = t + k * NTH, r = i / D, c = i - r * D;
+        if (i < kFuseMaxNew * D) xs[c * kFuseMaxNew + r] = (double)xv[k];
     }
     named_bar_sync(kBarConsumers, nthreads);
     if (t >= D) {

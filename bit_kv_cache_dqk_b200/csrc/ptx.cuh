@@ -80,6 +80,18 @@ __device__ __forceinline__ float4 ld_nc_f4(const float4 *ptr) {
     return v;
 }
 
+// Scalar global loads as asm statements (issued where they stand, see above).
+__device__ __forceinline__ float ld_f32_vol(const float *ptr) {
+    float v;
+    asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(ptr));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_u16_vol(const uint16_t *ptr) {
+    uint16_t v;
+    asm volatile("ld.global.u16 %0, [%1];" : "=h"(v) : "l"(ptr));
+    return v;
+}
+
 // Non-binding prefetch of one global line into L2 (address translation
 // included); no data is returned.
 __device__ __forceinline__ void prefetch_l2(const void *ptr) {

@@ -45,38 +45,51 @@ __device__ __forceinline__ uint16_t f16_piece(float x, int piece) {
     return __half_as_ushort(__float2half_rn(x - __half2float(hi)));
 }
 
-// A [D][D] fp32 transform staged in shared memory by the nthreads threads of
-// the caller (NTH of them, a compile-time count), with coalesced 16-byte
-// loads -- a warp reads 512 contiguous bytes, all of a thread's loads are in
-// flight before its first store -- into rows padded to D*4 + 16 bytes, so that
-// one thread per row then reads 16-byte chunks without bank conflicts (eight
+// A [D][D] fp32 transform staged in shared memory by the NTH threads of the
+// caller, with coalesced 16-byte loads -- a warp reads 512 contiguous bytes,
+// and all of a thread's loads (and the caller's next ones) are in flight
+// before its first store -- into rows padded to D*4 + 16 bytes, so that one
+// thread per row then reads 16-byte chunks without bank conflicts (eight
 // consecutive rows cover the 32 banks).
 template <int D>
 __host__ __device__ constexpr int pad_row_bytes() { return D * 4 + 16; }
 
 template <int D, int NTH>
-__device__ __forceinline__ void stage_rows(unsigned char *dst, const float *__restrict__ src, int t) {
-    constexpr int Q = D / 4;                     // 16-byte chunks per row
-    constexpr int N = (D * Q + NTH - 1) / NTH;   // chunks per thread
-    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+struct RowStage {
+    static constexpr int Q = D / 4;                     // 16-byte chunks per row
+    static constexpr int N = (D * Q + NTH - 1) / NTH;   // chunks per thread
     float4 v[N];
+    // asm loads: issued here, in order, ahead of whatever the caller loads next
+    __device__ __forceinline__ void load(const float *__restrict__ src, int t) {
+        const float4 *s4 = reinterpret_cast<const float4 *>(src);
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-        const int q = t + i * NTH;
-        if (q < D * Q) v[i] = __ldg(s4 + q);
+        for (int i = 0; i < N; ++i) {
+            const int q = t + i * NTH;
+            if (q < D * Q) v[i] = ld_nc_f4(s4 + q);
+        }
     }
-    const uint32_t base = smem_addr(dst);
+    __device__ __forceinline__ void store(unsigned char *dst, int t) const {
+        const uint32_t base = smem_addr(dst);
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-        const int q = t + i * NTH;
-        if (q < D * Q) st_s128(base + (uint32_t)((q / Q) * pad_row_bytes<D>() + (q % Q) * 16), *reinterpret_cast<uint4 *>(&v[i]));
+        for (int i = 0; i < N; ++i) {
+            const int q = t + i * NTH;
+            if (q < D * Q)
+                st_s128(base + (uint32_t)((q / Q) * pad_row_bytes<D>() + (q % Q) * 16),
+                        *reinterpret_cast<const uint4 *>(&v[i]));
+        }
     }
+};
+
+// An input element (fp32 or BF16 storage) as an asm load.
+__device__ __forceinline__ float load_elem_vol(const void *p, int dtype, size_t idx) {
+    if (dtype == DQK_BF16) return __uint_as_float(ld_u16_vol(reinterpret_cast<const uint16_t *>(p) + idx) << 16);
+    return ld_f32_vol(reinterpret_cast<const float *>(p) + idx);
 }
 
 // Sum over i ascending of (double)T[row][i] * x[i * xs + n], one fused
 // multiply-add after the other for each of the NX vectors (fp32 x fp32
 // products are exact in fp64, so the result does not depend on contraction),
-// T staged by stage_rows.  x is i-major (row stride xs doubles), so the NX
+// T staged by RowStage.  x is i-major (row stride xs doubles), so the NX
 // values of a column come in 16-byte loads.  Eight 16-byte chunks of the row
 // per iteration.
 template <int D, int NX>
@@ -162,14 +175,22 @@ __device__ void qprep_kv(const float *__restrict__ t_q, const void *__restrict__
     signed char *q8 = reinterpret_cast<signed char *>(qin + (size_t)G * D);
     float *qpv = reinterpret_cast<float *>(scratch);   // [G][D] after the sums
 
-    // stage T_Q[j] and the G query rows
+    // stage T_Q[j] and the G query rows (query h, channel c -> qin[c][h]):
+    // every load in flight before the first store
     named_bar_sync(bar, nthreads);   // the previous task is done with the scratch
-    stage_rows<D, NTH>(scratch, t_q + (size_t)j * D * D, t);
+    RowStage<D, NTH> rows;
+    rows.load(t_q + (size_t)j * D * D, t);
+    constexpr int QN = (G * D + NTH - 1) / NTH;
     const size_t qbase = ((size_t)b * hq + (size_t)j * G) * D;
-    for (int i = t; i < G * D; i += nthreads) {   // query h, channel c -> qin[c][h]
-        const int h = i / D, c = i - h * D;
-        qin[c * G + h] = (double)((dtype == DQK_BF16) ? bf16_to_f32(reinterpret_cast<const uint16_t *>(q)[qbase + i])
-                                                      : reinterpret_cast<const float *>(q)[qbase + i]);
+    float qv[QN];
+#pragma unroll
+    for (int k = 0; k < QN; ++k)
+        if (t + k * NTH < G * D) qv[k] = load_elem_vol(q, dtype, qbase + t + k * NTH);
+    rows.store(scratch, t);
+#pragma unroll
+    for (int k = 0; k < QN; ++k) {
+        const int i = t + k * NTH;
+        if (i < G * D) qin[(i % D) * G + i / D] = (double)qv[k];
     }
     named_bar_sync(bar, nthreads);   // T_Q[j] and the query rows are in
     // the warps the task leaves idle run the caller's `meanwhile` work
