@@ -273,7 +273,8 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
         for (int nt = 0; nt < NT; ++nt) {
             a0[b][nt] = 0.0f;
             a1[b][nt] = 0.0f;
-            mma_f16_zero(cmin[b][nt], km0[b], km1[b], 0u, 0u, st.qmin[nt], 0u);
+            cmin[b][nt][0] = cmin[b][nt][1] = cmin[b][nt][2] = cmin[b][nt][3] = 0.0f;
+            mma_f16(cmin[b][nt], km0[b], km1[b], 0u, 0u, st.qmin[nt], 0u);
         }
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
@@ -310,8 +311,8 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                int dg[4];
-                mma_u8s8(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y, 0);
+                int dg[4] = {0, 0, 0, 0};
+                mma_u8s8_acc(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y);
                 // rows gid, gid + 8: 256 D1 + D2 (exact), one rounding to fp32
                 const float y0 = (float)(dg[0] * 256 + dg[1]), y1 = (float)(dg[2] * 256 + dg[3]);
                 a0[b][nt] = fmaf(sa * kq[nt], y0, a0[b][nt]);
