@@ -266,13 +266,14 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
         k0a[b] = __uint_as_float(k0w << 16);
         k0b[b] = __uint_as_float(k0w & 0xffff0000u);
     }
-    float a0[NB][NT], a1[NB][NT], cmin[NB][NT][4];
+    // acc.x: token gid, acc.y: token gid + 8 (one packed instruction for both)
+    float2 acc[NB][NT];
+    float cmin[NB][NT][4];
 #pragma unroll
     for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            a0[b][nt] = 0.0f;
-            a1[b][nt] = 0.0f;
+            acc[b][nt] = make_float2(0.0f, 0.0f);
             cmin[b][nt][0] = cmin[b][nt][1] = cmin[b][nt][2] = cmin[b][nt][3] = 0.0f;
             mma_f16(cmin[b][nt], km0[b], km1[b], 0u, 0u, st.qmin[nt], 0u);
         }
@@ -314,9 +315,8 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
                 int dg[4] = {0, 0, 0, 0};
                 mma_u8s8_acc(dg, A0, A1, A2, A3, qb[nt].x, qb[nt].y);
                 // rows gid, gid + 8: 256 D1 + D2 (exact), one rounding to fp32
-                const float y0 = (float)(dg[0] * 256 + dg[1]), y1 = (float)(dg[2] * 256 + dg[3]);
-                a0[b][nt] = fmaf(sa * kq[nt], y0, a0[b][nt]);
-                a1[b][nt] = fmaf(sbv * kq[nt], y1, a1[b][nt]);
+                const float2 y = make_float2((float)(dg[0] * 256 + dg[1]), (float)(dg[2] * 256 + dg[3]));
+                acc[b][nt] = fma2(mul2(make_float2(sa, sbv), make_float2(kq[nt], kq[nt])), y, acc[b][nt]);
             }
         }
     }
@@ -324,8 +324,11 @@ __device__ __forceinline__ void qk_scores(const uint32_t (&sb)[NB], int nv, cons
     for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            s0[b][nt] = fmaf(st.sgh[nt], a0[b][nt], fmaf(st.q0v[nt], k0a[b], cmin[b][nt][0]));
-            s1[b][nt] = fmaf(st.sgh[nt], a1[b][nt], fmaf(st.q0v[nt], k0b[b], cmin[b][nt][2]));
+            const float2 t = fma2(make_float2(st.q0v[nt], st.q0v[nt]), make_float2(k0a[b], k0b[b]),
+                                  make_float2(cmin[b][nt][0], cmin[b][nt][2]));
+            const float2 sv = fma2(make_float2(st.sgh[nt], st.sgh[nt]), acc[b][nt], t);
+            s0[b][nt] = sv.x;
+            s1[b][nt] = sv.y;
             if constexpr (MASKED) {
                 if (gid >= nv) s0[b][nt] = -INFINITY;
                 if (gid + 8 >= nv) s1[b][nt] = -INFINITY;
