@@ -343,17 +343,20 @@ __device__ __forceinline__ void max_update(WarpState<D, G> &st, const float (&s0
                                            const float (&s1)[NB][AttendTile<D, G>::NT]) {
     using T = AttendTile<D, G>;
     constexpr int NT = T::NT;
+    float mxs[NT];
     bool grow = false;
 #pragma unroll
-    for (int b = 0; b < NB; ++b)
+    for (int nt = 0; nt < NT; ++nt) {
+        float mx = fmaxf(s0[0][nt], s1[0][nt]);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) grow |= (s0[b][nt] > st.m_run[nt]) | (s1[b][nt] > st.m_run[nt]);
+        for (int b = 1; b < NB; ++b) mx = fmaxf(mx, fmaxf(s0[b][nt], s1[b][nt]));
+        mxs[nt] = mx;
+        grow |= mx > st.m_run[nt];
+    }
     if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float mx = fmaxf(s0[0][nt], s1[0][nt]);
-#pragma unroll
-            for (int b = 1; b < NB; ++b) mx = fmaxf(mx, fmaxf(s0[b][nt], s1[b][nt]));
+            float mx = mxs[nt];
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -435,7 +438,8 @@ __device__ __forceinline__ void pv_accum(const uint32_t (&sb)[NB], int nv, WarpS
         uint32_t pb0[NT], pb1[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const float p0 = fast_exp2(s0[b][nt] - st.m_run[nt]), p1 = fast_exp2(s1[b][nt] - st.m_run[nt]);
+            const float2 e = add2(make_float2(s0[b][nt], s1[b][nt]), make_float2(-st.m_run[nt], -st.m_run[nt]));
+            const float p0 = fast_exp2(e.x), p1 = fast_exp2(e.y);
             const uint32_t pp = pack_f16x2(p0, p1);   // lo: token gid, hi: token gid+8
             const uint32_t w0 = __shfl_sync(0xffffffffu, pp, o.srcA);
             const uint32_t w1 = __shfl_sync(0xffffffffu, pp, o.srcA + 4);

@@ -262,7 +262,7 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
 }
 
 // Packed fp32 pairs (two IEEE operations in one instruction, sm_100):
-// d = a * b + c and d = a * b lane by lane, each lane rounded as fmaf / __fmul_rn.
+// d = a * b + c, a + b and a * b lane by lane, each lane rounded as the scalar operation.
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
@@ -270,6 +270,15 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
         "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
