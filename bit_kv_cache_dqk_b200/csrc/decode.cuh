@@ -399,21 +399,6 @@ __global__ void __launch_bounds__(attend_threads(G), 1) k_decode(const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = p.batch * p.nchunks;
     const int pps = p.pps;
-    // The transforms this CTA's prologue tasks stage (task k runs on CTA k mod
-    // C): into L2 and the descriptor cache already, while the kernel before
-    // this one may still run (a prefetch returns no data).
-    if (threadIdx.x == 0) {
-        const int n_app = dp.max_new > 0 ? p.batch * p.hkv : 0;
-        const int n_tasks = n_app + p.batch * p.hkv;
-        if ((int)blockIdx.x < n_tasks) {
-            const uint64_t keep = l2_policy_evict_last();
-            for (int k = (int)blockIdx.x; k < n_tasks; k += (int)gridDim.x) {
-                const bool app = k < n_app;
-                const int j = (app ? k : k - n_app) % p.hkv;
-                bulk_prefetch_l2((app ? dp.t_k : dp.t_q) + (size_t)j * D * D, D * D * 4, keep);
-            }
-        }
-    }
     // launched with programmatic serialization: everything read below may come
     // from the kernel before this one on the stream
     grid_dependency_wait();

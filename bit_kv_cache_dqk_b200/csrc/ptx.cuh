@@ -92,19 +92,6 @@ __device__ __forceinline__ uint32_t ld_u16_vol(const uint16_t *ptr) {
     return v;
 }
 
-// Non-binding prefetch of one global line into L2 (address translation
-// included); no data is returned.
-__device__ __forceinline__ void prefetch_l2(const void *ptr) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-
-// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) of global
-// memory into L2 with a cache policy; no data is returned.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *ptr, uint32_t bytes, uint64_t policy) {
-    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(ptr), "r"(bytes), "l"(policy)
-                 : "memory");
-}
-
 // Named barrier `id` over `n` threads: arrive without waiting, or arrive and
 // wait.  (Barrier 0 is __syncthreads.)
 __device__ __forceinline__ void named_bar_arrive(int id, int n) {
@@ -251,16 +238,6 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// D = A * B + C, m16n8k32, u8 x s8 operands, s32 accumulate; C is the same
-// value c in all four elements (kept in registers, no per-use copies).
-__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1, int c) {
-    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c));
-}
-
 // Packed fp32 pairs (two IEEE operations in one instruction, sm_100):
 // d = a * b + c, a + b and a * b lane by lane, each lane rounded as the scalar operation.
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
@@ -300,33 +277,6 @@ __device__ __forceinline__ void mma_u8s8_acc(int (&d)[4], uint32_t a0, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// The same with the accumulator of even columns started at c_even and of odd
-// columns at c_odd.
-__device__ __forceinline__ void mma_u8s8_c2(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                            uint32_t b0, uint32_t b1, int c_even, int c_odd) {
-    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%11,%10,%11};"
-        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c_even), "r"(c_odd));
-}
-
-// D = A * B (zero accumulator), m16n8k16 fp16, fp32 result.
-__device__ __forceinline__ void mma_f16_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                             uint32_t b0, uint32_t b1) {
-    const float z = 0.0f;
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
-}
-
-// 1.5 * 2^23: an int32 accumulator started at its bit pattern (0x4B400000)
-// reads as the float kMagicF + sum, exactly, while |sum| < 2^22.
-constexpr int kMagicI = 0x4B400000;
-constexpr float kMagicF = 12582912.0f;
-// 1.5 * 2^15 (0x47400000): reads as kMagicLoF + sum / 256, exactly, while |sum| < 2^22.
-constexpr int kMagicLoI = 0x47400000;
-constexpr float kMagicLoF = 49152.0f;
 
 // Two 2-bit codes at bit 2P of each 16-bit half of x -> an f16x2 holding the
 // exact values 0..3.  OR-ing the field into the mantissa of 2^(10-2P) gives
