@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(512) k_quant_pack(
 // bytes, as k_quant_pack.
 // ---------------------------------------------------------------------------
 constexpr int kDirectMaxNew = 64;   // dqk_append uses k_append_rows up to this many rows per sequence
-constexpr int kRowsPerCta = 4;
+constexpr int kRowsPerCta = 8;
 
 template <int D, int NS, int RW>
 struct RowStoreScratch {
@@ -406,59 +406,79 @@ __device__ __forceinline__ void quantize_store_rows(const float (&kp)[RW], const
 }
 
 // One CTA of D threads per (group of RW consecutive new rows of a sequence,
-// kv head) -- RW = 1 when every sequence appends one row, else kRowsPerCta;
-// thread c reads T_K's row c straight from global memory (the loads issued
-// before any is used).
+// kv head) -- RW = 1 when every sequence appends one row, else kRowsPerCta.
+// T_K[j] is staged in shared memory by coalesced 16-byte asynchronous copies
+// into rows padded by 16 bytes, so thread c then reads its row c without bank
+// conflicts; thread c forms k'_c of every row of the group (fp64 sequential
+// sums, the rows i-major in shared memory), then quantize_store_rows.
+template <int D, int NS, int RW>
+__host__ __device__ constexpr size_t append_rows_smem() {
+    return (size_t)D * (D * 4 + 16) + (size_t)RW * D * 8 + sizeof(RowStoreScratch<D, NS, RW>);
+}
+
 template <int D, int NS, int RW>
 __global__ void __launch_bounds__(D) k_append_rows(
     const float *__restrict__ t_k, const void *__restrict__ kin, const void *__restrict__ vin, int dtype,
     const int *__restrict__ new_lens, const int *__restrict__ seq_before, const int *__restrict__ page_table,
     int max_pages, int groups_per_seq, uint8_t *__restrict__ pool, long long num_pages, int hkv, int v_ch0,
     int early_release) {
-    __shared__ double xs[RW][D];
-    __shared__ RowStoreScratch<D, NS, RW> S;
+    constexpr int kPad = D * 4 + 16;   // bytes per staged row of T_K
+    extern __shared__ __align__(16) unsigned char append_rows_mem[];
+    unsigned char *sT = append_rows_mem;
+    double *xs = reinterpret_cast<double *>(append_rows_mem + (size_t)D * kPad);   // [D][RW], i-major
+    RowStoreScratch<D, NS, RW> &S = *reinterpret_cast<RowStoreScratch<D, NS, RW> *>(xs + (size_t)RW * D);
     const int j = blockIdx.y;
     const int b = blockIdx.x / groups_per_seq, t0 = (blockIdx.x - b * groups_per_seq) * RW;
     const int c = threadIdx.x, lane = c & 31;
     if (early_release) grid_dependents_launch();
-    // every load that depends only on (sequence, kv head, channel) is issued
-    // before the first one is used: the lengths, the row offset of the
-    // sequence and T_K's row c
     const int n = new_lens[b];
+    if (t0 >= n) return;   // the whole CTA
+    // T_K[j]: D rows of D / 4 chunks, a warp copies 32 consecutive chunks
+    {
+        const float *tj = t_k + (size_t)j * D * D;
+        const uint32_t base = smem_addr(sT);
+#pragma unroll 4
+        for (int q = c; q < D * D / 4; q += D)
+            cp_async16(base + (uint32_t)((q / (D / 4)) * kPad + (q % (D / 4)) * 16), tj + 4 * q);
+    }
     const int L0 = seq_before[b];
-    int row0 = 0;                             // rows of sequences 0..b-1 come first
+    int row0 = 0;   // rows of sequences 0..b-1 come first
     for (int bb = lane; bb < b; bb += 32) row0 += new_lens[bb];
-    const float4 *tr = reinterpret_cast<const float4 *>(t_k + ((size_t)j * D + c) * D);
-    float4 tv[D / 4];
-#pragma unroll
-    for (int u = 0; u < D / 4; ++u) tv[u] = ld_nc_f4(tr + u);
-    if (t0 >= n) return;                      // the whole CTA
-    const int nr = min(RW, n - t0);           // rows of this CTA
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) row0 += __shfl_xor_sync(0xffffffffu, row0, o);
+    const int nr = min(RW, n - t0);   // rows of this CTA
     float xv[RW];
     int phys[RW];
 #pragma unroll
     for (int i = 0; i < RW; ++i) {
         const int t = t0 + (i < nr ? i : 0);
         const size_t base = (((size_t)row0 + t) * hkv + j) * D;
-        xs[i][c] = (double)load_elem(kin, dtype, base + c);
+        xs[c * RW + i] = (double)load_elem(kin, dtype, base + c);
         xv[i] = load_elem(vin, dtype, base + c);
         const int page = (L0 + t) / kPage;
         phys[i] = (L0 >= 0 && page < max_pages) ? page_table[(size_t)b * max_pages + page] : -1;
     }
+    cp_async_wait_all();
     __syncthreads();
     // k'_c = sum_i T_K[c][i] x_i, ascending i, exact products summed in fp64
     double acc[RW];
+    {
 #pragma unroll
-    for (int i = 0; i < RW; ++i) acc[i] = 0.0;
+        for (int i = 0; i < RW; ++i) acc[i] = 0.0;
+        const unsigned char *row = sT + (size_t)c * kPad;
+#pragma unroll 1
+        for (int k = 0; k < D / 32; ++k) {
 #pragma unroll
-    for (int u = 0; u < D / 4; ++u) {
-        const double t4[4] = {(double)tv[u].x, (double)tv[u].y, (double)tv[u].z, (double)tv[u].w};
+            for (int u = 0; u < 8; ++u) {
+                const float4 tv = *reinterpret_cast<const float4 *>(row + (32 * k + 4 * u) * 4);
+                const double t4[4] = {(double)tv.x, (double)tv.y, (double)tv.z, (double)tv.w};
+                const double *xi = xs + (32 * k + 4 * u) * RW;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
+                for (int e = 0; e < 4; ++e)
 #pragma unroll
-            for (int i = 0; i < RW; ++i) acc[i] = fma(t4[e], xs[i][4 * u + e], acc[i]);
+                    for (int i = 0; i < RW; ++i) acc[i] = fma(t4[e], xi[e * RW + i], acc[i]);
+            }
+        }
     }
     float kp[RW];
 #pragma unroll

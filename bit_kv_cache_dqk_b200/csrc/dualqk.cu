@@ -326,14 +326,17 @@ dqk_status run_append(const dqk_layer_desc *L, const void *k, const void *v, dqk
     const int dev = current_device();
     if (max_new <= kDirectMaxNew) {
         // one row per sequence: one row per CTA, no idle row slots
-        if (max_new == 1) prefer_max_shared<k_append_rows<D, NS, 1>>(dev);
-        else prefer_max_shared<k_append_rows<D, NS, kRowsPerCta>>(dev);
-        auto kernel = max_new == 1 ? k_append_rows<D, NS, 1> : k_append_rows<D, NS, kRowsPerCta>;
-        const int rw = max_new == 1 ? 1 : kRowsPerCta;
+        const bool one_row = max_new == 1;
+        const size_t smem = one_row ? append_rows_smem<D, NS, 1>() : append_rows_smem<D, NS, kRowsPerCta>();
+        const dqk_status st = one_row ? prepare_kernel<k_append_rows<D, NS, 1>>(dev, smem, D)
+                                      : prepare_kernel<k_append_rows<D, NS, kRowsPerCta>>(dev, smem, D);
+        if (st != DQK_OK) return st;
+        auto kernel = one_row ? k_append_rows<D, NS, 1> : k_append_rows<D, NS, kRowsPerCta>;
+        const int rw = one_row ? 1 : kRowsPerCta;
         const int groups = (max_new + rw - 1) / rw;
         const long long gx = (long long)batch * groups;
         if (gx > 0x7fffffffLL) return DQK_ERR_UNSUPPORTED;
-        kernel<<<dim3((unsigned)gx, L->num_kv_heads), D, 0, stream>>>(
+        kernel<<<dim3((unsigned)gx, L->num_kv_heads), D, smem, stream>>>(
             L->t_k, k, v, dtype, new_lens, seq_before, page_table, max_pages, groups,
             static_cast<uint8_t *>(L->pool), L->num_pages, L->num_kv_heads, L->v_ch0_protect, 0);
         return launch_status();
@@ -373,6 +376,7 @@ dqk_status check_append(const dqk_layer_desc *layer, const void *k, const void *
     dqk_status st = check_layer(layer);
     if (st != DQK_OK) return st;
     if (!layer->t_k || !k || !v || !new_lens || !seq_lens_before || !page_table) return DQK_ERR_INVALID_ARG;
+    if (!aligned(layer->t_k, 16)) return DQK_ERR_INVALID_ARG;
     if (dtype != DQK_F32 && dtype != DQK_BF16) return DQK_ERR_INVALID_ARG;
     if (batch <= 0 || max_pages <= 0 || max_new < 0) return DQK_ERR_INVALID_ARG;
     if (!aligned(k, 4) || !aligned(v, 4)) return DQK_ERR_INVALID_ARG;

@@ -80,6 +80,12 @@ __device__ __forceinline__ float4 ld_nc_f4(const float4 *ptr) {
     return v;
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only; both addresses 16-byte
+// aligned); cp_async_wait_all below waits for it.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
 // Scalar global loads as asm statements (issued where they stand, see above).
 __device__ __forceinline__ float ld_f32_vol(const float *ptr) {
     float v;

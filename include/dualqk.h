@@ -70,7 +70,8 @@ typedef enum { DQK_F32 = 0, DQK_BF16 = 1 } dqk_dtype;
  *  v_ch0_protect  0: value channel 0 quantized like the others (default);
  *                 1: value channel 0 kept in BF16 as well.
  *  t_k, t_q       (device) fp32 [Hkv][d][d] row-major: k' = T_K k,
- *                 q' = T_Q q.  The caller supplies T_Q = T_K^{-T}.
+ *                 q' = T_Q q.  The caller supplies T_Q = T_K^{-T}.  16-byte
+ *                 aligned (DQK_ERR_INVALID_ARG otherwise).
  *  pool           (device) the paged cache: num_pages * Hkv blocks of
  *                 dqk_block_bytes() bytes, block (page p, kv head j) at byte
  *                 offset (p * Hkv + j) * dqk_block_bytes().  16-byte aligned.
