@@ -45,11 +45,13 @@
 
 namespace dqk {
 
-// CTA shape of k_attend: 8 consumer warps, each owning one kv head of a chunk
-// of 8 and taking attend_pages_per_warp pages of it per stage (processed as
-// independent instruction streams), plus one producer warp.  Four pages per
-// warp where the per-warp state allows (G <= 4), two for G = 8, whose two
-// query-head tiles double that state.
+// CTA shape of the decode kernel's streaming loop: consumer warps, each owning
+// one kv head of a chunk and taking attend_pages_per_warp pages of it per
+// stage (processed as independent instruction streams), plus one producer
+// warp.  Twelve consumer warps taking four pages each where the per-warp state
+// allows (G <= 4; thirteen warps keep 128 registers a thread, since the
+// register file is split between the four schedulers), eight taking two for
+// G = 8, whose two query-head tiles double that state.
 __host__ __device__ constexpr int attend_warps(int G) { return G > 4 ? 8 : 12; }
 __host__ __device__ constexpr int attend_pages_per_warp(int G) { return G > 4 ? 2 : 4; }
 __host__ __device__ constexpr int attend_stage_blocks(int G) { return attend_pages_per_warp(G) * attend_warps(G); }

@@ -1,8 +1,9 @@
 // bf16.cuh -- the BF16 comparison decode: a paged BF16 K/V cache with no
 // transform, no quantization and no channel pruning, the baseline Dual-QK's
 // decode speedup is measured against ("Throughput on SGLang": the 3.75x over
-// BF16 attention).  Same work split, producer warp, records and LSE combine as
-// k_attend; the consumers are plain bf16 tensor-core flash decoding.
+// BF16 attention).  Same cooperative launch, work split, producer warp,
+// records and log-sum-exp merge as k_decode, without its prologue; the
+// consumers are plain bf16 tensor-core flash decoding.
 //
 // Block of (page, kv head): K [16][d] then V [16][d], BF16, row-major per
 // token, with the 16-byte chunk x of row t stored at chunk position x ^ (t & 7)
