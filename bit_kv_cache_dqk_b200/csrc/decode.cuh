@@ -31,9 +31,8 @@
 
 namespace dqk {
 
-// Everything a decode launch needs besides the streaming parameters.  The
-// kernels take it as a __grid_constant__ parameter: the tensor maps of the
-// transforms are read from parameter space by the bulk tensor copies.
+// Everything a decode launch needs besides the streaming parameters, passed
+// as one __grid_constant__ kernel parameter.
 struct DecodeParams {
     AttendParams a;
     uint8_t *pool_w;             // the pool, for the step's appends
