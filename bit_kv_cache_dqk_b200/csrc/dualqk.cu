@@ -61,6 +61,19 @@ struct DecodePlan {
 
 constexpr int kMaxAttendCtas = 160;   // >= the 148 SMs of a B200; larger parts run 160 persistent CTAs
 
+// CTAs of a decode launch: one per SM, but no more than give every CTA about
+// three stages of pages when every sequence fills its max_pages: a small
+// problem spread over every SM leaves each CTA a stage or less, and each query
+// head then has records from dozens of CTAs to merge (several rounds of
+// record loads), where a few dozen CTAs stream the same bytes about as fast.
+int decode_ctas(int sms, int batch, int nchunks, int max_pages, int pps) {
+    const long long units = (long long)batch * nchunks * max_pages;
+    const long long per = 3LL * (pps > 0 ? pps : 1);
+    const long long want = std::max<long long>(1, (units + per - 1) / per);
+    return (int)std::min<long long>(std::min(sms, kMaxAttendCtas), want);
+}
+
+
 size_t records_bytes(size_t runs, int pw, int hc, int G, int d) {
     return ((size_t)kMaxAttendCtas + runs - 1) * pw * hc * G * rec_stride(d) * sizeof(float);
 }
@@ -237,7 +250,7 @@ dqk_status check_decode(const DecodeArgs &a, DecodePlan &P, int &dev) {
     if (a.ws_bytes < P.bytes) return DQK_ERR_WORKSPACE_TOO_SMALL;
     dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return DQK_ERR_CUDA;
-    P.num_ctas = std::min(device_sms(dev), kMaxAttendCtas);
+    P.num_ctas = decode_ctas(device_sms(dev), a.batch, P.nchunks, a.max_pages, P.pps);
     if (P.num_ctas <= 0) return DQK_ERR_CUDA;
     return DQK_OK;
 }
@@ -713,7 +726,7 @@ dqk_status dqk_bf16_decode(const dqk_layer_desc *layer, const void *q, dqk_dtype
     if (workspace_bytes < P.bytes) return DQK_ERR_WORKSPACE_TOO_SMALL;
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return DQK_ERR_CUDA;
-    P.num_ctas = std::min(device_sms(dev), kMaxAttendCtas);
+    P.num_ctas = decode_ctas(device_sms(dev), batch, P.nchunks, max_pages, P.pps);
     if (P.num_ctas <= 0) return DQK_ERR_CUDA;
     DecodeArgs a{layer, q, q_dtype, batch, seq_lens, page_table, max_pages, 0, out, nullptr,
                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};
