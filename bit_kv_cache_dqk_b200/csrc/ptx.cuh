@@ -81,7 +81,7 @@ __device__ __forceinline__ float4 ld_nc_f4(const float4 *ptr) {
 }
 
 // 16-byte asynchronous copy global -> shared (L2 only; both addresses 16-byte
-// aligned); cp_async_wait_all below waits for it.
+// aligned); cp_async_wait_all waits for it.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -116,14 +116,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return pol;
 }
 
-// L2 policy for small tensors every launch re-reads (the transforms): kept
-// in L2 ahead of the streamed pages.
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
 // 1-D bulk copy global -> shared, completion counted on `bar` (no multicast).
 __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -142,12 +134,7 @@ __device__ __forceinline__ void bulk_copy_g2s_hint(void *dst, const void *src, u
         : "memory");
 }
 
-
-// 4-byte asynchronous global -> shared copy (no register round trip), and the
-// wait for all of this thread's outstanding copies.
-__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
-}
+// Wait for all of this thread's cp.async copies in flight.
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
@@ -347,11 +334,6 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
     return r;
 }
 
-__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t v) {
-    __half2 h = *reinterpret_cast<__half2 *>(&v);
-    return __half22float2(h);
-}
-
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -365,13 +347,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return r;
 }
 
-// Non-negative fp16 values of an f16x2 word as fp32 numbers scaled by 2^-112:
-// the 15 value bits moved to bit 13 are a binary32 pattern whose exponent bias
-// differs by 127 - 15 = 112 (subnormal fp16 lands on subnormal fp32, so the
-// scaling is exact for every non-negative fp16).  Integer ops only.
-__device__ __forceinline__ float f16lo_scaled(uint32_t w) { return __uint_as_float((w << 13) & 0x0fffe000u); }
-__device__ __forceinline__ float f16hi_scaled(uint32_t w) { return __uint_as_float((w >> 3) & 0x0fffe000u); }
-constexpr float kTwoPow112 = 0x1p112f;
 // fp16 halves of a word as fp32 (exact; one conversion each)
 __device__ __forceinline__ float f16lo_to_f32(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
 __device__ __forceinline__ float f16hi_to_f32(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
@@ -423,8 +398,5 @@ __device__ __forceinline__ void mbar_arrive_if(uint64_t *bar, bool pred) {
         : "memory");
 }
 
-__device__ __forceinline__ uint4 lds128(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
-__device__ __forceinline__ uint2 lds64(const void *p) { return *reinterpret_cast<const uint2 *>(p); }
-__device__ __forceinline__ uint32_t lds32(const void *p) { return *reinterpret_cast<const uint32_t *>(p); }
 
 }  // namespace dqk
