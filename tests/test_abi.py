@@ -94,6 +94,18 @@ def test_invalid_arguments_rejected_on_host(Q):
     assert st == Q.DQK_ERR_UNSUPPORTED
 
 
+def test_misaligned_transforms_rejected_on_host(Q):
+    """The kernels read T_K and T_Q with 16-byte copies: a transform that is not
+    16-byte aligned is refused before anything is launched."""
+    desc = Q.layer_desc(128, 32, 8, 260, 256, 256, 10)   # T_K 4 bytes off
+    st = Q.dqk_append(desc, 256, 256, Q.DQK_BF16, 1, 256, 256, 1, 256, 1, stream=0, raise_on_error=False)
+    assert st == Q.DQK_ERR_INVALID_ARG
+    desc = Q.layer_desc(128, 32, 8, 256, 264, 256, 10)   # T_Q 8 bytes off
+    st = Q.dqk_decode(desc, 256, Q.DQK_BF16, 1, 256, 256, 4, 40, 256, None, 256, 1 << 30, stream=0,
+                      raise_on_error=False)
+    assert st == Q.DQK_ERR_INVALID_ARG
+
+
 def test_status_strings(Q):
     assert Q.dqk_status_string(Q.DQK_OK) == "DQK_OK"
     assert Q.dqk_status_string(Q.DQK_ERR_TIMEOUT) == "DQK_ERR_TIMEOUT"
